@@ -1,0 +1,372 @@
+"""Pins that tie the CPU oracle to something other than itself.
+
+Each check returns a list of failure messages (empty = pass), so the same checks
+serve the plain pin tests and the planted-mistake tests, which build deliberately
+broken copies of the oracle and require at least one check to fail.
+
+What pins what:
+  golden_*          worked examples derived by hand (tests/golden/hand_derived.json)
+  brute_codes       every code is the integer nearest to the IEEE binary32 quotient
+                    x'/s, found by exhaustive search with ties to even, then clamped;
+                    every scale is within two roundings of the exact alpha*amax/qmax
+  gemm_vs_matmul    int32 accumulators equal numpy's int64 matmul of codes unpacked
+                    here with a different bit trick
+  epilogue_fp64     each bf16 output is the bf16 value nearest to the fp64 result
+  textbook          cinv=1, alpha=1, beta=0 reduces to plain per-token /
+                    per-output-channel symmetric quantized GEMM
+  on_grid           inputs already on the quantization grid round-trip exactly and
+                    the output equals the fp64 product of the dequantized operands
+  requant           re-quantizing dequantized codes returns the same codes
+  scale_invariance  doubling a row doubles its scale and keeps its codes
+"""
+import numpy as np
+
+from activation_quantized_gemm_wq_b200.synth import f32_to_bf16_bits
+
+
+def f32_bits(a):
+    return np.asarray(a, np.float32).view(np.uint32)
+
+
+def bf16_from_values(v):
+    """Exact bf16 patterns of values that bf16 represents exactly."""
+    b = np.asarray(v, np.float32).view(np.uint32)
+    assert np.all((b & 0xFFFF) == 0), "golden value not exactly representable in bf16"
+    return (b >> 16).astype(np.uint16)
+
+
+def bf16_to_f32(bits):
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def unpack_nibbles(packed):
+    """Two's-complement nibbles, low nibble first: ((v & 0xF) ^ 8) - 8."""
+    p = np.asarray(packed, np.uint8).astype(np.int16)
+    lo = ((p & 0xF) ^ 8) - 8
+    hi = (((p >> 4) & 0xF) ^ 8) - 8
+    out = np.empty(p.shape[:-1] + (p.shape[-1] * 2,), np.int16)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
+
+
+def nearest_code_bruteforce(t, qmax):
+    """Integer in [-qmax, qmax] nearest to each float64 t, ties to the even one;
+    |t| beyond the range saturates.  Exhaustive over the candidates."""
+    t = np.asarray(t, np.float64)
+    cand = np.arange(-qmax, qmax + 1, dtype=np.float64)
+    d = np.abs(t[..., None] - cand)
+    best = d.min(axis=-1, keepdims=True)
+    hit = d == best
+    even = (np.abs(cand) % 2 == 0)
+    pick_even = hit & even
+    idx = np.where(pick_even.any(-1), pick_even.argmax(-1), hit.argmax(-1))
+    return cand[idx].astype(np.int64)
+
+
+# ----------------------------------------------------------------- golden cases
+
+def golden_act_quant(orc, golden):
+    fails = []
+    for case in golden["act_quant"]:
+        x = bf16_from_values(case["x"])
+        cinv = None if case["cinv"] is None else np.asarray(case["cinv"], np.float32)
+        qx, s = orc.act_quant(x, cinv, np.asarray(case["stream_id"], np.uint8),
+                              np.asarray(case["alpha"], np.float32), case["step"], case["act_bits"])
+        codes = unpack_nibbles(qx) if case["act_bits"] == 4 else qx.astype(np.int16)
+        if not np.array_equal(codes, np.asarray(case["codes"])):
+            fails.append(f"act_quant/{case['name']}: codes {codes.tolist()} != {case['codes']}")
+        if "packed" in case and not np.array_equal(qx, np.asarray(case["packed"], np.uint8)):
+            fails.append(f"act_quant/{case['name']}: packed {qx.tolist()} != {case['packed']}")
+        if not np.array_equal(f32_bits(s), f32_bits(case["s_tok"])):
+            fails.append(f"act_quant/{case['name']}: s_tok {s.tolist()} != {case['s_tok']}")
+    return fails
+
+
+def golden_pack(orc, golden):
+    fails = []
+    for case in golden["pack_int4"]:
+        W = bf16_from_values(case["W"])
+        c = None if case["c"] is None else np.asarray(case["c"], np.float32)
+        qw, s_w = orc.pack_int4(W, c)
+        if not np.array_equal(qw, np.asarray(case["packed"], np.uint8)):
+            fails.append(f"pack/{case['name']}: packed {qw.tolist()} != {case['packed']}")
+        if not np.array_equal(unpack_nibbles(qw), np.asarray(case["codes"])):
+            fails.append(f"pack/{case['name']}: codes differ")
+        if not np.array_equal(f32_bits(s_w), f32_bits(case["s_w"])):
+            fails.append(f"pack/{case['name']}: s_w {s_w.tolist()} != {case['s_w']}")
+    return fails
+
+
+def golden_channel_scale(orc, golden):
+    fails = []
+    for case in golden["channel_scale"]:
+        c, cinv = orc.channel_scale(bf16_from_values(case["x_cal"]), bf16_from_values(case["W"]))
+        if f32_bits(c).tolist() != case["c_bits"]:
+            fails.append(f"channel_scale/{case['name']}: c bits {f32_bits(c).tolist()}")
+        if f32_bits(cinv).tolist() != case["cinv_bits"]:
+            fails.append(f"channel_scale/{case['name']}: cinv bits {f32_bits(cinv).tolist()}")
+    return fails
+
+
+def golden_linear(orc, golden):
+    fails = []
+    for case in golden["linear"]:
+        x = bf16_from_values(case["x"])
+        y, qx, s_tok, acc = orc.linear(
+            x, np.asarray(case["cinv"], np.float32), np.asarray(case["stream_id"], np.uint8),
+            np.asarray(case["alpha"], np.float32), np.asarray(case["beta"], np.float32),
+            case["step"], case["act_bits"], np.asarray(case["qw_packed"], np.uint8),
+            np.asarray(case["s_w"], np.float32), np.asarray(case["bias"], np.float32))
+        if not np.array_equal(qx.astype(np.int16), np.asarray(case["codes"])):
+            fails.append(f"linear/{case['name']}: codes {qx.tolist()}")
+        if not np.array_equal(f32_bits(s_tok), f32_bits(case["s_tok"])):
+            fails.append(f"linear/{case['name']}: s_tok {s_tok.tolist()}")
+        if not np.array_equal(acc, np.asarray(case["acc"])):
+            fails.append(f"linear/{case['name']}: acc {acc.tolist()}")
+        if not np.array_equal(y, bf16_from_values(case["y"])):
+            fails.append(f"linear/{case['name']}: y {bf16_to_f32(y).tolist()} != {case['y']}")
+    return fails
+
+
+def golden_bf16_rounding(orc, golden):
+    g = golden["bf16_rounding"]
+    got = [int(orc.lib.oracle_double_to_bf16(v)) for v in g["values"]]
+    return [] if got == g["bits"] else [f"bf16 rounding {got} != {g['bits']}"]
+
+
+# --------------------------------------------------------------- random tiny data
+
+def _tiny_inputs(seed, M=48, K=64, N=40, T=3, S=3):
+    g = np.random.default_rng(seed)
+    x = f32_to_bf16_bits((g.standard_normal((M, K)) * g.uniform(0.2, 5.0, (M, 1))).astype(np.float32))
+    x[3, :] = 0  # a zero row
+    cinv = g.uniform(0.3, 3.0, K).astype(np.float32)
+    sid = g.integers(0, S, M).astype(np.uint8)
+    alpha = g.uniform(0.6, 1.1, (T, S)).astype(np.float32)
+    beta = g.normal(0, 1e-2, (T, S, N)).astype(np.float32)
+    W = f32_to_bf16_bits(g.normal(0, 0.05, (N, K)).astype(np.float32))
+    bias = g.normal(0, 0.05, N).astype(np.float32)
+    c = g.uniform(0.5, 2.0, K).astype(np.float32)
+    return x, cinv, sid, alpha, beta, W, bias, c
+
+
+def brute_codes(orc, seeds=(1, 2, 3)):
+    fails = []
+    for seed in seeds:
+        x, cinv, sid, alpha, _, W, _, c = _tiny_inputs(seed)
+        for bits, qmax in ((8, 127), (4, 7)):
+            for step in (0, 2):
+                qx, s = orc.act_quant(x, cinv, sid, alpha, step, bits)
+                codes = unpack_nibbles(qx) if bits == 4 else qx.astype(np.int64)
+                xp = bf16_to_f32(x) * cinv[None, :]            # binary32 products
+                amax = np.abs(xp).max(axis=1).astype(np.float64)
+                exact = alpha[step, sid].astype(np.float64) * amax / qmax
+                rel = np.abs(s.astype(np.float64) - exact) / np.maximum(exact, 1e-300)
+                if np.any((exact > 0) & (rel > 2.5 * 2.0 ** -24)) or np.any((exact == 0) & (s != 0)):
+                    fails.append(f"brute_codes seed {seed} bits {bits}: scale off by {rel.max():.3g}")
+                with np.errstate(divide="ignore", invalid="ignore"):
+                    t = (xp / s[:, None]).astype(np.float64)          # binary32 quotient
+                want = nearest_code_bruteforce(np.where(s[:, None] > 0, t, 0.0), qmax)
+                if not np.array_equal(codes, want):
+                    bad = np.argwhere(codes != want)[0]
+                    fails.append(f"brute_codes seed {seed} bits {bits} step {step}: code at "
+                                 f"{tuple(bad)} is {codes[tuple(bad)]}, search gives {want[tuple(bad)]}")
+        qw, s_w = orc.pack_int4(W, c)
+        wp = bf16_to_f32(W) * c[None, :]
+        exact = np.abs(wp).max(axis=1).astype(np.float64) / 7.0
+        if np.any(np.abs(s_w - exact) > 1.5 * 2.0 ** -24 * exact):
+            fails.append(f"brute_codes seed {seed}: weight scale off")
+        t = (wp / s_w[:, None]).astype(np.float64)
+        if not np.array_equal(unpack_nibbles(qw), nearest_code_bruteforce(t, 7)):
+            fails.append(f"brute_codes seed {seed}: weight codes differ from search")
+    return fails
+
+
+def gemm_vs_matmul(orc, seeds=(4, 5)):
+    fails = []
+    for seed in seeds:
+        g = np.random.default_rng(seed)
+        M, N, K = 17, 23, 96
+        qw = g.integers(0, 256, (N, K // 2), dtype=np.uint8)
+        w = unpack_nibbles(qw).astype(np.int64)
+        for bits in (8, 4):
+            if bits == 8:
+                qx = g.integers(-127, 128, (M, K), dtype=np.int8)
+                a = qx.astype(np.int64)
+            else:
+                qx = g.integers(0, 256, (M, K // 2), dtype=np.uint8)
+                a = unpack_nibbles(qx).astype(np.int64)
+            acc = orc.gemm_s32(qx, bits, qw, K)
+            if not np.array_equal(acc.astype(np.int64), a @ w.T):
+                fails.append(f"gemm_vs_matmul seed {seed} bits {bits}")
+    return fails
+
+
+def epilogue_fp64(orc, seeds=(6,)):
+    fails = []
+    for seed in seeds:
+        g = np.random.default_rng(seed)
+        M, N, T, S = 19, 21, 4, 3
+        acc = g.integers(-2 ** 20, 2 ** 20, (M, N)).astype(np.int32)
+        s_tok = g.uniform(1e-4, 1e-2, M).astype(np.float32)
+        s_w = g.uniform(1e-4, 1e-2, N).astype(np.float32)
+        bias = g.normal(0, 0.1, N).astype(np.float32)
+        beta = g.normal(0, 0.1, (T, S, N)).astype(np.float32)
+        sid = g.integers(0, S, M).astype(np.uint8)
+        step = 2
+        y = orc.epilogue(acc, s_tok, s_w, bias, beta, sid, step)
+        ref = (s_tok.astype(np.float64)[:, None] * s_w.astype(np.float64)[None, :] * acc
+               + bias.astype(np.float64)[None, :] + beta[step, sid].astype(np.float64))
+        # y must be the bf16 value nearest to the fp64 result: no bf16 neighbour of
+        # y (pattern +-1) may be closer to it.
+        err = np.abs(bf16_to_f32(y).astype(np.float64) - ref)
+        for d in (1, -1):
+            nb = bf16_to_f32((y.astype(np.int32) + d).astype(np.uint16)).astype(np.float64)
+            if np.any(np.abs(nb - ref) < err):
+                fails.append(f"epilogue_fp64 seed {seed}: not the nearest bf16 value")
+                break
+    return fails
+
+
+def tolerance_ok(y_bits, ref):
+    """max |y - y_ref| <= 2^-7 |y_ref| + 1e-3 rms(y_ref), element-wise."""
+    y = bf16_to_f32(y_bits).astype(np.float64)
+    ref = np.asarray(ref, np.float64)
+    rms = np.sqrt(np.mean(ref ** 2)) if ref.size else 0.0
+    return bool(np.all(np.abs(y - ref) <= 2.0 ** -7 * np.abs(ref) + 1e-3 * rms))
+
+
+def textbook(orc, seeds=(7,)):
+    """cinv=1, alpha=1, beta=0: plain per-token x per-output-channel symmetric GEMM."""
+    fails = []
+    for seed in seeds:
+        x, _, sid, _, _, W, bias, _ = _tiny_inputs(seed)
+        for bits, qmax in ((8, 127.0), (4, 7.0)):
+            qw, s_w = orc.pack_int4(W, None)
+            ones = np.ones((1, 3), np.float32)
+            y, _, _, _ = orc.linear(x, None, sid, ones, None, 0, bits, qw, s_w, bias)
+            xf = bf16_to_f32(x)
+            sx = (np.abs(xf).max(axis=1) / np.float32(qmax)).astype(np.float32)
+            with np.errstate(divide="ignore", invalid="ignore"):
+                qa = np.clip(np.rint(np.where(sx[:, None] > 0, xf / sx[:, None], 0)), -qmax, qmax)
+            wf = bf16_to_f32(W)
+            sw = (np.abs(wf).max(axis=1) / np.float32(7.0)).astype(np.float32)
+            qb = np.clip(np.rint(wf / sw[:, None]), -7, 7)
+            ref = (sx.astype(np.float64)[:, None] * sw.astype(np.float64)[None, :]
+                   * (qa.astype(np.float64) @ qb.astype(np.float64).T) + bias[None, :])
+            if not tolerance_ok(y, ref):
+                fails.append(f"textbook seed {seed} bits {bits}")
+    return fails
+
+
+def on_grid(orc, seeds=(8,)):
+    """x = q * 2^e with the row maximum at qmax: lossless, y = fp64 product."""
+    fails = []
+    for seed in seeds:
+        g = np.random.default_rng(seed)
+        M, K, N = 20, 64, 24
+        for bits, qmax in ((8, 127), (4, 7)):
+            q = g.integers(-qmax, qmax + 1, (M, K))
+            q[np.arange(M), g.integers(0, K, M)] = qmax * g.choice([-1, 1], M)
+            e = g.integers(-8, 4, M).astype(np.float64)
+            xv = (q * 2.0 ** e[:, None]).astype(np.float32)
+            x = bf16_from_values(xv)
+            sid = g.integers(0, 3, M).astype(np.uint8)
+            W = f32_to_bf16_bits(g.normal(0, 0.05, (N, K)).astype(np.float32))
+            qw, s_w = orc.pack_int4(W, None)
+            bias = g.normal(0, 0.01, N).astype(np.float32)
+            beta = g.normal(0, 1e-3, (1, 3, N)).astype(np.float32)
+            y, qx, s_tok, _ = orc.linear(x, None, sid, np.ones((1, 3), np.float32), beta, 0,
+                                         bits, qw, s_w, bias)
+            codes = unpack_nibbles(qx) if bits == 4 else qx.astype(np.int64)
+            if not np.array_equal(codes, q) or not np.array_equal(s_tok, 2.0 ** e):
+                fails.append(f"on_grid seed {seed} bits {bits}: not lossless")
+            wdq = unpack_nibbles(qw).astype(np.float64) * s_w.astype(np.float64)[:, None]
+            ref = xv.astype(np.float64) @ wdq.T + bias[None, :] + beta[0, sid]
+            if not tolerance_ok(y, ref):
+                fails.append(f"on_grid seed {seed} bits {bits}: y off")
+    return fails
+
+
+def requant(orc, seeds=(9,)):
+    fails = []
+    for seed in seeds:
+        x, cinv, sid, alpha, _, _, _, _ = _tiny_inputs(seed)
+        ones = np.ones((1, 3), np.float32)
+        qx, s = orc.act_quant(x, None, sid, ones, 0, 4)
+        codes = unpack_nibbles(qx).astype(np.float32)
+        xd = f32_to_bf16_bits(codes * s[:, None])
+        qx2, s2 = orc.act_quant(xd, None, sid, ones, 0, 4)
+        if not np.array_equal(qx2, qx):
+            fails.append(f"requant seed {seed}: codes changed")
+        if np.any(np.abs(s2 - s) > 2.0 ** -8 * s):
+            fails.append(f"requant seed {seed}: scale moved")
+    return fails
+
+
+def scale_invariance(orc, seeds=(10,)):
+    fails = []
+    for seed in seeds:
+        x, cinv, sid, alpha, _, _, _, _ = _tiny_inputs(seed)
+        x2 = f32_to_bf16_bits(bf16_to_f32(x) * np.float32(2.0))
+        for bits in (8, 4):
+            qa, sa = orc.act_quant(x, cinv, sid, alpha, 1, bits)
+            qb, sb = orc.act_quant(x2, cinv, sid, alpha, 1, bits)
+            if not np.array_equal(qa, qb) or not np.array_equal(sb, sa * np.float32(2.0)):
+                fails.append(f"scale_invariance seed {seed} bits {bits}")
+    return fails
+
+
+def near_tie_inputs(seed, K=4096, qmax=127):
+    """One row whose scaled values sit within a few ulps of half-integer multiples
+    of the row scale: x = 1 everywhere except x[0] = qmax (the row maximum), and
+    cinv[k] is chosen so x'[k] / s lands next to j + 1/2.  Builds inputs only."""
+    g = np.random.default_rng(seed)
+    c0 = g.uniform(1.0, 1.5)
+    j = g.integers(-qmax, qmax, K).astype(np.float64)
+    target = (j + 0.5) * c0
+    ulps = g.integers(-3, 4, K)
+    cinv = np.abs(target).astype(np.float32)      # the sign lives in x
+    for i in range(3):                            # move |ulps| steps up or down
+        step_to = np.where(ulps > 0, np.float32(np.inf), np.float32(0.0)).astype(np.float32)
+        cinv = np.where(np.abs(ulps) > i, np.nextafter(cinv, step_to), cinv).astype(np.float32)
+    x = np.where(target < 0, np.float32(-1.0), np.float32(1.0)).astype(np.float32)
+    x[0] = qmax
+    cinv[0] = np.float32(c0)
+    return bf16_from_values(x[None, :]), cinv
+
+
+def near_ties(orc, seeds=(11, 12)):
+    """Codes at near-ties must follow the IEEE binary32 quotient x'/s exactly; a
+    reciprocal-multiply shortcut (x' * (1/s)) rounds some of these differently."""
+    fails = []
+    for seed in seeds:
+        for bits, qmax in ((8, 127), (4, 7)):
+            x, cinv = near_tie_inputs(seed, qmax=qmax)
+            sid = np.zeros(1, np.uint8)
+            qx, s = orc.act_quant(x, cinv, sid, np.ones((1, 1), np.float32), 0, bits)
+            codes = unpack_nibbles(qx) if bits == 4 else qx.astype(np.int64)
+            xp = bf16_to_f32(x) * cinv[None, :]
+            t = (xp / s[:, None]).astype(np.float32)
+            want = np.clip(np.rint(t), -qmax, qmax).astype(np.int64)
+            if not np.array_equal(codes, want):
+                fails.append(f"near_ties seed {seed} bits {bits}: "
+                             f"{int((codes != want).sum())} codes differ")
+    return fails
+
+
+ALL_CHECKS = (golden_act_quant, golden_pack, golden_channel_scale, golden_linear,
+              golden_bf16_rounding, brute_codes, gemm_vs_matmul, epilogue_fp64, textbook,
+              on_grid, requant, scale_invariance, near_ties)
+GOLDEN_CHECKS = ALL_CHECKS[:5]
+
+
+def all_failures(orc, golden):
+    out = []
+    for chk in ALL_CHECKS:
+        try:
+            out += chk(orc, golden) if chk in GOLDEN_CHECKS else chk(orc)
+        except ValueError as e:  # the oracle refused an input
+            out.append(f"{chk.__name__}: {e}")
+    return out

@@ -1,0 +1,91 @@
+"""The CPU oracle against hand-derived examples, brute force, library routines and
+the invariants of the method; plus planted mistakes that the pins must catch.
+
+Each planted mistake is a textual edit of a temporary copy of oracle/oracle.c,
+built on the CPU; the real oracle source is never modified.
+"""
+import os
+import tempfile
+
+import pytest
+
+import oracle as oracle_pkg
+from oracle import Oracle
+from oracle import build as oracle_build
+
+import oracle_pins as P
+
+
+@pytest.mark.parametrize("check", P.GOLDEN_CHECKS, ids=lambda c: c.__name__)
+def test_golden(oracle, golden, check):
+    assert check(oracle, golden) == []
+
+
+@pytest.mark.parametrize("check", [c for c in P.ALL_CHECKS if c not in P.GOLDEN_CHECKS],
+                         ids=lambda c: c.__name__)
+def test_property(oracle, check):
+    assert check(oracle) == []
+
+
+# (description, [(text in oracle.c, replacement), ...])
+MUTANTS = [
+    ("reciprocal multiply instead of division",
+     [("float t = v / s;", "float t = v * (1.0f / s);")]),
+    ("round half away from zero", [("float r = rintf(t);", "float r = roundf(t);")]),
+    ("no clamp at +qmax", [("if (r > qmax) r = qmax;", "")]),
+    ("channel scale not folded into activations",
+     [("xp[k] = oracle_bf16_to_float(x[(size_t)m * K + k]) * ck;",
+       "xp[k] = oracle_bf16_to_float(x[(size_t)m * K + k]);")]),
+    ("clip ratio ignored", [("float clip = alpha[(size_t)step * S + sid] * amax;",
+                             "float clip = amax;")]),
+    ("clip table indexed [stream][step]",
+     [("float clip = alpha[(size_t)step * S + sid] * amax;",
+       "float clip = alpha[(size_t)sid * T + step] * amax;")]),
+    ("signed maximum instead of absolute", [("      float a = fabsf(xp[k]);", "      float a = xp[k];")]),
+    ("weight qmax 8", [("const float qmax = 7.0f;", "const float qmax = 8.0f;")]),
+    ("high nibble holds the even k (pack and unpack)",
+     [("return (uint8_t)(((unsigned)lo & 0xFu) | (((unsigned)hi & 0xFu) << 4));",
+       "return (uint8_t)(((unsigned)hi & 0xFu) | (((unsigned)lo & 0xFu) << 4));"),
+      ("int v = high ? (byte >> 4) & 0xF : byte & 0xF;",
+       "int v = high ? byte & 0xF : (byte >> 4) & 0xF;")]),
+    ("nibble sign extension wrong", [("return v >= 8 ? v - 16 : v;", "return v >= 8 ? 16 - v : v;")]),
+    ("weight nibble off by one",
+     [("int w = unpack_nibble(qw[(size_t)n * (K / 2) + k / 2], k & 1);",
+       "int w = unpack_nibble(qw[(size_t)n * (K / 2) + k / 2], (k + 1) & 1);")]),
+    ("bias dropped", [("if (bias) v += (double)bias[n];", "")]),
+    ("output compensation indexed [stream][step]",
+     [("if (beta) v += (double)beta[((size_t)step * S + sid) * N + n];",
+       "if (beta) v += (double)beta[((size_t)sid * T + step) * N + n];")]),
+    ("accumulator transposed",
+     [("(double)acc[(size_t)m * N + n];", "(double)acc[(size_t)n * M + m];")]),
+    ("token and channel scales swapped",
+     [("double v = (double)s_tok[m] * (double)s_w[n]", "double v = (double)s_tok[n] * (double)s_w[m]")]),
+    ("bf16 rounding half away from zero",
+     [("double r = nearbyint(ldexp(a, 8 - e));", "double r = round(ldexp(a, 8 - e));")]),
+    ("channel scale inverted", [("if (a > 0.0f && b > 0.0f) ck = sqrtf(a / b);",
+                                 "if (a > 0.0f && b > 0.0f) ck = sqrtf(b / a);")]),
+]
+
+
+@pytest.fixture(scope="module")
+def mutant_dir():
+    with tempfile.TemporaryDirectory() as d:
+        yield d
+
+
+@pytest.mark.parametrize("desc,edits", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(golden, mutant_dir, desc, edits):
+    src = open(oracle_build.SRC).read()
+    for old, new in edits:
+        assert src.count(old) == 1, f"edit site not unique or missing: {old!r}"
+        src = src.replace(old, new)
+    tag = "".join(ch if ch.isalnum() else "_" for ch in desc)
+    c_path = os.path.join(mutant_dir, f"{tag}.c")
+    with open(c_path, "w") as f:
+        f.write(src)
+    # the mutant includes "oracle.h" from the real source directory
+    so = oracle_build.build(c_path, os.path.join(mutant_dir, f"{tag}.so"),
+                            extra=("-I", os.path.dirname(oracle_build.SRC)))
+    mutant = Oracle(oracle_pkg.load(so))
+    fails = P.all_failures(mutant, golden)
+    assert fails, f"planted mistake '{desc}' passed every pin"
