@@ -1,0 +1,193 @@
+// C ABI of libwq (declared in include/wq.h): host-side validation, workspace
+// layout and launches.  The whole library is this one translation unit; the
+// kernels live in the included .cuh files.
+#include "../../include/wq.h"
+
+#include <cstdint>
+
+#include "wq_gemm.cuh"
+#include "wq_internal.h"
+#include "wq_quant.cuh"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+wq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
+
+wq_status check_mk(int M, int K) {
+  if (M < 0 || K < 128 || (K % 128) != 0 || K > wq::kMaxK) return WQ_ERR_SHAPE;
+  return WQ_OK;
+}
+
+wq_status check_n(int N) { return (N < 16 || (N % 16) != 0) ? WQ_ERR_SHAPE : WQ_OK; }
+
+wq_status check_table(int S, int T, int step) {
+  if (S < 1 || S > 255 || T < 1 || step < 0 || step >= T) return WQ_ERR_ARG;
+  return WQ_OK;
+}
+
+size_t act_bytes(int M, int K, int act_bits) {
+  return act_bits == 8 ? static_cast<size_t>(M) * K : static_cast<size_t>(M) * (K / 2);
+}
+
+#define WQ_TRY(expr)                 \
+  do {                               \
+    const wq_status _s = (expr);     \
+    if (_s != WQ_OK) return _s;      \
+  } while (0)
+
+wq_status gemm_checks(const void* qx, const float* s_tok, int act_bits, int M, int K, int N,
+                      const uint8_t* stream_id, const float* beta, int S, int T, int step,
+                      const uint8_t* qw, const float* s_w, const float* bias, const void* y) {
+  if (act_bits != 8 && act_bits != 4) return WQ_ERR_ARG;
+  WQ_TRY(check_mk(M, K));
+  WQ_TRY(check_n(N));
+  WQ_TRY(check_table(S, T, step));
+  if (!qx || !s_tok || !stream_id || !qw || !s_w || !y) return WQ_ERR_NULL;
+  if (!aligned16(qx) || !aligned16(qw) || !aligned16(y) || !aligned16(s_tok) ||
+      !aligned16(s_w) || (bias && !aligned16(bias)) || (beta && !aligned16(beta)))
+    return WQ_ERR_ALIGN;
+  return WQ_OK;
+}
+
+wq_status linear(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                 const uint8_t* stream_id, const float* alpha, const float* beta, int S, int T,
+                 int step, const uint8_t* qw, const float* s_w, const float* bias, wq_bf16* y,
+                 void* workspace, size_t ws_bytes, wq_stream_t stream, int act_bits) {
+  WQ_TRY(check_mk(M, K));
+  WQ_TRY(check_n(N));
+  WQ_TRY(check_table(S, T, step));
+  if (!x || !stream_id || !alpha || !qw || !s_w || !y || (!workspace && M > 0))
+    return WQ_ERR_NULL;
+  if (!aligned16(x) || !aligned16(qw) || !aligned16(y) || !aligned16(s_w) ||
+      (cinv && !aligned16(cinv)) || (bias && !aligned16(bias)) || (beta && !aligned16(beta)) ||
+      (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return WQ_ERR_ALIGN;
+  if (ws_bytes < wq_workspace_bytes(M, K, N, act_bits)) return WQ_ERR_ARG;
+  if (M == 0) return WQ_OK;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* qx = ws;
+  float* s_tok = reinterpret_cast<float*>(ws + round_up(act_bytes(M, K, act_bits)));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  WQ_TRY(from_cuda(wq::launch_act_quant(x, M, K, cinv, stream_id, alpha, S, step, act_bits, qx,
+                                        s_tok, st)));
+  const wq::EpilogueArgs ep{s_tok, stream_id, s_w, bias, beta, S, step};
+  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, y, false, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* wq_status_string(wq_status s) {
+  switch (s) {
+    case WQ_OK: return "WQ_OK";
+    case WQ_ERR_NULL: return "WQ_ERR_NULL: a required pointer is NULL";
+    case WQ_ERR_SHAPE: return "WQ_ERR_SHAPE: M, N or K outside the supported range";
+    case WQ_ERR_ALIGN: return "WQ_ERR_ALIGN: a tensor pointer is not 16-byte aligned";
+    case WQ_ERR_ARG: return "WQ_ERR_ARG: bad act_bits, S, T, step or workspace size";
+    case WQ_ERR_CUDA: return "WQ_ERR_CUDA: the CUDA runtime rejected a launch";
+    case WQ_ERR_TIMEOUT: return "WQ_ERR_TIMEOUT: a kernel's bounded wait gave up";
+    case WQ_ERR_DEVICE: return "WQ_ERR_DEVICE: a device-side precondition failed";
+  }
+  return "unknown wq_status";
+}
+
+int wq_version(void) { return 100; }
+
+size_t wq_workspace_bytes(int M, int K, int N, int act_bits) {
+  if ((act_bits != 8 && act_bits != 4) || check_mk(M, K) != WQ_OK || check_n(N) != WQ_OK)
+    return 0;
+  return round_up(act_bytes(M, K, act_bits)) + round_up(sizeof(float) * static_cast<size_t>(M));
+}
+
+wq_status wq_channel_scale(const wq_bf16* x_cal, int Mcal, const wq_bf16* W, int N, int K,
+                           float* c, float* cinv, wq_stream_t stream) {
+  if (Mcal < 1 || N < 1 || K < 1) return WQ_ERR_SHAPE;
+  if (!x_cal || !W || !c || !cinv) return WQ_ERR_NULL;
+  return from_cuda(wq::launch_channel_scale(x_cal, Mcal, W, N, K, c, cinv,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_pack_int4(const wq_bf16* W, const float* c, int N, int K, uint8_t* qw,
+                       float* s_w, wq_stream_t stream) {
+  WQ_TRY(check_mk(0, K));
+  if (N < 1) return WQ_ERR_SHAPE;
+  if (!W || !qw || !s_w) return WQ_ERR_NULL;
+  if (!aligned16(W) || !aligned16(qw) || (c && !aligned16(c))) return WQ_ERR_ALIGN;
+  return from_cuda(
+      wq::launch_pack_int4(W, c, N, K, qw, s_w, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_act_quant(const wq_bf16* x, int M, int K, const float* cinv,
+                       const uint8_t* stream_id, const float* alpha, int S, int T, int step,
+                       int act_bits, void* qx, float* s_tok, wq_stream_t stream) {
+  if (act_bits != 8 && act_bits != 4) return WQ_ERR_ARG;
+  WQ_TRY(check_mk(M, K));
+  WQ_TRY(check_table(S, T, step));
+  if (!x || !stream_id || !alpha || !qx || !s_tok) return WQ_ERR_NULL;
+  if (!aligned16(x) || !aligned16(qx) || (cinv && !aligned16(cinv))) return WQ_ERR_ALIGN;
+  return from_cuda(wq::launch_act_quant(x, M, K, cinv, stream_id, alpha, S, step, act_bits, qx,
+                                        s_tok, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_gemm_w4ax(const void* qx, const float* s_tok, int act_bits, int M, int K, int N,
+                       const uint8_t* stream_id, const float* beta, int S, int T, int step,
+                       const uint8_t* qw, const float* s_w, const float* bias, wq_bf16* y,
+                       wq_stream_t stream) {
+  WQ_TRY(gemm_checks(qx, s_tok, act_bits, M, K, N, stream_id, beta, S, T, step, qw, s_w, bias,
+                     y));
+  const wq::EpilogueArgs ep{s_tok, stream_id, s_w, bias, beta, S, step};
+  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, y, false,
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_linear_w4a8(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                         const uint8_t* stream_id, const float* alpha, const float* beta,
+                         int S, int T, int step, const uint8_t* qw, const float* s_w,
+                         const float* bias, wq_bf16* y, void* workspace, size_t ws_bytes,
+                         wq_stream_t stream) {
+  return linear(x, M, K, N, cinv, stream_id, alpha, beta, S, T, step, qw, s_w, bias, y,
+                workspace, ws_bytes, stream, 8);
+}
+
+wq_status wq_linear_w4a4(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                         const uint8_t* stream_id, const float* alpha, const float* beta,
+                         int S, int T, int step, const uint8_t* qw, const float* s_w,
+                         const float* bias, wq_bf16* y, void* workspace, size_t ws_bytes,
+                         wq_stream_t stream) {
+  return linear(x, M, K, N, cinv, stream_id, alpha, beta, S, T, step, qw, s_w, bias, y,
+                workspace, ws_bytes, stream, 4);
+}
+
+wq_status wq_debug_gemm_s32(const void* qx, int act_bits, const uint8_t* qw, int M, int N,
+                            int K, int32_t* acc, wq_stream_t stream) {
+  if (act_bits != 8 && act_bits != 4) return WQ_ERR_ARG;
+  WQ_TRY(check_mk(M, K));
+  WQ_TRY(check_n(N));
+  if (!qx || !qw || !acc) return WQ_ERR_NULL;
+  if (!aligned16(qx) || !aligned16(qw) || !aligned16(acc)) return WQ_ERR_ALIGN;
+  const wq::EpilogueArgs ep{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 0};
+  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, acc, true,
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_device_status(unsigned* flags) {
+  unsigned word = 0;
+  const unsigned zero = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return WQ_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&word, wq::g_error_word, sizeof word) != cudaSuccess) return WQ_ERR_CUDA;
+  if (word != 0 && cudaMemcpyToSymbol(wq::g_error_word, &zero, sizeof zero) != cudaSuccess)
+    return WQ_ERR_CUDA;
+  if (flags) *flags = word;
+  if (word & WQ_DEVICE_ERR_TIMEOUT) return WQ_ERR_TIMEOUT;
+  if (word) return WQ_ERR_DEVICE;
+  return WQ_OK;
+}
+
+}  // extern "C"

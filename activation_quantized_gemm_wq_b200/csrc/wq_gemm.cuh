@@ -1,0 +1,487 @@
+// The second Rudder kernel (SteerQuant §4.4): low-bit GEMM of integer activation
+// codes with one static int4 weight matrix, int32 accumulation, and a fused
+// epilogue doing dequantization (s_tok * s_w), bias and the per-(step, stream)
+// output compensation beta (§1: Rudder fuses scaling and output compensation).
+//
+// sm_100a design (one persistent CTA per SM, warp-specialised):
+//   warp 0      TMA producer: packed int4 weight tile [128 n][64 B] (64-byte
+//               swizzle) and the activation tile [BN tokens][BK] (int8: 128-byte
+//               swizzle, consumed directly by the MMA; int4: 64-byte swizzle)
+//   warp 1      TMEM allocator and the single MMA-issuing thread:
+//               tcgen05.mma kind::i8, M=128 (output channels), N=BN (tokens),
+//               K=32 per instruction, accumulators in TMEM, double-buffered so the
+//               epilogue of tile i overlaps the mainloop of tile i+1
+//   unpack      int4 -> int8 conversion in shared memory, written in the 128-byte
+//   warps       swizzled K-major layout the MMA descriptors expect (weights, and
+//               activations when they are int4)
+//   epilogue    tcgen05.ld of the accumulator, y = bf16((s_tok*s_w)*acc + bias +
+//   warps       beta[step][stream][n]), staged in shared memory and written with
+//               TMA stores (tails clipped by the tensor map)
+// The output-channel dimension is the MMA's M ("swap AB"), so the same kernel
+// serves any token count from 1 to the full batch, with token tiles of 16..256.
+//
+// Every mbarrier wait is bounded (see wq_ptx.cuh): on timeout the kernel raises
+// a device error bit, drains, frees its TMEM and returns.
+#pragma once
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "wq_internal.h"
+#include "wq_ptx.cuh"
+
+namespace wq {
+namespace {
+
+struct TileArgs {
+  int M, N, K;
+  int tiles_m, tiles_n, num_tiles;
+  int n_fastest;
+  EpilogueArgs ep;
+};
+
+template <int BN_, int ACT_BITS_, bool OUT_S32_>
+struct Cfg {
+  static constexpr int BN = BN_;
+  static constexpr int ACT_BITS = ACT_BITS_;
+  static constexpr bool OUT_S32 = OUT_S32_;
+  static constexpr int BM = 128;  // output channels per tile (MMA M)
+  static constexpr int BK = 128;  // K elements per pipeline stage
+  static constexpr int UNPACK_WARPS = ACT_BITS == 4 ? 8 : 4;
+  static constexpr int EPI_WARPS = 4;
+  static constexpr int FIRST_UNPACK_WARP = 2;
+  static constexpr int FIRST_EPI_WARP = FIRST_UNPACK_WARP + UNPACK_WARPS;
+  static constexpr int NUM_WARPS = FIRST_EPI_WARP + EPI_WARPS;
+  static constexpr int THREADS = NUM_WARPS * 32;
+
+  static constexpr int WP_BYTES = BM * BK / 2;                               // packed W
+  static constexpr int WU_BYTES = BM * BK;                                   // int8 W
+  static constexpr int XS_BYTES = ACT_BITS == 8 ? BN * BK : BN * BK / 2;     // staged x
+  static constexpr int XU_BYTES = ACT_BITS == 8 ? 0 : BN * BK;               // int8 x (A4)
+  static constexpr int STAGE_BYTES = WP_BYTES + XS_BYTES;
+  static constexpr int NU = 2;  // unpacked buffers
+  static constexpr int EPI_ELEM = OUT_S32 ? 4 : 2;
+  static constexpr int EPI_CHUNK = BN < 32 ? BN : 32;  // token columns per TMEM load
+  static constexpr int EPI_BUF_BYTES = EPI_CHUNK * 32 * EPI_ELEM;
+  static constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BUF_BYTES;
+  static constexpr int SMEM_LIMIT = 232448;  // 227 KB opt-in per CTA
+  static constexpr int RESERVED = 1024 /*alignment slack*/ + 512 /*barriers*/;
+  static constexpr int NS_FIT =
+      (SMEM_LIMIT - RESERVED - NU * (WU_BYTES + XU_BYTES) - EPI_BYTES) / STAGE_BYTES;
+  static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
+  static_assert(NS >= 2, "pipeline needs at least two stages");
+
+  static constexpr int OFF_WP = 0;
+  static constexpr int OFF_XS = OFF_WP + NS * WP_BYTES;
+  static constexpr int OFF_WU = OFF_XS + NS * XS_BYTES;
+  static constexpr int OFF_XU = OFF_WU + NU * WU_BYTES;
+  static constexpr int OFF_EPI = OFF_XU + NU * XU_BYTES;
+  static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
+  static constexpr int NUM_BARS = 2 * NS + 2 * NU + 4;
+  static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
+  static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
+  static_assert(OFF_XS % 1024 == 0 && XS_BYTES % 512 == 0 && OFF_WU % 1024 == 0 &&
+                    OFF_XU % 1024 == 0 && OFF_EPI % 1024 == 0,
+                "swizzled tiles need 1024-byte alignment");
+
+  static constexpr uint32_t TMEM_COLS =
+      2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
+};
+
+__device__ __forceinline__ void decode_tile(const TileArgs& a, int tile, int& n_tile,
+                                            int& m_tile) {
+  if (a.n_fastest) {
+    n_tile = tile % a.tiles_n;
+    m_tile = tile / a.tiles_n;
+  } else {
+    m_tile = tile % a.tiles_m;
+    n_tile = tile / a.tiles_m;
+  }
+}
+
+// 16 packed bytes (32 int4 codes, low nibble first) -> 32 int8 codes.
+__device__ __forceinline__ void unpack32(const uint4 p, uint4& lo16, uint4& hi16) {
+  const uint32_t w[4] = {p.x, p.y, p.z, p.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    // bytes of e: even-k nibbles, of f: odd-k nibbles, each biased by ^8
+    const uint32_t e = (w[i] & 0x0F0F0F0Fu) ^ 0x08080808u;
+    const uint32_t f = ((w[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+    uint32_t a = __byte_perm(e, f, 0x5140);  // k0 k1 k2 k3
+    uint32_t b = __byte_perm(e, f, 0x7362);  // k4 k5 k6 k7
+    // per byte: (n ^ 8) + 0x78 stays below 0x100; ^0x80 then yields n - 16*(n >= 8)
+    o[2 * i] = (a + 0x78787878u) ^ 0x80808080u;
+    o[2 * i + 1] = (b + 0x78787878u) ^ 0x80808080u;
+  }
+  lo16 = make_uint4(o[0], o[1], o[2], o[3]);
+  hi16 = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// Packed tile [rows][64 B] with the 64-byte swizzle -> int8 tile [rows][128 B]
+// with the 128-byte swizzle.  Task i covers row i/4, packed 16-byte chunk i%4.
+__device__ __forceinline__ void unpack_tile(const uint8_t* src, uint8_t* dst, int rows,
+                                            int tid, int nthreads) {
+  for (int i = tid; i < rows * 4; i += nthreads) {
+    const int r = i >> 2, p = i & 3;
+    const uint4 v =
+        *reinterpret_cast<const uint4*>(src + r * 64 + ((p ^ ((r >> 1) & 3)) << 4));
+    uint4 lo, hi;
+    unpack32(v, lo, hi);
+    uint8_t* row = dst + r * 128;
+    *reinterpret_cast<uint4*>(row + (((2 * p) ^ (r & 7)) << 4)) = lo;
+    *reinterpret_cast<uint4*>(row + (((2 * p + 1) ^ (r & 7)) << 4)) = hi;
+  }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                const __grid_constant__ CUtensorMap tm_out, const TileArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* empty = full + C::NS;
+  uint64_t* ufull = empty + C::NS;
+  uint64_t* uempty = ufull + C::NU;
+  uint64_t* tfull = uempty + C::NU;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_k = args.K / C::BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], C::ACT_BITS == 8 ? 1 : C::UNPACK_WARPS);
+    }
+    for (int u = 0; u < C::NU; ++u) {
+      mbar_init(&ufull[u], C::UNPACK_WARPS);
+      mbar_init(&uempty[u], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], C::EPI_WARPS);
+    }
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_out);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+        int n_tile, m_tile;
+        decode_tile(args, tile, n_tile, m_tile);
+        for (int kb = 0; kb < num_k; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+          tma_load_2d(smem + C::OFF_WP + s * C::WP_BYTES, &tm_w, &full[s], kb * (C::BK / 2),
+                      n_tile * C::BM);
+          tma_load_2d(smem + C::OFF_XS + s * C::XS_BYTES, &tm_x, &full[s],
+                      kb * (C::ACT_BITS == 8 ? C::BK : C::BK / 2), m_tile * C::BN);
+          ++issued;
+          if (++s == C::NS) { s = 0; ph ^= 1u; }
+        }
+      }
+      // Drain: every issued stage's copies must have landed before the CTA exits.
+      // (Normally they were all consumed already and these waits return at once.)
+      for (int i = 0; i < C::NS && i < issued; ++i) {
+        if (--s < 0) { s = C::NS - 1; ph ^= 1u; }
+        mbar_wait(&full[s], ph);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(C::BN);
+      int s = 0, u = 0, b = 0;
+      uint32_t ph_s = 0, ph_u = 0, ph_b = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[b], ph_b ^ 1u)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * C::BN);
+        for (int kb = 0; kb < num_k; ++kb) {
+          if (C::ACT_BITS == 8 && !mbar_wait(&full[s], ph_s)) { ok = false; break; }
+          if (!mbar_wait(&ufull[u], ph_u)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + C::OFF_WU + u * C::WU_BYTES);
+          const uint32_t b_addr =
+              C::ACT_BITS == 8 ? smem_u32(smem + C::OFF_XS + s * C::XS_BYTES)
+                               : smem_u32(smem + C::OFF_XU + u * C::XU_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < C::BK / 32; ++kk) {
+            mma_i8_ss(d_tmem, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32),
+                      idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&uempty[u]);
+          if (C::ACT_BITS == 8) mma_commit(&empty[s]);
+          if (++u == C::NU) { u = 0; ph_u ^= 1u; }
+          if (++s == C::NS) { s = 0; ph_s ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[b]);
+        if (++b == 2) { b = 0; ph_b ^= 1u; }
+      }
+    }
+    __syncwarp();
+  } else if (warp < C::FIRST_EPI_WARP) {
+    // ------------------------------------------------------------ int4 -> int8
+    const int tid = threadIdx.x - C::FIRST_UNPACK_WARP * 32;
+    constexpr int NT = C::UNPACK_WARPS * 32;
+    int s = 0, u = 0;
+    uint32_t ph_s = 0, ph_u = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+      for (int kb = 0; kb < num_k; ++kb) {
+        bool w = mbar_wait(&full[s], ph_s);
+        w = w && mbar_wait(&uempty[u], ph_u ^ 1u);
+        if (!__all_sync(0xFFFFFFFFu, w)) {  // keep the warp's decision uniform
+          ok = false;
+          break;
+        }
+        unpack_tile(smem + C::OFF_WP + s * C::WP_BYTES, smem + C::OFF_WU + u * C::WU_BYTES,
+                    C::BM, tid, NT);
+        if constexpr (C::ACT_BITS == 4) {
+          unpack_tile(smem + C::OFF_XS + s * C::XS_BYTES, smem + C::OFF_XU + u * C::XU_BYTES,
+                      C::BN, tid, NT);
+        }
+        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&ufull[u]);
+          if (C::ACT_BITS == 4) mbar_arrive(&empty[s]);
+        }
+        if (++u == C::NU) { u = 0; ph_u ^= 1u; }
+        if (++s == C::NS) { s = 0; ph_s ^= 1u; }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int e = warp - C::FIRST_EPI_WARP;
+    uint8_t* ebuf = smem + C::OFF_EPI + e * 2 * C::EPI_BUF_BYTES;
+    int b = 0, buf = 0;
+    uint32_t ph_b = 0;
+    const EpilogueArgs& ep = args.ep;
+    const bool small_s = ep.S <= 4;
+    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
+      int n_tile, m_tile;
+      decode_tile(args, tile, n_tile, m_tile);
+      const int n_base = n_tile * C::BM + q * 32;
+      const int n = n_base + lane;
+      const int m0 = m_tile * C::BN;
+      float sw = 0.0f, bs = 0.0f, bt[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (!C::OUT_S32 && n < args.N) {
+        sw = ep.s_w[n];
+        bs = ep.bias ? ep.bias[n] : 0.0f;
+        if (ep.beta && small_s) {
+          const float* row = ep.beta + (size_t)ep.step * ep.S * args.N + n;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (j < ep.S) bt[j] = row[(size_t)j * args.N];
+        }
+      }
+      const bool w = mbar_wait(&tfull[b], ph_b);
+      if (!__all_sync(0xFFFFFFFFu, w)) break;  // uniform, and converged for tcgen05.ld
+      tc_fence_after();
+      for (int j0 = 0; j0 < C::BN; j0 += C::EPI_CHUNK) {
+        uint32_t r[32];
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>(b * C::BN + j0);
+        if constexpr (C::EPI_CHUNK == 32) {
+          tmem_ld_32x32b_x32(taddr, r);
+        } else {
+          uint32_t (&r16)[16] = *reinterpret_cast<uint32_t(*)[16]>(r);
+          tmem_ld_32x32b_x16(taddr, r16);
+        }
+        tmem_wait_ld();
+        if (m0 + j0 >= args.M) continue;  // whole chunk beyond the last token
+        // this lane's token (for broadcast by shuffle)
+        const int ml = m0 + j0 + lane;
+        float st_l = 0.0f;
+        int sid_l = 0;
+        if (!C::OUT_S32 && lane < C::EPI_CHUNK && ml < args.M) {
+          st_l = ep.s_tok[ml];
+          sid_l = ep.stream_id[ml];
+        }
+        uint8_t* sb = ebuf + buf * C::EPI_BUF_BYTES;
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < C::EPI_CHUNK; ++j) {
+          if constexpr (C::OUT_S32) {
+            reinterpret_cast<uint32_t*>(sb)[j * 32 + lane] = r[j];
+          } else {
+            const float st = __shfl_sync(0xFFFFFFFFu, st_l, j);
+            const int sd = __shfl_sync(0xFFFFFFFFu, sid_l, j);
+            float bv;
+            if (ep.beta == nullptr) {
+              bv = 0.0f;
+            } else if (small_s) {
+              bv = sd == 0 ? bt[0] : sd == 1 ? bt[1] : sd == 2 ? bt[2] : bt[3];
+            } else {
+              bv = n < args.N ? ep.beta[((size_t)ep.step * ep.S + sd) * args.N + n] : 0.0f;
+            }
+            float v = __fmul_rn(__fmul_rn(st, sw), __int2float_rn(static_cast<int>(r[j])));
+            v = __fadd_rn(__fadd_rn(v, bs), bv);
+            reinterpret_cast<__nv_bfloat16*>(sb)[j * 32 + lane] = __float2bfloat16_rn(v);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && n_base < args.N) {
+          tma_store_2d(&tm_out, sb, n_base, m0 + j0);
+          bulk_commit_group();
+        }
+        buf ^= 1;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[b]);
+      if (++b == 2) { b = 0; ph_b ^= 1u; }
+    }
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major 2-D tensor [rows][cols] of `esize`-byte elements.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int cols,
+              int rows, int box_cols, int box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * esize};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <class C>
+cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
+                     const EpilogueArgs& ep, void* out, cudaStream_t st) {
+  CUtensorMap tm_w, tm_x, tm_out;
+  bool ok = make_map(&tm_w, qw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, C::BK / 2, C::BM,
+                     CU_TENSOR_MAP_SWIZZLE_64B);
+  if (C::ACT_BITS == 8)
+    ok = ok && make_map(&tm_x, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, C::BK, C::BN,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    ok = ok && make_map(&tm_x, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, C::BK / 2, C::BN,
+                        CU_TENSOR_MAP_SWIZZLE_64B);
+  if (C::OUT_S32)
+    ok = ok && make_map(&tm_out, out, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, N, M, 32, C::EPI_CHUNK,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+  else
+    ok = ok && make_map(&tm_out, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 32, C::EPI_CHUNK,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!ok) return cudaErrorInvalidValue;
+
+  TileArgs a;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.tiles_m = (M + C::BN - 1) / C::BN;
+  a.tiles_n = (N + C::BM - 1) / C::BM;
+  a.num_tiles = a.tiles_m * a.tiles_n;
+  // Keep the smaller operand resident in L2: sweep output channels fastest when
+  // the packed weights fit comfortably, so each activation tile streams once.
+  a.n_fastest = (static_cast<size_t>(N) * K / 2) <= (48u << 20) ? 1 : 0;
+  a.ep = ep;
+
+  static bool attr_set = false;  // per template instance
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int grid = a.num_tiles < sm_count() ? a.num_tiles : sm_count();
+  gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tm_w, tm_x, tm_out, a);
+  return cudaGetLastError();
+}
+
+template <int ACT_BITS, bool OUT_S32>
+cudaError_t dispatch_bn(const void* qx, const uint8_t* qw, int M, int N, int K,
+                        const EpilogueArgs& ep, void* out, cudaStream_t st) {
+  if (M <= 16) return run_gemm<Cfg<16, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, st);
+  if (M <= 32) return run_gemm<Cfg<32, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, st);
+  if (M <= 64) return run_gemm<Cfg<64, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, st);
+  if (M <= 128) return run_gemm<Cfg<128, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, st);
+  return run_gemm<Cfg<256, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, st);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const void* qx, int act_bits, const uint8_t* qw, int M, int N, int K,
+                        const EpilogueArgs& ep, void* out, bool out_s32, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  if (act_bits == 8)
+    return out_s32 ? dispatch_bn<8, true>(qx, qw, M, N, K, ep, out, st)
+                   : dispatch_bn<8, false>(qx, qw, M, N, K, ep, out, st);
+  return out_s32 ? dispatch_bn<4, true>(qx, qw, M, N, K, ep, out, st)
+                 : dispatch_bn<4, false>(qx, qw, M, N, K, ep, out, st);
+}
+
+}  // namespace wq

@@ -1,0 +1,236 @@
+// Quantization kernels of the fused low-bit linear (SteerQuant / Rudder):
+//   act_quant     the first Rudder kernel (SteerQuant §4.4): per-token quantization
+//                 with the shared channel scale (§4.2) and the per-(step, stream)
+//                 clip ratio from the layer-step table (§4.3) folded in
+//   pack_int4     offline weight preparation (Figure 2): W' = W * c, one symmetric
+//                 int4 code matrix with per-output-channel scales
+//   channel_scale the shared diagonal c[k] = sqrt(max|x_cal[:,k]| / max|W[:,k]|)
+//                 (SmoothQuant-style equivalent scaling, cited in §2)
+//
+// All arithmetic that decides a code is IEEE binary32 with round-to-nearest-even:
+// explicit __fmul_rn / __fdiv_rn / __fsqrt_rn intrinsics, no contraction, no
+// fast-math, so codes and scales are reproducible bit for bit.
+#pragma once
+#include <cuda_bf16.h>
+
+#include "wq_internal.h"
+#include "wq_ptx.cuh"
+
+namespace wq {
+namespace {
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+template <int QMAX>
+__device__ __forceinline__ int quantize(float v, float s) {
+  if (s == 0.0f) return 0;
+  int q = __float2int_rn(__fdiv_rn(v, s));  // saturating convert, ties to even
+  q = q > QMAX ? QMAX : q;
+  q = q < -QMAX ? -QMAX : q;
+  return q;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+// One token row per TPR threads; each thread holds CPT chunks of 8 channels in
+// registers, so x is read from HBM exactly once.
+template <int ACT_BITS, int TPR, int CPT>
+__global__ void __launch_bounds__(256) act_quant_kernel(
+    const uint16_t* __restrict__ x, int M, int K, const float* __restrict__ cinv,
+    const uint8_t* __restrict__ stream_id, const float* __restrict__ alpha, int S, int step,
+    void* __restrict__ qx, float* __restrict__ s_tok) {
+  constexpr int RPC = 256 / TPR;  // rows per CTA
+  constexpr int WPR = TPR / 32;   // warps per row
+  constexpr int QMAX = ACT_BITS == 8 ? 127 : 7;
+  __shared__ float red[8];
+
+  const int local_row = threadIdx.x / TPR;
+  const int t = threadIdx.x % TPR;
+  const int row = blockIdx.x * RPC + local_row;
+  const bool row_ok = row < M;
+  const int nchunk = K >> 3;
+
+  float v[CPT][8];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = t + i * TPR;
+    if (row_ok && c < nchunk) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x + (size_t)row * K) + c);
+      float ci[8];
+      if (cinv != nullptr) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(cinv) + 2 * c);
+        const float4 b = __ldg(reinterpret_cast<const float4*>(cinv) + 2 * c + 1);
+        ci[0] = a.x; ci[1] = a.y; ci[2] = a.z; ci[3] = a.w;
+        ci[4] = b.x; ci[5] = b.y; ci[6] = b.z; ci[7] = b.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ci[e] = 1.0f;
+      }
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[i][2 * e] = __fmul_rn(bf16lo(w[e]), ci[2 * e]);
+        v[i][2 * e + 1] = __fmul_rn(bf16hi(w[e]), ci[2 * e + 1]);
+        amax = fmaxf(amax, fmaxf(fabsf(v[i][2 * e]), fabsf(v[i][2 * e + 1])));
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[i][e] = 0.0f;
+    }
+  }
+  amax = warp_max(amax);
+  if constexpr (WPR > 1) {
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < WPR; ++j) amax = fmaxf(amax, red[local_row * WPR + j]);
+  }
+  if (!row_ok) return;
+
+  float s = 0.0f;
+  const int sid = stream_id[row];
+  if (sid < S) {
+    const float clip = __fmul_rn(__ldg(alpha + step * S + sid), amax);
+    s = __fdiv_rn(clip, static_cast<float>(QMAX));
+  } else if (t == 0) {
+    raise_error(kErrBadStreamId);
+  }
+  if (t == 0) s_tok[row] = s;
+
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = t + i * TPR;
+    if (c >= nchunk) continue;
+    int q[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) q[e] = quantize<QMAX>(v[i][e], s);
+    if constexpr (ACT_BITS == 8) {
+      uint2 o;
+      o.x = (q[0] & 0xFF) | ((q[1] & 0xFF) << 8) | ((q[2] & 0xFF) << 16) | ((uint32_t)q[3] << 24);
+      o.y = (q[4] & 0xFF) | ((q[5] & 0xFF) << 8) | ((q[6] & 0xFF) << 16) | ((uint32_t)q[7] << 24);
+      reinterpret_cast<uint2*>(static_cast<int8_t*>(qx) + (size_t)row * K)[c] = o;
+    } else {
+      uint32_t o = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o |= (uint32_t)(q[e] & 0xF) << (4 * e);
+      reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(qx) + (size_t)row * (K / 2))[c] = o;
+    }
+  }
+}
+
+template <int ACT_BITS, int TPR, int CPT>
+cudaError_t run_act_quant(const uint16_t* x, int M, int K, const float* cinv,
+                          const uint8_t* sid, const float* alpha, int S, int step, void* qx,
+                          float* s_tok, cudaStream_t st) {
+  constexpr int RPC = 256 / TPR;
+  const int grid = (M + RPC - 1) / RPC;
+  act_quant_kernel<ACT_BITS, TPR, CPT>
+      <<<grid, 256, 0, st>>>(x, M, K, cinv, sid, alpha, S, step, qx, s_tok);
+  return cudaGetLastError();
+}
+
+template <int ACT_BITS>
+cudaError_t dispatch_act_quant(const uint16_t* x, int M, int K, const float* cinv,
+                               const uint8_t* sid, const float* alpha, int S, int step,
+                               void* qx, float* s_tok, cudaStream_t st) {
+  const int nchunk = K / 8;
+#define WQ_AQ(TPR, CPT) \
+  return run_act_quant<ACT_BITS, TPR, CPT>(x, M, K, cinv, sid, alpha, S, step, qx, s_tok, st)
+  if (nchunk <= 32) WQ_AQ(32, 1);
+  if (nchunk <= 64) WQ_AQ(64, 1);
+  if (nchunk <= 128) WQ_AQ(128, 1);
+  if (nchunk <= 256) WQ_AQ(256, 1);
+  if (nchunk <= 512) WQ_AQ(256, 2);
+  if (nchunk <= 1024) WQ_AQ(256, 4);
+  if (nchunk <= 2048) WQ_AQ(256, 8);
+  WQ_AQ(256, 16);
+#undef WQ_AQ
+}
+
+// ------------------------------------------------------------ offline weights
+
+__device__ __forceinline__ float block_max_256(float v, float* red) {
+  v = warp_max(v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int j = 1; j < 8; ++j) r = fmaxf(r, red[j]);
+  __syncthreads();
+  return r;
+}
+
+// One CTA per output channel n: s_w[n] = max_k |W[n,k]*c[k]| / 7, codes packed
+// two per byte (low nibble = even k).
+__global__ void __launch_bounds__(256) pack_int4_kernel(const uint16_t* __restrict__ W,
+                                                        const float* __restrict__ c, int K,
+                                                        uint8_t* __restrict__ qw,
+                                                        float* __restrict__ s_w) {
+  __shared__ float red[8];
+  const int n = blockIdx.x;
+  const uint16_t* row = W + (size_t)n * K;
+  float amax = 0.0f;
+  for (int k = threadIdx.x; k < K; k += 256) {
+    const float w = __fmul_rn(__uint_as_float((uint32_t)row[k] << 16), c ? c[k] : 1.0f);
+    amax = fmaxf(amax, fabsf(w));
+  }
+  amax = block_max_256(amax, red);
+  const float s = __fdiv_rn(amax, 7.0f);
+  if (threadIdx.x == 0) s_w[n] = s;
+  for (int j = threadIdx.x; j < K / 2; j += 256) {
+    const int k = 2 * j;
+    const float w0 = __fmul_rn(__uint_as_float((uint32_t)row[k] << 16), c ? c[k] : 1.0f);
+    const float w1 = __fmul_rn(__uint_as_float((uint32_t)row[k + 1] << 16), c ? c[k + 1] : 1.0f);
+    const int q0 = quantize<7>(w0, s), q1 = quantize<7>(w1, s);
+    qw[(size_t)n * (K / 2) + j] = (uint8_t)((q0 & 0xF) | ((q1 & 0xF) << 4));
+  }
+}
+
+// One thread per input channel k: column maxima over the calibration batch and
+// over the weight rows, then c = sqrt(a / b) (1 when either maximum is 0).
+__global__ void channel_scale_kernel(const uint16_t* __restrict__ x_cal, int Mcal,
+                                     const uint16_t* __restrict__ W, int N, int K,
+                                     float* __restrict__ c, float* __restrict__ cinv) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= K) return;
+  float a = 0.0f, b = 0.0f;
+  for (int m = 0; m < Mcal; ++m)
+    a = fmaxf(a, fabsf(__uint_as_float((uint32_t)x_cal[(size_t)m * K + k] << 16)));
+  for (int n = 0; n < N; ++n)
+    b = fmaxf(b, fabsf(__uint_as_float((uint32_t)W[(size_t)n * K + k] << 16)));
+  float ck = 1.0f;
+  if (a > 0.0f && b > 0.0f) ck = __fsqrt_rn(__fdiv_rn(a, b));
+  c[k] = ck;
+  cinv[k] = __fdiv_rn(1.0f, ck);
+}
+
+}  // namespace
+
+cudaError_t launch_act_quant(const uint16_t* x, int M, int K, const float* cinv,
+                             const uint8_t* stream_id, const float* alpha, int S, int step,
+                             int act_bits, void* qx, float* s_tok, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  if (act_bits == 8)
+    return dispatch_act_quant<8>(x, M, K, cinv, stream_id, alpha, S, step, qx, s_tok, st);
+  return dispatch_act_quant<4>(x, M, K, cinv, stream_id, alpha, S, step, qx, s_tok, st);
+}
+
+cudaError_t launch_pack_int4(const uint16_t* W, const float* c, int N, int K, uint8_t* qw,
+                             float* s_w, cudaStream_t st) {
+  pack_int4_kernel<<<N, 256, 0, st>>>(W, c, K, qw, s_w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_channel_scale(const uint16_t* x_cal, int Mcal, const uint16_t* W, int N,
+                                 int K, float* c, float* cinv, cudaStream_t st) {
+  channel_scale_kernel<<<(K + 127) / 128, 128, 0, st>>>(x_cal, Mcal, W, N, K, c, cinv);
+  return cudaGetLastError();
+}
+
+}  // namespace wq

@@ -1,0 +1,153 @@
+/*
+ * wq.h -- C ABI of the fused low-bit (W4A8 / W4A4) linear layer of SteerQuant's
+ * Rudder kernels, for NVIDIA B200 (sm_100a).
+ *
+ * Source: "SteerQuant: Steering Quantization Error with Action-Guided Scaling in
+ * World-Action Models" (paperlayer.ai abstract page 2609.39056v1), cited below by
+ * section.  The method keeps ONE static int4 weight matrix per layer (§1, §4.2,
+ * Figure 2) and, per layer and denoising step, a lookup table of activation clip
+ * settings per token stream (video / proprio / action; §4.3).  Rudder runs two
+ * fused kernels (§4.4): (1) activation quantization with the channel scaling and
+ * stream gains folded in, (2) a low-bit GEMM whose epilogue applies
+ * dequantization, inverse-gain compensation, bias and output compensation (§1).
+ * Only integer activations and per-row scales pass between the two kernels.
+ *
+ * Arithmetic contract (readings where the pages are silent):
+ *   x'[m,k]  = fp32(x[m,k]) * cinv[k]                        (fp32, no rounding to bf16)
+ *   amax[m]  = max_k |x'[m,k]|
+ *   s_tok[m] = (alpha[step][sid] * amax[m]) / qmax            qmax = 127 (A8) or 7 (A4)
+ *   q[m,k]   = clamp(rint_half_even(x'[m,k] / s_tok[m]), -qmax, qmax)   (IEEE fp32 divide)
+ *   acc[m,n] = sum_k q[m,k] * qw[n,k]                          (int32)
+ *   y[m,n]   = bf16( s_tok[m]*s_w[n]*acc[m,n] + bias[n] + beta[step][sid][n] )
+ * with sid = stream_id[m].  The stream gain is carried as the clip ratio
+ * alpha = 1/gain, so the inverse-gain compensation lives inside s_tok.  A row
+ * whose scale is 0 gets all-zero codes.  Codes, scales and accumulators are
+ * exactly reproducible; y is computed in fp32 (one rounding to bf16 at the end).
+ *
+ * Packed int4 layout (weights and 4-bit activations): two's-complement nibbles,
+ * two per byte, the LOW nibble holds the even k.  Row-major, K/2 bytes per row.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never frees or retains them.  Row-major, densely packed.
+ *   - bf16 tensors are passed as raw 16-bit patterns (wq_bf16).
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream).
+ *     Argument errors are returned synchronously before anything is launched.
+ *   - Nothing throws or aborts across this boundary.
+ *   - Preconditions checked on the host: M >= 0 (M == 0 is a no-op), K a
+ *     multiple of 128 with 128 <= K <= 32768, N a multiple of 16 and >= 16,
+ *     1 <= S <= 255, T >= 1, 0 <= step < T, act_bits in {4, 8}, every tensor
+ *     pointer 16-byte aligned, the workspace at least wq_workspace_bytes().
+ *   - Precondition checked on the device: stream_id[m] < S.  A violation gives
+ *     that row scale 0 and sets WQ_DEVICE_ERR_STREAM_ID (see wq_device_status).
+ *   - Inputs must be finite; alpha entries must be positive.
+ */
+#ifndef WQ_H
+#define WQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* wq_stream_t; /* identical to cudaStream_t */
+typedef uint16_t wq_bf16;                /* raw bfloat16 bit pattern */
+
+typedef enum {
+  WQ_OK = 0,
+  WQ_ERR_NULL = 1,    /* a required pointer is NULL */
+  WQ_ERR_SHAPE = 2,   /* M, N or K outside the supported range */
+  WQ_ERR_ALIGN = 3,   /* a tensor pointer is not 16-byte aligned */
+  WQ_ERR_ARG = 4,     /* bad act_bits, S, T, step, or workspace too small */
+  WQ_ERR_CUDA = 5,    /* the CUDA runtime rejected a launch */
+  WQ_ERR_TIMEOUT = 6, /* wq_device_status: a kernel's bounded wait gave up */
+  WQ_ERR_DEVICE = 7   /* wq_device_status: a device-side precondition failed */
+} wq_status;
+
+/* Device error bits reported by wq_device_status(). */
+#define WQ_DEVICE_ERR_TIMEOUT 1u
+#define WQ_DEVICE_ERR_STREAM_ID 2u
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* wq_status_string(wq_status s);
+
+/* ABI version of this library (major * 100 + minor). */
+int wq_version(void);
+
+/* Bytes of device workspace wq_linear_w4a8 / wq_linear_w4a4 need for M token
+ * rows, K input channels, N output channels: the integer activation codes
+ * (M*K bytes for A8, M*K/2 for A4) and the per-token scales (4*M bytes), each
+ * rounded up to 256 bytes.  Returns 0 for invalid sizes. */
+size_t wq_workspace_bytes(int M, int K, int N, int act_bits);
+
+/* §4.2 (calibration side of the shared diagonal D): for each input channel k,
+ * c[k] = sqrt(max_m |x_cal[m,k]| / max_n |W[n,k]|), 1 when either maximum is 0,
+ * and cinv[k] = 1 / c[k], both IEEE fp32 correctly rounded.
+ *   x_cal [Mcal][K] bf16 calibration activations; W [N][K] bf16 weights;
+ *   c, cinv [K] fp32 outputs.  Offline (run once per layer). */
+wq_status wq_channel_scale(const wq_bf16* x_cal, int Mcal, const wq_bf16* W, int N, int K,
+                           float* c, float* cinv, wq_stream_t stream);
+
+/* Figure 2 / §4.2 / §3.1: offline weight preparation.  W' = W * c (c may be
+ * NULL, meaning 1), s_w[n] = max_k |W'[n,k]| / 7, qw = clamp(rint(W'/s_w), -7, 7)
+ * packed two per byte.
+ *   W [N][K] bf16 in; qw [N][K/2] uint8 out; s_w [N] fp32 out. */
+wq_status wq_pack_int4(const wq_bf16* W, const float* c, int N, int K, uint8_t* qw,
+                       float* s_w, wq_stream_t stream);
+
+/* §4.4 first kernel: per-token activation quantization with the channel scale
+ * (§4.2) and the (step, stream) clip ratio (§4.3) folded in.
+ *   x [M][K] bf16; cinv [K] fp32 or NULL (= 1); stream_id [M] uint8;
+ *   alpha [T][S] fp32 clip ratios; step in [0, T).
+ *   act_bits 8: qx is int8 [M][K]; act_bits 4: qx is packed uint8 [M][K/2].
+ *   s_tok [M] fp32 out. */
+wq_status wq_act_quant(const wq_bf16* x, int M, int K, const float* cinv,
+                       const uint8_t* stream_id, const float* alpha, int S, int T, int step,
+                       int act_bits, void* qx, float* s_tok, wq_stream_t stream);
+
+/* §4.4 second kernel on already-quantized activations: GEMM with int32
+ * accumulation on tcgen05 tensor cores and the fused epilogue.
+ *   qx: int8 [M][K] (act_bits 8) or packed [M][K/2] (act_bits 4); s_tok [M];
+ *   stream_id [M]; beta [T][S][N] fp32 or NULL; qw [N][K/2]; s_w [N];
+ *   bias [N] fp32 or NULL; y [M][N] bf16 out. */
+wq_status wq_gemm_w4ax(const void* qx, const float* s_tok, int act_bits, int M, int K, int N,
+                       const uint8_t* stream_id, const float* beta, int S, int T, int step,
+                       const uint8_t* qw, const float* s_w, const float* bias, wq_bf16* y,
+                       wq_stream_t stream);
+
+/* The fused W4A8 linear: wq_act_quant (8-bit) then wq_gemm_w4ax, with the codes
+ * and token scales kept in the caller's workspace (device memory of at least
+ * wq_workspace_bytes(M, K, N, 8) bytes, 256-byte aligned; its contents are
+ * overwritten).  Arguments as in the two calls above. */
+wq_status wq_linear_w4a8(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                         const uint8_t* stream_id, const float* alpha, const float* beta,
+                         int S, int T, int step, const uint8_t* qw, const float* s_w,
+                         const float* bias, wq_bf16* y, void* workspace, size_t ws_bytes,
+                         wq_stream_t stream);
+
+/* The fused W4A4 linear: as wq_linear_w4a8 with 4-bit activation codes
+ * (workspace of wq_workspace_bytes(M, K, N, 4) bytes). */
+wq_status wq_linear_w4a4(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                         const uint8_t* stream_id, const float* alpha, const float* beta,
+                         int S, int T, int step, const uint8_t* qw, const float* s_w,
+                         const float* bias, wq_bf16* y, void* workspace, size_t ws_bytes,
+                         wq_stream_t stream);
+
+/* Debug view of the GEMM's integer core: the same tensor-core mainloop with the
+ * epilogue replaced by a raw store of the int32 accumulators acc [M][N]. */
+wq_status wq_debug_gemm_s32(const void* qx, int act_bits, const uint8_t* qw, int M, int N,
+                            int K, int32_t* acc, wq_stream_t stream);
+
+/* Reads and clears the device error word of the current device (synchronizes
+ * the device).  *flags receives the WQ_DEVICE_ERR_* bits seen since the last
+ * call (may be NULL).  Returns WQ_OK, WQ_ERR_TIMEOUT, WQ_ERR_DEVICE or
+ * WQ_ERR_CUDA. */
+wq_status wq_device_status(unsigned* flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H */

@@ -1,0 +1,79 @@
+"""Helpers shared by the GPU tests: moving numpy arrays to and from the device,
+running the library's entry points, and comparing with the oracle."""
+import numpy as np
+import torch
+
+import activation_quantized_gemm_wq_b200 as wq
+
+
+def dev(a):
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).cuda()
+
+
+def host(t, dtype=None):
+    a = t.detach().cpu().numpy()
+    if dtype is not None:
+        a = a.view(dtype)
+    return a
+
+
+def bf16_to_f64(bits):
+    return (np.asarray(bits).view(np.uint16).astype(np.uint32) << 16).view(np.float32).astype(
+        np.float64)
+
+
+def within_tolerance(y_bits, ref_bits):
+    """max |y - y_ref| <= 2^-7 |y_ref| + 1e-3 rms(y_ref), element-wise; returns
+    (ok, worst ratio of error to allowance)."""
+    y = bf16_to_f64(y_bits)
+    ref = bf16_to_f64(ref_bits)
+    rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
+    allow = 2.0 ** -7 * np.abs(ref) + 1e-3 * rms
+    err = np.abs(y - ref)
+    worst = float(np.max(err / np.maximum(allow, 1e-300))) if ref.size else 0.0
+    return bool(np.all(err <= allow)), worst
+
+
+def gpu_prep(W, x_cal):
+    """Channel scale and packed weights computed on the GPU."""
+    N, K = W.shape
+    c = torch.empty(K, dtype=torch.float32, device="cuda")
+    cinv = torch.empty_like(c)
+    qw = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+    s_w = torch.empty(N, dtype=torch.float32, device="cuda")
+    dW = dev(W)
+    wq.wq_channel_scale(dev(x_cal), dW, c, cinv)
+    wq.wq_pack_int4(dW, c, qw, s_w)
+    return c, cinv, qw, s_w
+
+
+def gpu_act_quant(x, cinv, sid, alpha, step, bits):
+    M, K = x.shape
+    qx = torch.empty((M, K) if bits == 8 else (M, K // 2),
+                     dtype=torch.int8 if bits == 8 else torch.uint8, device="cuda")
+    s_tok = torch.empty(M, dtype=torch.float32, device="cuda")
+    wq.wq_act_quant(dev(x), None if cinv is None else dev(cinv), dev(sid), dev(alpha), step, bits,
+                    qx, s_tok)
+    return host(qx), host(s_tok)
+
+
+def gpu_linear(x, cinv, sid, alpha, beta, step, bits, qw, s_w, bias):
+    """The fused linear through the C ABI; qw/s_w/cinv may be numpy or device tensors."""
+    M, K = x.shape
+    N = qw.shape[0]
+    t = lambda a: None if a is None else (a if isinstance(a, torch.Tensor) else dev(a))
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = wq.alloc_workspace(M, K, N, bits)
+    fn = wq.wq_linear_w4a8 if bits == 8 else wq.wq_linear_w4a4
+    fn(t(x), t(cinv), t(sid), t(alpha), t(beta), step, t(qw), t(s_w), t(bias), y, ws)
+    return host(y.view(torch.int16), np.uint16)
+
+
+def gpu_gemm_s32(qx, bits, qw, K):
+    M, N = qx.shape[0], qw.shape[0]
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    wq.wq_debug_gemm_s32(dev(qx), bits, dev(qw), K, acc)
+    return host(acc)

@@ -1,0 +1,84 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry point
+include/wq.h declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import activation_quantized_gemm_wq_b200 as wq
+from activation_quantized_gemm_wq_b200 import build as wq_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "wq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(wq_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if wq_build.needs_build():
+        wq_build.build()
+    return wq.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), f"libwq.so does not export {n}"
+        assert n in wq._SIGS, f"binding has no signature for {n}"
+    assert set(wq._SIGS) == set(names)
+
+
+def test_status_strings_and_version(lib):
+    assert wq.wq_version() == 100
+    for code, name in wq.STATUS.items():
+        assert lib.wq_status_string(code).decode().startswith(name)
+
+
+def test_workspace_bytes(lib):
+    assert wq.wq_workspace_bytes(4288, 2048, 6144, 8) == 4288 * 2048 + 17152
+    assert wq.wq_workspace_bytes(4288, 2048, 6144, 4) == 4288 * 1024 + 17152
+    assert wq.wq_workspace_bytes(1, 128, 16, 8) == 256 + 256
+    assert wq.wq_workspace_bytes(64, 100, 256, 8) == 0      # K not a multiple of 128
+    assert wq.wq_workspace_bytes(64, 256, 250, 8) == 0      # N not a multiple of 16
+    assert wq.wq_workspace_bytes(64, 256, 256, 6) == 0      # bits
+
+
+FAKE = 1 << 20          # a 16-byte aligned, never dereferenced address
+MIS = FAKE + 8
+
+
+def _linear(lib, **kw):
+    a = dict(x=FAKE, M=64, K=256, N=256, cinv=FAKE, sid=FAKE, alpha=FAKE, beta=FAKE, S=3, T=1,
+             step=0, qw=FAKE, s_w=FAKE, bias=FAKE, y=FAKE, ws=FAKE, ws_bytes=1 << 30, st=None)
+    a.update(kw)
+    return lib.wq_linear_w4a8(a["x"], a["M"], a["K"], a["N"], a["cinv"], a["sid"], a["alpha"],
+                              a["beta"], a["S"], a["T"], a["step"], a["qw"], a["s_w"], a["bias"],
+                              a["y"], a["ws"], a["ws_bytes"], a["st"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(K=100), 2), (dict(K=0), 2), (dict(K=65536), 2), (dict(N=250), 2), (dict(N=0), 2),
+    (dict(M=-1), 2), (dict(x=None), 1), (dict(qw=None), 1), (dict(alpha=None), 1),
+    (dict(ws=None), 1), (dict(x=MIS), 3), (dict(y=MIS), 3), (dict(ws=FAKE + 16), 3),
+    (dict(step=1), 4), (dict(step=-1), 4), (dict(S=0), 4), (dict(S=256), 4), (dict(T=0), 4),
+    (dict(ws_bytes=100), 4),
+])
+def test_linear_rejects_bad_arguments_on_host(lib, kw, code):
+    assert _linear(lib, **kw) == code
+
+
+def test_other_entry_points_reject_on_host(lib):
+    assert lib.wq_act_quant(FAKE, 8, 256, None, FAKE, FAKE, 3, 1, 0, 6, FAKE, FAKE, None) == 4
+    assert lib.wq_act_quant(FAKE, 8, 200, None, FAKE, FAKE, 3, 1, 0, 8, FAKE, FAKE, None) == 2
+    assert lib.wq_pack_int4(FAKE, None, 16, 96, FAKE, FAKE, None) == 2
+    assert lib.wq_pack_int4(None, None, 16, 128, FAKE, FAKE, None) == 1
+    assert lib.wq_debug_gemm_s32(FAKE, 8, FAKE, 16, 24, 128, FAKE, None) == 2
+    assert lib.wq_gemm_w4ax(FAKE, FAKE, 4, 16, 128, 32, FAKE, None, 3, 2, 2, FAKE, FAKE, None,
+                            FAKE, None) == 4
+    assert lib.wq_channel_scale(None, 4, FAKE, 4, 128, FAKE, FAKE, None) == 1
