@@ -1,7 +1,7 @@
 // C ABI of libwq (declared in include/wq.h): host-side validation, workspace
 // layout and launches.  The whole library is this one translation unit; the
 // kernels live in the included .cuh files.
-#include "../../include/wq.h"
+#include "wq.h"
 
 #include <cstdint>
 
@@ -48,6 +48,7 @@ wq_status gemm_checks(const void* qx, const float* s_tok, int act_bits, int M, i
   WQ_TRY(check_mk(M, K));
   WQ_TRY(check_n(N));
   WQ_TRY(check_table(S, T, step));
+  if (M == 0) return WQ_OK;
   if (!qx || !s_tok || !stream_id || !qw || !s_w || !y) return WQ_ERR_NULL;
   if (!aligned16(qx) || !aligned16(qw) || !aligned16(y) || !aligned16(s_tok) ||
       !aligned16(s_w) || (bias && !aligned16(bias)) || (beta && !aligned16(beta)))
@@ -62,14 +63,13 @@ wq_status linear(const wq_bf16* x, int M, int K, int N, const float* cinv,
   WQ_TRY(check_mk(M, K));
   WQ_TRY(check_n(N));
   WQ_TRY(check_table(S, T, step));
-  if (!x || !stream_id || !alpha || !qw || !s_w || !y || (!workspace && M > 0))
-    return WQ_ERR_NULL;
+  if (M == 0) return WQ_OK;  // empty batch: token tensors may be NULL
+  if (!x || !stream_id || !alpha || !qw || !s_w || !y || !workspace) return WQ_ERR_NULL;
   if (!aligned16(x) || !aligned16(qw) || !aligned16(y) || !aligned16(s_w) ||
       (cinv && !aligned16(cinv)) || (bias && !aligned16(bias)) || (beta && !aligned16(beta)) ||
       (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
     return WQ_ERR_ALIGN;
   if (ws_bytes < wq_workspace_bytes(M, K, N, act_bits)) return WQ_ERR_ARG;
-  if (M == 0) return WQ_OK;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* qx = ws;
   float* s_tok = reinterpret_cast<float*>(ws + round_up(act_bytes(M, K, act_bits)));
@@ -130,6 +130,7 @@ wq_status wq_act_quant(const wq_bf16* x, int M, int K, const float* cinv,
   if (act_bits != 8 && act_bits != 4) return WQ_ERR_ARG;
   WQ_TRY(check_mk(M, K));
   WQ_TRY(check_table(S, T, step));
+  if (M == 0) return WQ_OK;
   if (!x || !stream_id || !alpha || !qx || !s_tok) return WQ_ERR_NULL;
   if (!aligned16(x) || !aligned16(qx) || (cinv && !aligned16(cinv))) return WQ_ERR_ALIGN;
   return from_cuda(wq::launch_act_quant(x, M, K, cinv, stream_id, alpha, S, step, act_bits, qx,
@@ -170,6 +171,7 @@ wq_status wq_debug_gemm_s32(const void* qx, int act_bits, const uint8_t* qw, int
   if (act_bits != 8 && act_bits != 4) return WQ_ERR_ARG;
   WQ_TRY(check_mk(M, K));
   WQ_TRY(check_n(N));
+  if (M == 0) return WQ_OK;
   if (!qx || !qw || !acc) return WQ_ERR_NULL;
   if (!aligned16(qx) || !aligned16(qw) || !aligned16(acc)) return WQ_ERR_ALIGN;
   const wq::EpilogueArgs ep{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 0};

@@ -48,7 +48,8 @@ struct Cfg {
   static constexpr int BM = 128;  // output channels per tile (MMA M)
   static constexpr int BK = 128;  // K elements per pipeline stage
   static constexpr int UNPACK_WARPS = ACT_BITS == 4 ? 8 : 4;
-  static constexpr int EPI_WARPS = 4;
+  static constexpr int EPI_WARPS = 8;  // two per TMEM lane quadrant
+  static constexpr int EPI_THREADS = EPI_WARPS * 32;
   static constexpr int FIRST_UNPACK_WARP = 2;
   static constexpr int FIRST_EPI_WARP = FIRST_UNPACK_WARP + UNPACK_WARPS;
   static constexpr int NUM_WARPS = FIRST_EPI_WARP + EPI_WARPS;
@@ -61,27 +62,31 @@ struct Cfg {
   static constexpr int STAGE_BYTES = WP_BYTES + XS_BYTES;
   static constexpr int NU = 2;  // unpacked buffers
   static constexpr int EPI_ELEM = OUT_S32 ? 4 : 2;
-  static constexpr int EPI_CHUNK = BN < 32 ? BN : 32;  // token columns per TMEM load
+  static constexpr int EPI_CHUNK = 16;  // token columns per TMEM load / TMA store
+  static constexpr int NUM_CHUNKS = BN / EPI_CHUNK;
   static constexpr int EPI_BUF_BYTES = EPI_CHUNK * 32 * EPI_ELEM;
   static constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BUF_BYTES;
+  static constexpr int TOK_BYTES = 2 * BN * 4 + 2 * BN;  // staged s_tok and stream ids, x2
   static constexpr int SMEM_LIMIT = 232448;  // 227 KB opt-in per CTA
   static constexpr int RESERVED = 1024 /*alignment slack*/ + 512 /*barriers*/;
   static constexpr int NS_FIT =
-      (SMEM_LIMIT - RESERVED - NU * (WU_BYTES + XU_BYTES) - EPI_BYTES) / STAGE_BYTES;
+      (SMEM_LIMIT - RESERVED - NU * (WU_BYTES + XU_BYTES) - EPI_BYTES - TOK_BYTES) / STAGE_BYTES;
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
   static_assert(NS >= 2, "pipeline needs at least two stages");
+  static_assert(BN % EPI_CHUNK == 0 && NUM_CHUNKS >= 1, "token tile is a multiple of 16");
 
   static constexpr int OFF_WP = 0;
   static constexpr int OFF_XS = OFF_WP + NS * WP_BYTES;
   static constexpr int OFF_WU = OFF_XS + NS * XS_BYTES;
   static constexpr int OFF_XU = OFF_WU + NU * WU_BYTES;
   static constexpr int OFF_EPI = OFF_XU + NU * XU_BYTES;
-  static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
-  static constexpr int NUM_BARS = 2 * NS + 2 * NU + 4;
+  static constexpr int OFF_TOK = OFF_EPI + EPI_BYTES;
+  static constexpr int OFF_BAR = OFF_TOK + TOK_BYTES;
+  static constexpr int NUM_BARS = 2 * NS + 2 * NU + 6;
   static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
   static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
   static_assert(OFF_XS % 1024 == 0 && XS_BYTES % 512 == 0 && OFF_WU % 1024 == 0 &&
-                    OFF_XU % 1024 == 0 && OFF_EPI % 1024 == 0,
+                    OFF_XU % 1024 == 0 && OFF_EPI % 1024 == 0 && OFF_BAR % 8 == 0,
                 "swizzled tiles need 1024-byte alignment");
 
   static constexpr uint32_t TMEM_COLS =
@@ -118,19 +123,33 @@ __device__ __forceinline__ void unpack32(const uint4 p, uint4& lo16, uint4& hi16
   hi16 = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// Packed tile [rows][64 B] with the 64-byte swizzle -> int8 tile [rows][128 B]
-// with the 128-byte swizzle.  Task i covers row i/4, packed 16-byte chunk i%4.
-__device__ __forceinline__ void unpack_tile(const uint8_t* src, uint8_t* dst, int rows,
-                                            int tid, int nthreads) {
-  for (int i = tid; i < rows * 4; i += nthreads) {
-    const int r = i >> 2, p = i & 3;
-    const uint4 v =
-        *reinterpret_cast<const uint4*>(src + r * 64 + ((p ^ ((r >> 1) & 3)) << 4));
-    uint4 lo, hi;
-    unpack32(v, lo, hi);
-    uint8_t* row = dst + r * 128;
-    *reinterpret_cast<uint4*>(row + (((2 * p) ^ (r & 7)) << 4)) = lo;
-    *reinterpret_cast<uint4*>(row + (((2 * p + 1) ^ (r & 7)) << 4)) = hi;
+// Packed tile [ROWS][64 B] with the 64-byte swizzle -> int8 tile [ROWS][128 B]
+// with the 128-byte swizzle.  Task i covers row i/4, packed 16-byte chunk i%4;
+// each thread issues all of its loads before converting (latency hiding).
+template <int ROWS, int NT>
+__device__ __forceinline__ void unpack_tile(const uint8_t* src, uint8_t* dst, int tid) {
+  constexpr int TASKS = ROWS * 4;
+  constexpr int PER = (TASKS + NT - 1) / NT;
+  uint4 v[PER];
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int i = tid + k * NT;
+    if (TASKS % NT == 0 || i < TASKS) {
+      const int r = i >> 2, p = i & 3;
+      v[k] = *reinterpret_cast<const uint4*>(src + r * 64 + ((p ^ ((r >> 1) & 3)) << 4));
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int i = tid + k * NT;
+    if (TASKS % NT == 0 || i < TASKS) {
+      const int r = i >> 2, p = i & 3;
+      uint4 lo, hi;
+      unpack32(v[k], lo, hi);
+      uint8_t* row = dst + r * 128;
+      *reinterpret_cast<uint4*>(row + (((2 * p) ^ (r & 7)) << 4)) = lo;
+      *reinterpret_cast<uint4*>(row + (((2 * p + 1) ^ (r & 7)) << 4)) = hi;
+    }
   }
 }
 
@@ -147,7 +166,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* uempty = ufull + C::NU;
   uint64_t* tfull = uempty + C::NU;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* tokbar = tempty + 2;  // epilogue warps: token staging of buffer i complete
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tokbar + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -165,6 +185,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], C::EPI_WARPS);
+      mbar_init(&tokbar[b], C::EPI_WARPS);
     }
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -262,11 +283,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           ok = false;
           break;
         }
-        unpack_tile(smem + C::OFF_WP + s * C::WP_BYTES, smem + C::OFF_WU + u * C::WU_BYTES,
-                    C::BM, tid, NT);
+        unpack_tile<C::BM, NT>(smem + C::OFF_WP + s * C::WP_BYTES,
+                               smem + C::OFF_WU + u * C::WU_BYTES, tid);
         if constexpr (C::ACT_BITS == 4) {
-          unpack_tile(smem + C::OFF_XS + s * C::XS_BYTES, smem + C::OFF_XU + u * C::XU_BYTES,
-                      C::BN, tid, NT);
+          unpack_tile<C::BN, NT>(smem + C::OFF_XS + s * C::XS_BYTES,
+                                 smem + C::OFF_XU + u * C::XU_BYTES, tid);
         }
         fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
         __syncwarp();
@@ -280,74 +301,110 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    // Warp e covers TMEM lanes 32q..32q+31 (output channels) and every other
+    // 16-column chunk (tokens) of the tile, starting at chunk h.
     const int e = warp - C::FIRST_EPI_WARP;
+    const int q = warp & 3;
+    const int h = e >> 2;
+    const int et = threadIdx.x - C::FIRST_EPI_WARP * 32;
     uint8_t* ebuf = smem + C::OFF_EPI + e * 2 * C::EPI_BUF_BYTES;
-    int b = 0, buf = 0;
+    float* tok_s = reinterpret_cast<float*>(smem + C::OFF_TOK);
+    uint8_t* tok_id = smem + C::OFF_TOK + 2 * C::BN * 4;
+    int b = 0, buf = 0, it = 0;
     uint32_t ph_b = 0;
     const EpilogueArgs& ep = args.ep;
     const bool small_s = ep.S <= 4;
-    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
+    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++it) {
       int n_tile, m_tile;
       decode_tile(args, tile, n_tile, m_tile);
       const int n_base = n_tile * C::BM + q * 32;
       const int n = n_base + lane;
       const int m0 = m_tile * C::BN;
-      float sw = 0.0f, bs = 0.0f, bt[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      if (!C::OUT_S32 && n < args.N) {
-        sw = ep.s_w[n];
-        bs = ep.bias ? ep.bias[n] : 0.0f;
-        if (ep.beta && small_s) {
-          const float* row = ep.beta + (size_t)ep.step * ep.S * args.N + n;
+      float* sts = tok_s + (it & 1) * C::BN;
+      uint8_t* sds = tok_id + (it & 1) * C::BN;
+      // per-lane channel constants; bias and the compensation of each stream
+      // combined once per tile
+      float sw = 0.0f, bb[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (!C::OUT_S32) {
+        for (int i = et; i < C::BN; i += C::EPI_THREADS) {
+          const int m = m0 + i;
+          sts[i] = m < args.M ? ep.s_tok[m] : 0.0f;
+          sds[i] = m < args.M ? ep.stream_id[m] : 0;
+        }
+        if (n < args.N) {
+          sw = ep.s_w[n];
+          const float bs = ep.bias ? ep.bias[n] : 0.0f;
+          const float* brow = ep.beta ? ep.beta + (size_t)ep.step * ep.S * args.N + n : nullptr;
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            if (j < ep.S) bt[j] = row[(size_t)j * args.N];
+            bb[j] = (brow && j < ep.S && small_s) ? __fadd_rn(bs, brow[(size_t)j * args.N]) : bs;
         }
       }
-      const bool w = mbar_wait(&tfull[b], ph_b);
+      // staging visible to every epilogue warp (and the warps kept within one tile)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tokbar[it & 1]);
+      bool w = mbar_wait(&tokbar[it & 1], (it >> 1) & 1);
+      w = w && mbar_wait(&tfull[b], ph_b);
       if (!__all_sync(0xFFFFFFFFu, w)) break;  // uniform, and converged for tcgen05.ld
       tc_fence_after();
-      for (int j0 = 0; j0 < C::BN; j0 += C::EPI_CHUNK) {
-        uint32_t r[32];
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                               static_cast<uint32_t>(b * C::BN + j0);
-        if constexpr (C::EPI_CHUNK == 32) {
-          tmem_ld_32x32b_x32(taddr, r);
-        } else {
-          uint32_t (&r16)[16] = *reinterpret_cast<uint32_t(*)[16]>(r);
-          tmem_ld_32x32b_x16(taddr, r16);
-        }
+      if (h >= C::NUM_CHUNKS) {  // no chunk for this warp (token tiles of 16)
+        tc_fence_before();
+        if (lane == 0) mbar_arrive(&tempty[b]);
+      }
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * C::BN);
+      for (int c = h; c < C::NUM_CHUNKS; c += 2) {
+        const int j0 = c * C::EPI_CHUNK;
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tbase + j0, r);
         tmem_wait_ld();
-        if (m0 + j0 >= args.M) continue;  // whole chunk beyond the last token
-        // this lane's token (for broadcast by shuffle)
-        const int ml = m0 + j0 + lane;
-        float st_l = 0.0f;
-        int sid_l = 0;
-        if (!C::OUT_S32 && lane < C::EPI_CHUNK && ml < args.M) {
-          st_l = ep.s_tok[ml];
-          sid_l = ep.stream_id[ml];
+        if (c + 2 >= C::NUM_CHUNKS) {  // last chunk of this warp: hand the accumulator back
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[b]);
         }
+        if (m0 + j0 >= args.M) continue;  // whole chunk beyond the last token
         uint8_t* sb = ebuf + buf * C::EPI_BUF_BYTES;
         if (lane == 0) bulk_wait_group_read<1>();
         __syncwarp();
+        if constexpr (C::OUT_S32) {
 #pragma unroll
-        for (int j = 0; j < C::EPI_CHUNK; ++j) {
-          if constexpr (C::OUT_S32) {
-            reinterpret_cast<uint32_t*>(sb)[j * 32 + lane] = r[j];
-          } else {
-            const float st = __shfl_sync(0xFFFFFFFFu, st_l, j);
-            const int sd = __shfl_sync(0xFFFFFFFFu, sid_l, j);
-            float bv;
-            if (ep.beta == nullptr) {
-              bv = 0.0f;
-            } else if (small_s) {
-              bv = sd == 0 ? bt[0] : sd == 1 ? bt[1] : sd == 2 ? bt[2] : bt[3];
-            } else {
-              bv = n < args.N ? ep.beta[((size_t)ep.step * ep.S + sd) * args.N + n] : 0.0f;
+          for (int j = 0; j < 16; ++j) reinterpret_cast<uint32_t*>(sb)[j * 32 + lane] = r[j];
+        } else {
+          __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(sb);
+          const float4* st4 = reinterpret_cast<const float4*>(sts + j0);
+          const int sd_l = sds[j0 + (lane & 15)];
+          const int sd0 = sds[j0];
+          if (small_s && __all_sync(0xFFFFFFFFu, sd_l == sd0)) {
+            // one stream in the whole chunk (the common case: streams are runs of rows)
+            const float bsel = sd0 == 0 ? bb[0] : sd0 == 1 ? bb[1] : sd0 == 2 ? bb[2] : bb[3];
+#pragma unroll
+            for (int j4 = 0; j4 < 4; ++j4) {
+              const float4 t = st4[j4];
+              const float tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int j = 4 * j4 + k;
+                const float v =
+                    fmaf(tv[k] * sw, __int2float_rn(static_cast<int>(r[j])), bsel);
+                ob[j * 32 + lane] = __float2bfloat16_rn(v);
+              }
             }
-            float v = __fmul_rn(__fmul_rn(st, sw), __int2float_rn(static_cast<int>(r[j])));
-            v = __fadd_rn(__fadd_rn(v, bs), bv);
-            reinterpret_cast<__nv_bfloat16*>(sb)[j * 32 + lane] = __float2bfloat16_rn(v);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int sd = sds[j0 + j];
+              float bv;
+              if (small_s) {
+                bv = sd == 0 ? bb[0] : sd == 1 ? bb[1] : sd == 2 ? bb[2] : bb[3];
+              } else {
+                bv = n < args.N ? (ep.bias ? ep.bias[n] : 0.0f) : 0.0f;
+                if (ep.beta && n < args.N)
+                  bv = __fadd_rn(bv, ep.beta[((size_t)ep.step * ep.S + sd) * args.N + n]);
+              }
+              const float v = fmaf(sts[j0 + j] * sw, __int2float_rn(static_cast<int>(r[j])), bv);
+              ob[j * 32 + lane] = __float2bfloat16_rn(v);
+            }
           }
         }
         fence_proxy_async_smem();
@@ -358,9 +415,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         buf ^= 1;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[b]);
       if (++b == 2) { b = 0; ph_b ^= 1u; }
     }
     if (lane == 0) bulk_wait_group<0>();

@@ -1,0 +1,497 @@
+"""Throughput of the fused W4A8 / W4A4 linear (SteerQuant's Rudder kernels) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl wq|reference]
+                    [--workload NAME] [--sweep]
+
+A step is one pass of the whole hot path over one batch: for every linear of the
+workload, per-token activation quantization (channel scale and per-(step,
+stream) clip folded in) followed by the int4 x int8 tensor-core GEMM with the
+fused dequantization / bias / output-compensation epilogue.  Weight preparation
+(channel scale, int4 packing) is offline and runs before timing.
+
+Default workload: one hidden-2048 transformer block (QKV 2048->6144, attn-out
+2048->2048, MLP-up 2048->8192, MLP-down 8192->2048), W4A8, M = 4096 video + 64
+proprio + 128 action tokens, seeded synthetic inputs.  Metric: int8 tensor ops
+(2*M*N*K per linear) per second, whole job.
+
+Multi-GPU: every rank runs an independent replica of the step (the path has no
+exchange step); the time is the max over ranks and the value counts all ranks'
+work ("scaling": "weak").  --impl reference times the CPU oracle instead.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from activation_quantized_gemm_wq_b200 import synth as S  # noqa: E402
+
+METRIC = "fused W4A8/W4A4 linear TOPS (and GB/s at small M) vs roofline; vs oracle"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+INT8_PER_BF16 = 2.0  # nominal dense ratio (4.5 POPS int8 / 2.25 PFLOP/s bf16)
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=500)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["wq", "reference"], default="wq")
+    p.add_argument("--workload", default="block2048_w4a8", choices=sorted(S.WORKLOADS))
+    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--sweep", action="store_true",
+                   help="per-shape table over every configured workload (not the JSON line)")
+    return p.parse_args()
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            d = json.load(f)
+        return d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), d["hbm_gbs"], \
+            "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_init(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    """Max of a float over ranks (timing reduction only, not a data-path collective)."""
+    if world <= 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(v)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_done(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples, kept only inside [t0, t1]."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.samples = []
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.5)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [f.strip() for f in line.split(",")]))
+
+    def stop(self):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = [f for t, f in self.samples if self.t0 is not None and self.t0 <= t <= self.t1]
+        if not rows:
+            rows = [f for _, f in self.samples]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"]}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if len(r) > 2 and num(r[1]) is not None]
+        smax = [num(r[2]) for r in rows if len(r) > 2 and num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for i, n in enumerate(names):
+                if len(r) > 5 + i and r[5 + i].lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ the GPU path
+
+class Layer:
+    """Device-resident inputs of one linear: packed weights, tables, activations."""
+
+    def __init__(self, wl, i, n_sets, wq, torch, dev):
+        lin = wl.linears[i]
+        self.K, self.N, self.M = lin.K, lin.N, wl.M
+        L = S.layer_inputs(wl, i)
+        self.c = torch.empty(self.K, dtype=torch.float32, device="cuda")
+        self.cinv = torch.empty_like(self.c)
+        self.qw = torch.empty((self.N, self.K // 2), dtype=torch.uint8, device="cuda")
+        self.s_w = torch.empty(self.N, dtype=torch.float32, device="cuda")
+        W = dev(L.W)
+        wq.wq_channel_scale(dev(L.x_cal), W, self.c, self.cinv)   # offline prep, on the GPU
+        wq.wq_pack_int4(W, self.c, self.qw, self.s_w)
+        del W
+        self.alpha, self.beta, self.bias = dev(L.alpha), dev(L.beta), dev(L.bias)
+        self.T, self.S = L.alpha.shape
+        self.sid = dev(S.stream_ids(wl))
+        self.host_x = [S.activations(wl, i, step=t % wl.T) for t in range(n_sets)]
+        self.x = [dev(h) for h in self.host_x]
+        bits = wl.act_bits
+        self.bits = bits
+        self.qx = torch.empty((self.M, self.K) if bits == 8 else (self.M, self.K // 2),
+                              dtype=torch.int8 if bits == 8 else torch.uint8, device="cuda")
+        self.s_tok = torch.empty(self.M, dtype=torch.float32, device="cuda")
+        self.y = torch.empty((self.M, self.N), dtype=torch.bfloat16, device="cuda")
+        self.ws = wq.alloc_workspace(self.M, self.K, self.N, bits)
+
+    def ops(self):
+        return 2 * self.M * self.N * self.K
+
+
+def run_gpu(args, rank, world, local):
+    import torch
+
+    import activation_quantized_gemm_wq_b200 as wq
+
+    torch.cuda.set_device(local)
+    wl = S.WORKLOADS[args.workload]
+
+    def dev(a):
+        a = np.ascontiguousarray(a)
+        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
+
+    in_bytes = sum(l.K * wl.M * 2 + l.N * l.K // 2 for l in wl.linears)
+    n_sets = 2 if in_bytes > L2_BYTES else max(2, -(-2 * L2_BYTES // in_bytes))
+    layers = [Layer(wl, i, n_sets, wq, torch, dev) for i in range(len(wl.linears))]
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    T = wl.T
+
+    def step(it, gemm_events=None):
+        t = it % T
+        r = it % n_sets
+        for j, L in enumerate(layers):
+            wq.wq_act_quant(L.x[r], L.cinv, L.sid, L.alpha, t, L.bits, L.qx, L.s_tok)
+            if gemm_events is not None:
+                gemm_events[j][0].record(stream)
+            wq.wq_gemm_w4ax(L.qx, L.s_tok, L.bits, L.K, L.sid, L.beta, L.S, L.T, t, L.qw, L.s_w,
+                            L.bias, L.y)
+            if gemm_events is not None:
+                gemm_events[j][1].record(stream)
+
+    for it in range(args.warmup):
+        step(it)
+    torch.cuda.synchronize()
+    assert wq.wq_device_status() == ("WQ_OK", 0)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+           for _ in layers] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.t0 = time.time()
+    start.record(stream)
+    for it in range(args.steps):
+        step(args.warmup + it, ev[it])
+    end.record(stream)
+    torch.cuda.synchronize()
+    clocks.t1 = time.time()
+    barrier(world)
+    clocks.stop()
+    elapsed_ms = start.elapsed_time(end)
+    gemm_ms = sum(a.elapsed_time(b) for per_step in ev for a, b in per_step)
+    status = wq.wq_device_status()
+    assert status == ("WQ_OK", 0), status
+
+    t_max = max_over_ranks(elapsed_ms, world)
+    ops_step = sum(L.ops() for L in layers)
+    value = world * ops_step * args.steps / (t_max * 1e-3) / 1e12
+
+    # end to end through the public call with host buffers: pinned x in, y out
+    e2e = run_e2e(args, layers, wq, torch, world)
+
+    # torch bf16 matmul of the same shapes, reported beside (not the product)
+    tb = torch_bf16(layers, torch)
+
+    bf16_burst, bf16_sust, hbm, src = peaks()
+    peak = bf16_burst * INT8_PER_BF16
+    gemm_launches = args.steps * len(layers)
+    gemm_avg_ms = gemm_ms / gemm_launches
+    achieved = ops_step * args.steps / (gemm_ms * 1e-3) / 1e12
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(t_max / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic (seeded; stream-structured token rows, outlier channels)",
+        "config": {
+            "workload": wl.name,
+            "linears": [f"{l.name} {l.K}->{l.N}" for l in wl.linears],
+            "M": wl.M,
+            "token_rows": {"video": dict(wl.rows).get(0, 0), "proprio": dict(wl.rows).get(1, 0),
+                           "action": dict(wl.rows).get(2, 0)},
+            "act_bits": wl.act_bits,
+            "denoising_steps_in_table": T,
+            "l2": f"inputs larger than L2: {in_bytes / 2**20:.0f} MiB of activations+weights "
+                  f"per step, {n_sets} rotating activation sets",
+            "parallelism": f"replicas x{world}",
+        },
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "gemm_kernel (tcgen05 kind::i8)",
+            "achieved": round(achieved, 1),
+            "peak": round(peak, 1),
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": None,
+            "peak_source": f"{src} bf16 burst {bf16_burst} TFLOP/s x{INT8_PER_BF16} (dense int8 "
+                           "/ bf16 nominal ratio); units are int8 tera-ops",
+            "gemm_avg_launch_ms": round(gemm_avg_ms, 5),
+            "gemm_share_of_step": round(gemm_ms / (t_max if world == 1 else elapsed_ms), 4),
+        },
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "gpu_launches": 2 * len(layers) * args.steps,
+        "torch_bf16_same_shapes": tb,
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        out["cpu_baseline"] = cpu_baseline(wl, budget_s=12.0)
+    return out
+
+
+def run_e2e(args, layers, wq, torch, world):
+    """Same metric through wq_linear_w4a8/w4a4 with host buffers: pinned x copied in
+    and y copied out inside the timed region, every step."""
+    stream = torch.cuda.current_stream()
+    hx = [[torch.from_numpy(h.view(np.int16)).pin_memory() for h in L.host_x] for L in layers]
+    hy = [torch.empty((L.M, L.N), dtype=torch.bfloat16).pin_memory() for L in layers]
+    n_sets = len(layers[0].host_x)
+    fn = {8: wq.wq_linear_w4a8, 4: wq.wq_linear_w4a4}
+
+    def step(it):
+        t = it % layers[0].T
+        r = it % n_sets
+        for j, L in enumerate(layers):
+            xd = L.x[r]
+            xd.copy_(hx[j][r], non_blocking=True)
+            fn[L.bits](xd, L.cinv, L.sid, L.alpha, L.beta, t, L.qw, L.s_w, L.bias, L.y, L.ws)
+            hy[j].copy_(L.y, non_blocking=True)
+
+    for it in range(2):
+        step(it)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for it in range(args.e2e_steps):
+        step(it)
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(start.elapsed_time(end), world)
+    ops = sum(L.ops() for L in layers)
+    h2d = sum(L.M * L.K * 2 for L in layers)
+    d2h = sum(L.M * L.N * 2 for L in layers)
+    return {"value": round(world * ops * args.e2e_steps / (ms * 1e-3) / 1e12, 2), "unit": "TOPS",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms / args.e2e_steps, 4), "steps": args.e2e_steps}
+
+
+def torch_bf16(layers, torch):
+    """F.linear in bf16 on the same shapes (dequantized-weight baseline), same protocol."""
+    import torch.nn.functional as F
+    ws = [torch.randn((L.N, L.K), dtype=torch.bfloat16, device="cuda") * 0.02 for L in layers]
+    xs = [L.x[0].view(torch.bfloat16) for L in layers]
+    for _ in range(3):
+        for x, w in zip(xs, ws):
+            F.linear(x, w)
+    torch.cuda.synchronize()
+    n = 20
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(n):
+        for x, w in zip(xs, ws):
+            F.linear(x, w)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / n
+    ops = sum(L.ops() for L in layers)
+    del ws
+    return {"ms_per_step": round(ms, 5), "value": round(ops / (ms * 1e-3) / 1e12, 1),
+            "unit": "TFLOP/s"}
+
+
+# ------------------------------------------------------------------ the CPU oracle
+
+def oracle_sample(wl, rows_per_layer, seed=0):
+    """Token rows (spread over the streams) for a bounded CPU sample."""
+    g = np.random.default_rng(seed)
+    return np.sort(g.choice(wl.M, size=min(rows_per_layer, wl.M), replace=False))
+
+
+def oracle_seconds_per_row(orc, wl, prepared, sid_all):
+    sel = np.arange(2)
+    t0 = time.perf_counter()
+    for L, cinv, qw, s_w, x in prepared:
+        orc.linear(x[sel], cinv, sid_all[sel], L.alpha, L.beta, 0, wl.act_bits, qw, s_w, L.bias)
+    return (time.perf_counter() - t0) / len(sel)
+
+
+def cpu_baseline(wl, budget_s=12.0, rows=None):
+    """The oracle as it stands (single-threaded C), timed on this host on a bounded
+    sample of the workload; value in TOPS of the same metric."""
+    from oracle import Oracle
+    orc = Oracle()
+    prepared = []
+    for i, lin in enumerate(wl.linears):
+        L = S.layer_inputs(wl, i)
+        c, cinv = orc.channel_scale(L.x_cal, L.W)
+        qw, s_w = orc.pack_int4(L.W, c)
+        prepared.append((L, cinv, qw, s_w, S.activations(wl, i, 0)))
+    sid_all = S.stream_ids(wl)
+    macs_per_row = sum(l.N * l.K for l in wl.linears)
+    if rows is None:  # size the sample to the time budget from a 2-row probe
+        rows = max(1, int(budget_s / oracle_seconds_per_row(orc, wl, prepared, sid_all)))
+    sel = oracle_sample(wl, rows)
+    t0 = time.perf_counter()
+    for L, cinv, qw, s_w, x in prepared:
+        orc.linear(x[sel], cinv, sid_all[sel], L.alpha, L.beta, 0, wl.act_bits, qw, s_w, L.bias)
+    dt = time.perf_counter() - t0
+    ops = 2 * len(sel) * macs_per_row
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": 1, "kind": "oracle",
+            "sample": f"oracle_linear on {len(sel)} of {wl.M} token rows of each of the "
+                      f"{len(wl.linears)} linears ({ops / 1e9:.1f} G ops, {dt:.1f} s, "
+                      "single-threaded C)",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    wl = S.WORKLOADS[args.workload]
+    macs_per_row = sum(l.N * l.K for l in wl.linears)
+    from oracle import Oracle
+    orc = Oracle()
+    prepared = []
+    for i, lin in enumerate(wl.linears):
+        L = S.layer_inputs(wl, i)
+        c, cinv = orc.channel_scale(L.x_cal, L.W)
+        qw, s_w = orc.pack_int4(L.W, c)
+        prepared.append((L, cinv, qw, s_w, S.activations(wl, i, 0)))
+    sid_all = S.stream_ids(wl)
+    # each step: a bounded sample sized so warm-up + steps end within a few minutes
+    total = max(1, args.steps + args.warmup)
+    per_row = oracle_seconds_per_row(orc, wl, prepared, sid_all)
+    rows = max(1, int(min(150.0 / total, 15.0) / per_row))
+    times = []
+    for it in range(args.warmup + args.steps):
+        sel = oracle_sample(wl, rows, seed=it)
+        t0 = time.perf_counter()
+        for L, cinv, qw, s_w, x in prepared:
+            orc.linear(x[sel], cinv, sid_all[sel], L.alpha, L.beta, it % wl.T, wl.act_bits, qw,
+                       s_w, L.bias)
+        if it >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    ops = 2 * rows * macs_per_row
+    dt = sum(times)
+    value = ops * len(times) / dt / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic (seeded)",
+        "config": {"workload": wl.name, "M": wl.M, "act_bits": wl.act_bits,
+                   "linears": [f"{l.name} {l.K}->{l.N}" for l in wl.linears]},
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: oracle_linear on {rows} of {wl.M} token rows "
+                                   f"of every linear, single-threaded C"},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    if args.sweep:
+        from activation_quantized_gemm_wq_b200 import sweep
+        sweep.main()
+        return
+    rank, world, local = dist_init(args.gpus)
+    try:
+        if args.impl == "reference":
+            out = run_reference(args, rank, world)
+        else:
+            out = run_gpu(args, rank, world, local)
+        if rank == 0 and out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        dist_done(world)
+
+
+if __name__ == "__main__":
+    main()

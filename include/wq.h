@@ -34,7 +34,8 @@
  *   - Calls are asynchronous on `stream` (NULL = the legacy default stream).
  *     Argument errors are returned synchronously before anything is launched.
  *   - Nothing throws or aborts across this boundary.
- *   - Preconditions checked on the host: M >= 0 (M == 0 is a no-op), K a
+ *   - Preconditions checked on the host: M >= 0 (M == 0 returns WQ_OK at once
+ *     after the size and table checks; token tensors may then be NULL), K a
  *     multiple of 128 with 128 <= K <= 32768, N a multiple of 16 and >= 16,
  *     1 <= S <= 255, T >= 1, 0 <= step < T, act_bits in {4, 8}, every tensor
  *     pointer 16-byte aligned, the workspace at least wq_workspace_bytes().

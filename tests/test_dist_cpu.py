@@ -1,0 +1,54 @@
+"""Host logic of the multi-GPU benchmark path on CPU: two gloo ranks on 127.0.0.1.
+
+The fused linear has no exchange step (every token row is independent), so N GPUs
+run N replicas; the only collectives are the timing barrier and the max-over-ranks
+reduction of the elapsed time."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    r, w, local = bench.dist_init(world)
+    try:
+        bench.barrier(w)
+        t = bench.max_over_ranks(10.0 + 5.0 * r, w)   # rank-dependent elapsed times
+        q.put((r, w, local, t))
+    finally:
+        bench.dist_done(w)
+
+
+@pytest.mark.timeout(120)
+def test_two_gloo_ranks_take_the_max_time():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(90)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=5) for _ in range(world))
+    assert [g[0] for g in got] == [0, 1]
+    assert all(g[1] == 2 for g in got)
+    assert all(g[3] == 15.0 for g in got)   # every rank sees the slowest rank's time
+
+
+def test_single_process_needs_no_process_group():
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        os.environ.pop(k, None)
+    assert bench.dist_init(1) == (0, 1, 0)
+    assert bench.max_over_ranks(3.5, 1) == 3.5
