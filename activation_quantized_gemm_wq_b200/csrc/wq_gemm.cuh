@@ -34,6 +34,7 @@ namespace wq {
 namespace {
 
 struct TileArgs {
+  void* out;  // y [M][N] bf16, or acc [M][N] int32
   int M, N, K;
   int tiles_m, tiles_n, num_tiles;
   int n_fastest;
@@ -62,6 +63,9 @@ struct Cfg {
   static constexpr int STAGE_BYTES = WP_BYTES + XS_BYTES;
   static constexpr int NU = 2;  // unpacked buffers
   static constexpr int EPI_ELEM = OUT_S32 ? 4 : 2;
+  // The tensor cores accumulate 16x (int8 activations) or 256x (both operands
+  // unpacked from int4) the code products; see unpack32.
+  static constexpr int ACC_SHIFT = ACT_BITS == 8 ? 4 : 8;
   static constexpr int EPI_CHUNK = 16;  // token columns per TMEM load / TMA store
   static constexpr int NUM_CHUNKS = BN / EPI_CHUNK;
   static constexpr int EPI_BUF_BYTES = EPI_CHUNK * 32 * EPI_ELEM;
@@ -104,20 +108,20 @@ __device__ __forceinline__ void decode_tile(const TileArgs& a, int tile, int& n_
   }
 }
 
-// 16 packed bytes (32 int4 codes, low nibble first) -> 32 int8 codes.
+// 16 packed bytes (32 int4 codes, low nibble first) -> 32 bytes holding 16 * code,
+// in k order.  Moving each nibble into the high half of its byte makes the byte
+// the two's-complement value 16 * code, so no sign extension is needed; the
+// factor 16 per unpacked operand is exact in int32 and is divided out in the
+// epilogue.
 __device__ __forceinline__ void unpack32(const uint4 p, uint4& lo16, uint4& hi16) {
   const uint32_t w[4] = {p.x, p.y, p.z, p.w};
   uint32_t o[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    // bytes of e: even-k nibbles, of f: odd-k nibbles, each biased by ^8
-    const uint32_t e = (w[i] & 0x0F0F0F0Fu) ^ 0x08080808u;
-    const uint32_t f = ((w[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
-    uint32_t a = __byte_perm(e, f, 0x5140);  // k0 k1 k2 k3
-    uint32_t b = __byte_perm(e, f, 0x7362);  // k4 k5 k6 k7
-    // per byte: (n ^ 8) + 0x78 stays below 0x100; ^0x80 then yields n - 16*(n >= 8)
-    o[2 * i] = (a + 0x78787878u) ^ 0x80808080u;
-    o[2 * i + 1] = (b + 0x78787878u) ^ 0x80808080u;
+    const uint32_t e = (w[i] << 4) & 0xF0F0F0F0u;  // 16 * codes k0 k2 k4 k6
+    const uint32_t f = w[i] & 0xF0F0F0F0u;         // 16 * codes k1 k3 k5 k7
+    o[2 * i] = __byte_perm(e, f, 0x5140);          // k0 k1 k2 k3
+    o[2 * i + 1] = __byte_perm(e, f, 0x7362);      // k4 k5 k6 k7
   }
   lo16 = make_uint4(o[0], o[1], o[2], o[3]);
   hi16 = make_uint4(o[4], o[5], o[6], o[7]);
@@ -332,7 +336,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           sds[i] = m < args.M ? ep.stream_id[m] : 0;
         }
         if (n < args.N) {
-          sw = ep.s_w[n];
+          sw = ldexpf(ep.s_w[n], -C::ACC_SHIFT);  // exact power-of-two rescale
           const float bs = ep.bias ? ep.bias[n] : 0.0f;
           const float* brow = ep.beta ? ep.beta + (size_t)ep.step * ep.S * args.N + n : nullptr;
 #pragma unroll
@@ -369,7 +373,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         __syncwarp();
         if constexpr (C::OUT_S32) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) reinterpret_cast<uint32_t*>(sb)[j * 32 + lane] = r[j];
+          for (int j = 0; j < 16; ++j)  // exact: the scaled sums are multiples of 2^ACC_SHIFT
+            reinterpret_cast<int32_t*>(sb)[j * 32 + lane] = static_cast<int32_t>(r[j]) >> C::ACC_SHIFT;
         } else {
           __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(sb);
           const float4* st4 = reinterpret_cast<const float4*>(sts + j0);
@@ -493,6 +498,7 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
   if (!ok) return cudaErrorInvalidValue;
 
   TileArgs a;
+  a.out = out;
   a.M = M;
   a.N = N;
   a.K = K;
