@@ -31,6 +31,41 @@ __device__ __forceinline__ int quantize(float v, float s) {
   return q;
 }
 
+// Exact code through the IEEE quotient; kept out of line so the rare near-tie
+// path below stays a real branch instead of being computed for every element.
+template <int QMAX>
+__device__ __noinline__ int quantize_exact(float v, float s) {
+  return quantize<QMAX>(v, s);
+}
+
+// Eight codes from the correctly rounded reciprocal r = 1/s (s > 0, r finite),
+// identical to quantize<QMAX>(v[e], s) for every input.  t = v*r lies within
+// |t|*2^-22 of the IEEE quotient fl(v/s) (three roundings of at most 2^-24
+// each).  Two values that close round to different integers only if a
+// half-integer lies between them, so whenever t is farther than
+// |t|*2^-20 + 2^-20 from every half-integer, rint(t) is the rounding of
+// fl(v/s); the few other elements take the exact quotient.
+template <int QMAX>
+__device__ __forceinline__ void quantize8_recip(const float (&v)[8], float s, float r,
+                                                int (&q)[8]) {
+  uint32_t near_tie = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float t = __fmul_rn(v[e], r);
+    const float ti = rintf(t);
+    const float d = fabsf(__fsub_rn(t, ti));  // distance to the nearest integer
+    const float margin = __fmaf_rn(fabsf(t), 0x1p-20f, 0x1p-20f);
+    near_tie |= (__fsub_rn(0.5f, d) <= margin ? 1u : 0u) << e;
+    const float qf = fminf(fmaxf(ti, -static_cast<float>(QMAX)), static_cast<float>(QMAX));
+    q[e] = __float2int_rn(qf);
+  }
+  if (near_tie != 0u) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (near_tie & (1u << e)) q[e] = quantize_exact<QMAX>(v[e], s);
+  }
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
@@ -102,14 +137,20 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
     raise_error(kErrBadStreamId);
   }
   if (t == 0) s_tok[row] = s;
+  const float r = s > 0.0f ? __frcp_rn(s) : 0.0f;
+  const bool fast = s > 0.0f && isfinite(r);  // else: zero row, or a tiny scale
 
 #pragma unroll
   for (int i = 0; i < CPT; ++i) {
     const int c = t + i * TPR;
     if (c >= nchunk) continue;
     int q[8];
+    if (fast) {
+      quantize8_recip<QMAX>(v[i], s, r, q);
+    } else {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) q[e] = quantize<QMAX>(v[i][e], s);
+      for (int e = 0; e < 8; ++e) q[e] = quantize<QMAX>(v[i][e], s);
+    }
     if constexpr (ACT_BITS == 8) {
       uint2 o;
       o.x = (q[0] & 0xFF) | ((q[1] & 0xFF) << 8) | ((q[2] & 0xFF) << 16) | ((uint32_t)q[3] << 24);
@@ -142,12 +183,14 @@ cudaError_t dispatch_act_quant(const uint16_t* x, int M, int K, const float* cin
   const int nchunk = K / 8;
 #define WQ_AQ(TPR, CPT) \
   return run_act_quant<ACT_BITS, TPR, CPT>(x, M, K, cinv, sid, alpha, S, step, qx, s_tok, st)
+  // one warp per row up to K = 2048 (no block-level reduction), 8 chunks of 8
+  // channels per thread beyond that
   if (nchunk <= 32) WQ_AQ(32, 1);
-  if (nchunk <= 64) WQ_AQ(64, 1);
-  if (nchunk <= 128) WQ_AQ(128, 1);
-  if (nchunk <= 256) WQ_AQ(256, 1);
-  if (nchunk <= 512) WQ_AQ(256, 2);
-  if (nchunk <= 1024) WQ_AQ(256, 4);
+  if (nchunk <= 64) WQ_AQ(32, 2);
+  if (nchunk <= 128) WQ_AQ(32, 4);
+  if (nchunk <= 256) WQ_AQ(32, 8);
+  if (nchunk <= 512) WQ_AQ(64, 8);
+  if (nchunk <= 1024) WQ_AQ(128, 8);
   if (nchunk <= 2048) WQ_AQ(256, 8);
   WQ_AQ(256, 16);
 #undef WQ_AQ
