@@ -61,7 +61,12 @@ struct Cfg {
   static constexpr int XS_BYTES = ACT_BITS == 8 ? BN * BK : BN * BK / 2;     // staged x
   static constexpr int XU_BYTES = ACT_BITS == 8 ? 0 : BN * BK;               // int8 x (A4)
   static constexpr int STAGE_BYTES = WP_BYTES + XS_BYTES;
-  static constexpr int NU = 2;  // unpacked buffers
+  // Pipeline: NS TMA stages (packed weights + activation tile), NU unpacked
+  // buffers, and one "MMA done with K block g" barrier per stage (a ring of NS).
+  // The single MMA-issuing thread does one wait and one commit per K block: it
+  // can queue barely one instruction ahead of the tensor pipe, so its per-block
+  // overhead, not the pipeline depth alone, decides whether the pipe stays fed.
+  static constexpr int NU = ACT_BITS == 8 ? 3 : 2;
   static constexpr int EPI_ELEM = OUT_S32 ? 4 : 2;
   // The tensor cores accumulate 16x (int8 activations) or 256x (both operands
   // unpacked from int4) the code products; see unpack32.
@@ -69,14 +74,18 @@ struct Cfg {
   static constexpr int EPI_CHUNK = 16;  // token columns per TMEM load / TMA store
   static constexpr int NUM_CHUNKS = BN / EPI_CHUNK;
   static constexpr int EPI_BUF_BYTES = EPI_CHUNK * 32 * EPI_ELEM;
-  static constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BUF_BYTES;
   static constexpr int TOK_BYTES = 2 * BN * 4 + 2 * BN;  // staged s_tok and stream ids, x2
   static constexpr int SMEM_LIMIT = 232448;  // 227 KB opt-in per CTA
   static constexpr int RESERVED = 1024 /*alignment slack*/ + 512 /*barriers*/;
-  static constexpr int NS_FIT =
-      (SMEM_LIMIT - RESERVED - NU * (WU_BYTES + XU_BYTES) - EPI_BYTES - TOK_BYTES) / STAGE_BYTES;
+  static constexpr int FIXED = RESERVED + NU * (WU_BYTES + XU_BYTES) + TOK_BYTES;
+  // double-buffered epilogue staging unless that would cost a TMA stage below 4
+  static constexpr int NS_WITH_2 =
+      (SMEM_LIMIT - FIXED - EPI_WARPS * 2 * EPI_BUF_BYTES) / STAGE_BYTES;
+  static constexpr int EPI_NBUF = NS_WITH_2 >= 4 ? 2 : 1;
+  static constexpr int EPI_BYTES = EPI_WARPS * EPI_NBUF * EPI_BUF_BYTES;
+  static constexpr int NS_FIT = (SMEM_LIMIT - FIXED - EPI_BYTES) / STAGE_BYTES;
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
-  static_assert(NS >= 2, "pipeline needs at least two stages");
+  static_assert(NS >= NU && NS >= 2, "the done ring needs NS >= NU");
   static_assert(BN % EPI_CHUNK == 0 && NUM_CHUNKS >= 1, "token tile is a multiple of 16");
 
   static constexpr int OFF_WP = 0;
@@ -86,7 +95,7 @@ struct Cfg {
   static constexpr int OFF_EPI = OFF_XU + NU * XU_BYTES;
   static constexpr int OFF_TOK = OFF_EPI + EPI_BYTES;
   static constexpr int OFF_BAR = OFF_TOK + TOK_BYTES;
-  static constexpr int NUM_BARS = 2 * NS + 2 * NU + 6;
+  static constexpr int NUM_BARS = 2 * NS + NU + 6;
   static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
   static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
   static_assert(OFF_XS % 1024 == 0 && XS_BYTES % 512 == 0 && OFF_WU % 1024 == 0 &&
@@ -173,11 +182,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* empty = full + C::NS;
-  uint64_t* ufull = empty + C::NS;
-  uint64_t* uempty = ufull + C::NU;
-  uint64_t* tfull = uempty + C::NU;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // TMA landed, stage s
+  uint64_t* done = full + C::NS;     // MMA finished K block g, slot g % NS (one commit)
+  uint64_t* ufull = done + C::NS;    // unpacked buffer u ready
+  uint64_t* tfull = ufull + C::NU;
   uint64_t* tempty = tfull + 2;
   uint64_t* tokbar = tempty + 2;  // epilogue warps: token staging of buffer i complete
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tokbar + 2);
@@ -189,12 +197,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], C::ACT_BITS == 8 ? 1 : C::UNPACK_WARPS);
+      mbar_init(&done[s], 1);
     }
-    for (int u = 0; u < C::NU; ++u) {
-      mbar_init(&ufull[u], C::UNPACK_WARPS);
-      mbar_init(&uempty[u], 1);
-    }
+    for (int u = 0; u < C::NU; ++u) mbar_init(&ufull[u], C::UNPACK_WARPS);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], C::EPI_WARPS);
@@ -219,47 +224,54 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // K block g (counted over all of this CTA's tiles) goes to stage g % NS once
+    // the MMA has finished K block g - NS, the previous user of that stage.
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
-      int issued = 0;
+      uint32_t g = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
         int n_tile, m_tile;
         decode_tile(args, tile, n_tile, m_tile);
-        for (int kb = 0; kb < num_k; ++kb) {
-          if (!mbar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
+        for (int kb = 0; kb < num_k; ++kb, ++g) {
+          const uint32_t s = g % C::NS;
+          if (g >= static_cast<uint32_t>(C::NS) &&
+              !mbar_wait(&done[s], ((g / C::NS) - 1) & 1u)) {
+            ok = false;
+            break;
+          }
           mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
           tma_load_2d(smem + C::OFF_WP + s * C::WP_BYTES, &tm_w, &full[s], kb * (C::BK / 2),
                       n_tile * C::BM);
           tma_load_2d(smem + C::OFF_XS + s * C::XS_BYTES, &tm_x, &full[s],
                       kb * (C::ACT_BITS == 8 ? C::BK : C::BK / 2), m_tile * C::BN);
-          ++issued;
-          if (++s == C::NS) { s = 0; ph ^= 1u; }
         }
       }
-      // Drain: every issued stage's copies must have landed before the CTA exits.
-      // (Normally they were all consumed already and these waits return at once.)
-      for (int i = 0; i < C::NS && i < issued; ++i) {
-        if (--s < 0) { s = C::NS - 1; ph ^= 1u; }
-        mbar_wait(&full[s], ph);
+      // Drain: the copies of every issued stage must have landed before the CTA
+      // exits (normally all were consumed already and these waits return at once).
+      for (uint32_t i = 0; i < static_cast<uint32_t>(C::NS) && i < g; ++i) {
+        const uint32_t j = g - 1 - i;
+        mbar_wait(&full[j % C::NS], (j / C::NS) & 1u);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Per K block: one wait (its unpacked buffer; the unpack warps arrive there
+    // only after the stage's TMA landed, which orders the activation tile too),
+    // four MMAs, one commit (frees the stage and the unpacked buffer).
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_i8(C::BN);
-      int s = 0, u = 0, b = 0;
-      uint32_t ph_s = 0, ph_u = 0, ph_b = 0;
+      uint32_t g = 0;
+      int b = 0;
+      uint32_t ph_b = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
         if (!mbar_wait(&tempty[b], ph_b ^ 1u)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * C::BN);
-        for (int kb = 0; kb < num_k; ++kb) {
-          if (C::ACT_BITS == 8 && !mbar_wait(&full[s], ph_s)) { ok = false; break; }
-          if (!mbar_wait(&ufull[u], ph_u)) { ok = false; break; }
+        for (int kb = 0; kb < num_k; ++kb, ++g) {
+          const uint32_t s = g % C::NS, u = g % C::NU;
+          if (!mbar_wait(&ufull[u], (g / C::NU) & 1u)) { ok = false; break; }
           tc_fence_after();
           const uint32_t b_addr =
               C::ACT_BITS == 8 ? smem_u32(smem + C::OFF_XS + s * C::XS_BYTES)
@@ -269,10 +281,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           for (int kk = 0; kk < C::BK / 32; ++kk)
             mma_i8_ss(d_tmem, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32),
                       idesc, (kb | kk) != 0 ? 1u : 0u);
-          mma_commit(&uempty[u]);
-          if (C::ACT_BITS == 8) mma_commit(&empty[s]);
-          if (++u == C::NU) { u = 0; ph_u ^= 1u; }
-          if (++s == C::NS) { s = 0; ph_s ^= 1u; }
+          mma_commit(&done[s]);
         }
         if (!ok) break;
         mma_commit(&tfull[b]);
@@ -282,15 +291,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncwarp();
   } else if (warp < C::FIRST_EPI_WARP) {
     // ------------------------------------------------------------ int4 -> int8
+    // K block g: wait for its TMA stage and for the MMA to have finished K block
+    // g - NU (the previous user of unpacked buffer g % NU).
     const int tid = threadIdx.x - C::FIRST_UNPACK_WARP * 32;
     constexpr int NT = C::UNPACK_WARPS * 32;
-    int s = 0, u = 0;
-    uint32_t ph_s = 0, ph_u = 0;
+    uint32_t g = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
-      for (int kb = 0; kb < num_k; ++kb) {
-        bool w = mbar_wait(&full[s], ph_s);
-        w = w && mbar_wait(&uempty[u], ph_u ^ 1u);
+      for (int kb = 0; kb < num_k; ++kb, ++g) {
+        const uint32_t s = g % C::NS, u = g % C::NU;
+        bool w = mbar_wait(&full[s], (g / C::NS) & 1u);
+        if (g >= static_cast<uint32_t>(C::NU)) {
+          const uint32_t j = g - C::NU;
+          w = w && mbar_wait(&done[j % C::NS], (j / C::NS) & 1u);
+        }
         if (!__all_sync(0xFFFFFFFFu, w)) {  // keep the warp's decision uniform
           ok = false;
           break;
@@ -306,12 +320,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&ufull[u]);
-          if (C::ACT_BITS == 4) mbar_arrive(&empty[s]);
-        }
-        if (++u == C::NU) { u = 0; ph_u ^= 1u; }
-        if (++s == C::NS) { s = 0; ph_s ^= 1u; }
+        if (lane == 0) mbar_arrive(&ufull[u]);
       }
     }
   } else {
@@ -322,7 +331,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int q = warp & 3;
     const int h = e >> 2;
     const int et = threadIdx.x - C::FIRST_EPI_WARP * 32;
-    uint8_t* ebuf = smem + C::OFF_EPI + e * 2 * C::EPI_BUF_BYTES;
+    uint8_t* ebuf = smem + C::OFF_EPI + e * C::EPI_NBUF * C::EPI_BUF_BYTES;
     float* tok_s = reinterpret_cast<float*>(smem + C::OFF_TOK);
     uint8_t* tok_id = smem + C::OFF_TOK + 2 * C::BN * 4;
     int b = 0, buf = 0, it = 0;
@@ -380,7 +389,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         if (m0 + j0 >= args.M) continue;  // whole chunk beyond the last token
         uint8_t* sb = ebuf + buf * C::EPI_BUF_BYTES;
-        if (lane == 0) bulk_wait_group_read<1>();
+        if (lane == 0) {  // this buffer's previous TMA store has read it
+          if constexpr (C::EPI_NBUF == 2) bulk_wait_group_read<1>();
+          else bulk_wait_group_read<0>();
+        }
         __syncwarp();
         if constexpr (C::OUT_S32) {
 #pragma unroll
@@ -429,7 +441,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           tma_store_2d(&tm_out, sb, n_base, m0 + j0);
           bulk_commit_group();
         }
-        buf ^= 1;
+        if constexpr (C::EPI_NBUF == 2) buf ^= 1;
       }
       if (++b == 2) { b = 0; ph_b ^= 1u; }
     }
