@@ -20,7 +20,7 @@ _I = ctypes.c_int
 
 WQ_OK = 0
 STATUS = {0: "WQ_OK", 1: "WQ_ERR_NULL", 2: "WQ_ERR_SHAPE", 3: "WQ_ERR_ALIGN", 4: "WQ_ERR_ARG",
-          5: "WQ_ERR_CUDA", 6: "WQ_ERR_TIMEOUT", 7: "WQ_ERR_DEVICE"}
+          5: "WQ_ERR_CUDA", 6: "WQ_ERR_TIMEOUT", 7: "WQ_ERR_DEVICE", 8: "WQ_ERR_SCRATCH"}
 
 # name -> (restype, argtypes); mirrors include/wq.h
 _SIGS = {
@@ -35,6 +35,8 @@ _SIGS = {
                             ctypes.c_size_t, _P]),
     "wq_linear_w4a4": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P,
                             ctypes.c_size_t, _P]),
+    "wq_linear_w4a8_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P,
+                                    _P]),
     "wq_debug_gemm_s32": (_I, [_P, _I, _P, _I, _I, _I, _P, _P]),
     "wq_device_status": (_I, [ctypes.POINTER(ctypes.c_uint)]),
 }
@@ -141,6 +143,17 @@ def wq_linear_w4a4(x, cinv, stream_id, alpha, beta, step, qw, s_w, bias, y, work
                    stream=None):
     _linear("wq_linear_w4a4", x, cinv, stream_id, alpha, beta, step, qw, s_w, bias, y,
             workspace, stream)
+
+
+def wq_linear_w4a8_noalloc(x, cinv, stream_id, alpha, beta, step, qw, s_w, bias, y,
+                           stream=None):
+    """wq_linear_w4a8 without a workspace: for callers that cannot allocate device
+    memory while they run.  Uses the library's fixed 16 MiB scratch (see wq.h)."""
+    M, K = x.shape
+    N = qw.shape[0]
+    T, S = alpha.shape
+    _call("wq_linear_w4a8_noalloc", _ptr(x), M, K, N, _ptr(cinv), _ptr(stream_id), _ptr(alpha),
+          _ptr(beta), S, T, step, _ptr(qw), _ptr(s_w), _ptr(bias), _ptr(y), _stream(stream))
 
 
 def wq_debug_gemm_s32(qx, act_bits, qw, K, acc, stream=None):

@@ -4,6 +4,7 @@
 #include "wq.h"
 
 #include <cstdint>
+#include <mutex>
 
 #include "wq_gemm.cuh"
 #include "wq_internal.h"
@@ -80,6 +81,39 @@ wq_status linear(const wq_bf16* x, int M, int K, int N, const float* cinv,
   return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, y, false, st));
 }
 
+// ------------------------------------------------------------ no-alloc variant
+// Scratch of wq_linear_w4a8_noalloc: the int8 codes and token scales that pass
+// between the two kernels.  One copy per GPU that loads the library, held until
+// the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+
+}  // namespace
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device with that device current.  (In host code the array's name is only a
+// host-side stand-in, not a device address.)
+wq_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return WQ_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return WQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -94,6 +128,9 @@ const char* wq_status_string(wq_status s) {
     case WQ_ERR_CUDA: return "WQ_ERR_CUDA: the CUDA runtime rejected a launch";
     case WQ_ERR_TIMEOUT: return "WQ_ERR_TIMEOUT: a kernel's bounded wait gave up";
     case WQ_ERR_DEVICE: return "WQ_ERR_DEVICE: a device-side precondition failed";
+    case WQ_ERR_SCRATCH:
+      return "WQ_ERR_SCRATCH: codes and token scales exceed the 16 MiB fixed scratch of "
+             "wq_linear_w4a8_noalloc";
   }
   return "unknown wq_status";
 }
@@ -177,6 +214,19 @@ wq_status wq_debug_gemm_s32(const void* qx, int act_bits, const uint8_t* qw, int
   const wq::EpilogueArgs ep{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 0};
   return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, acc, true,
                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_linear_w4a8_noalloc(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                                 const uint8_t* stream_id, const float* alpha,
+                                 const float* beta, int S, int T, int step, const uint8_t* qw,
+                                 const float* s_w, const float* bias, wq_bf16* y,
+                                 wq_stream_t stream) {
+  const size_t need = wq_workspace_bytes(M, K, N, 8);  // 0: invalid sizes, or M == 0
+  if (need > kNoAllocScratchBytes) return WQ_ERR_SCRATCH;
+  void* scratch = nullptr;
+  if (need > 0) WQ_TRY(noalloc_scratch(&scratch));
+  return linear(x, M, K, N, cinv, stream_id, alpha, beta, S, T, step, qw, s_w, bias, y, scratch,
+                need > 0 ? kNoAllocScratchBytes : 0, stream, 8);
 }
 
 wq_status wq_device_status(unsigned* flags) {

@@ -64,7 +64,8 @@ typedef enum {
   WQ_ERR_ARG = 4,     /* bad act_bits, S, T, step, or workspace too small */
   WQ_ERR_CUDA = 5,    /* the CUDA runtime rejected a launch */
   WQ_ERR_TIMEOUT = 6, /* wq_device_status: a kernel's bounded wait gave up */
-  WQ_ERR_DEVICE = 7   /* wq_device_status: a device-side precondition failed */
+  WQ_ERR_DEVICE = 7,  /* wq_device_status: a device-side precondition failed */
+  WQ_ERR_SCRATCH = 8  /* wq_linear_w4a8_noalloc: the sizes exceed its fixed scratch */
 } wq_status;
 
 /* Device error bits reported by wq_device_status(). */
@@ -140,6 +141,35 @@ wq_status wq_linear_w4a4(const wq_bf16* x, int M, int K, int N, const float* cin
  * epilogue replaced by a raw store of the int32 accumulators acc [M][N]. */
 wq_status wq_debug_gemm_s32(const void* qx, int act_bits, const uint8_t* qw, int M, int N,
                             int K, int32_t* acc, wq_stream_t stream);
+
+/* The fused W4A8 linear for callers that cannot allocate device memory.  The
+ * paper has no counterpart to this entry point.
+ *
+ * Some callers may not allocate while they run: a robot controller's real-time
+ * inference loop, where cudaMalloc can synchronize the device and take an
+ * unbounded time; or a host application that owns all device memory and hands
+ * the library no allocator.  This call takes no workspace.  The int8 codes and
+ * token scales that pass between the two kernels live instead in a fixed
+ * scratch array inside the library: 16 MiB, declared at file scope, so every
+ * GPU that loads the library holds it until the process exits.  No cudaMalloc,
+ * cudaFree or other allocating routine is called.
+ *
+ * Limit: wq_workspace_bytes(M, K, N, 8) must not exceed 16 MiB (about
+ * M*K + 4*M bytes; for example M = 4096 tokens at K = 4096).  Larger sizes
+ * return WQ_ERR_SCRATCH before anything is launched.
+ * The first call on a device looks up the scratch array's device address with
+ * that device current (cudaGetSymbolAddress) and caches it; make that first
+ * call before any stream capture on the device.
+ * Every call shares the one array and reuses it as it stands: each call
+ * rewrites all of the scratch it reads before reading it, so nothing needs
+ * clearing, but calls whose work overlaps on the GPU (concurrent streams, or
+ * concurrent host threads on the same device) race on it.
+ * Other arguments and all results are exactly as in wq_linear_w4a8. */
+wq_status wq_linear_w4a8_noalloc(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                                 const uint8_t* stream_id, const float* alpha,
+                                 const float* beta, int S, int T, int step, const uint8_t* qw,
+                                 const float* s_w, const float* bias, wq_bf16* y,
+                                 wq_stream_t stream);
 
 /* Reads and clears the device error word of the current device (synchronizes
  * the device).  *flags receives the WQ_DEVICE_ERR_* bits seen since the last
