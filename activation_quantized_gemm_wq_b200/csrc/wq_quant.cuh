@@ -38,32 +38,57 @@ __device__ __noinline__ int quantize_exact(float v, float s) {
   return quantize<QMAX>(v, s);
 }
 
+// Adding 1.5 * 2^23 to a float of magnitude below 2^22 rounds it to an integer
+// (the addition's own round-half-to-even), and that integer sits in the low
+// bits of the sum's bit pattern, two's complement for negative values.
+constexpr float kRoundMagic = 12582912.0f;
+
 // Eight codes from the correctly rounded reciprocal r = 1/s (s > 0, r finite),
 // identical to quantize<QMAX>(v[e], s) for every input.  t = v*r lies within
 // |t|*2^-22 of the IEEE quotient fl(v/s) (three roundings of at most 2^-24
-// each).  Two values that close round to different integers only if a
-// half-integer lies between them, so whenever t is farther than
-// |t|*2^-20 + 2^-20 from every half-integer, rint(t) is the rounding of
-// fl(v/s); the few other elements take the exact quotient.
+// each), i.e. within 2^-12 while |t| <= 2^10.  Two values that close round to
+// different integers only if a half-integer lies between them, so whenever t is
+// farther than 2^-12 from every half-integer, the rounding of t is the rounding
+// of fl(v/s); beyond |t| = 2^10 both clamp to the same end of the range.  The few
+// other elements take the exact quotient.  Each result's low byte is the code.
 template <int QMAX>
 __device__ __forceinline__ void quantize8_recip(const float (&v)[8], float s, float r,
-                                                int (&q)[8]) {
-  uint32_t near_tie = 0;
+                                                uint32_t (&c)[8]) {
+  constexpr float lo = kRoundMagic - static_cast<float>(QMAX);
+  constexpr float hi = kRoundMagic + static_cast<float>(QMAX);
+  bool near_tie = false;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     const float t = __fmul_rn(v[e], r);
-    const float ti = rintf(t);
-    const float d = fabsf(__fsub_rn(t, ti));  // distance to the nearest integer
-    const float margin = __fmaf_rn(fabsf(t), 0x1p-20f, 0x1p-20f);
-    near_tie |= (__fsub_rn(0.5f, d) <= margin ? 1u : 0u) << e;
-    const float qf = fminf(fmaxf(ti, -static_cast<float>(QMAX)), static_cast<float>(QMAX));
-    q[e] = __float2int_rn(qf);
+    const float u = __fadd_rn(t, kRoundMagic);                 // kRoundMagic + rint(t)
+    const float d = __fsub_rn(t, __fsub_rn(u, kRoundMagic));   // t - rint(t), exact
+    near_tie = near_tie || fabsf(d) >= 0.5f - 0x1p-12f;
+    c[e] = __float_as_uint(fminf(fmaxf(u, lo), hi));           // clamp to +-QMAX
   }
-  if (near_tie != 0u) {
+  if (near_tie) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      if (near_tie & (1u << e)) q[e] = quantize_exact<QMAX>(v[e], s);
+    for (int e = 0; e < 8; ++e) {
+      const float t = __fmul_rn(v[e], r);
+      const float u = __fadd_rn(t, kRoundMagic);
+      const float d = __fsub_rn(t, __fsub_rn(u, kRoundMagic));
+      if (fabsf(d) >= 0.5f - 0x1p-12f) c[e] = static_cast<uint32_t>(quantize_exact<QMAX>(v[e], s));
+    }
   }
+}
+
+// Low bytes of four words -> one word.
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c,
+                                                   uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Low nibbles of eight words -> one word, code 2j in the low nibble of byte j.
+__device__ __forceinline__ uint32_t pack_low_nibbles(const uint32_t (&c)[8]) {
+  uint32_t n = pack_low_bytes(c[0], c[1], c[2], c[3]) & 0x0F0F0F0Fu;
+  uint32_t m = pack_low_bytes(c[4], c[5], c[6], c[7]) & 0x0F0F0F0Fu;
+  n |= n >> 4;  // bytes 0 and 2 now hold (c0 | c1 << 4) and (c2 | c3 << 4)
+  m |= m >> 4;
+  return __byte_perm(n, m, 0x6420);
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -72,95 +97,118 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// One token row per TPR threads; each thread holds CPT chunks of 8 channels in
-// registers, so x is read from HBM exactly once.
+// cinv chunk c from the CTA's shared-memory copy (8 floats).
+__device__ __forceinline__ void load_cinv8(const float* cinv_s, int c, float (&ci)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(cinv_s)[2 * c];
+  const float4 b = reinterpret_cast<const float4*>(cinv_s)[2 * c + 1];
+  ci[0] = a.x; ci[1] = a.y; ci[2] = a.z; ci[3] = a.w;
+  ci[4] = b.x; ci[5] = b.y; ci[6] = b.z; ci[7] = b.w;
+}
+
+// x' = x * cinv for one chunk of 8 channels (bf16 widening is exact).
+__device__ __forceinline__ void scale8(const uint4 raw, const float (&ci)[8], float (&v)[8]) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    v[2 * e] = __fmul_rn(bf16lo(w[e]), ci[2 * e]);
+    v[2 * e + 1] = __fmul_rn(bf16hi(w[e]), ci[2 * e + 1]);
+  }
+}
+
+// Persistent CTAs; each pass handles RPC token rows, one row per TPR threads.
+// cinv is copied to shared memory once per CTA.  Each thread loads its CPT
+// chunks of 8 channels (128-bit loads, all issued before any use, so x is read
+// from HBM once with CPT loads in flight per thread), then forms x * cinv twice:
+// once for the row maximum and once for the codes, which keeps register use low.
 template <int ACT_BITS, int TPR, int CPT>
 __global__ void __launch_bounds__(256) act_quant_kernel(
     const uint16_t* __restrict__ x, int M, int K, const float* __restrict__ cinv,
     const uint8_t* __restrict__ stream_id, const float* __restrict__ alpha, int S, int step,
     void* __restrict__ qx, float* __restrict__ s_tok) {
-  constexpr int RPC = 256 / TPR;  // rows per CTA
+  constexpr int RPC = 256 / TPR;  // rows per CTA pass
   constexpr int WPR = TPR / 32;   // warps per row
   constexpr int QMAX = ACT_BITS == 8 ? 127 : 7;
+  extern __shared__ float4 cinv_s4[];
+  float* cinv_s = reinterpret_cast<float*>(cinv_s4);
   __shared__ float red[8];
+
+  for (int k = threadIdx.x * 4; k < K; k += 256 * 4)
+    *reinterpret_cast<float4*>(cinv_s + k) =
+        cinv ? __ldg(reinterpret_cast<const float4*>(cinv + k)) : make_float4(1.f, 1.f, 1.f, 1.f);
+  __syncthreads();
 
   const int local_row = threadIdx.x / TPR;
   const int t = threadIdx.x % TPR;
-  const int row = blockIdx.x * RPC + local_row;
-  const bool row_ok = row < M;
   const int nchunk = K >> 3;
+  const int groups = (M + RPC - 1) / RPC;
 
-  float v[CPT][8];
-  float amax = 0.0f;
+  for (int grp = blockIdx.x; grp < groups; grp += gridDim.x) {  // CTA-uniform loop
+    const int row = grp * RPC + local_row;
+    const bool row_ok = row < M;
+    uint4 raw[CPT];
 #pragma unroll
-  for (int i = 0; i < CPT; ++i) {
-    const int c = t + i * TPR;
-    if (row_ok && c < nchunk) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x + (size_t)row * K) + c);
-      float ci[8];
-      if (cinv != nullptr) {
-        const float4 a = __ldg(reinterpret_cast<const float4*>(cinv) + 2 * c);
-        const float4 b = __ldg(reinterpret_cast<const float4*>(cinv) + 2 * c + 1);
-        ci[0] = a.x; ci[1] = a.y; ci[2] = a.z; ci[3] = a.w;
-        ci[4] = b.x; ci[5] = b.y; ci[6] = b.z; ci[7] = b.w;
+    for (int i = 0; i < CPT; ++i) {
+      const int c = t + i * TPR;
+      raw[i] = (row_ok && c < nchunk)
+                   ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)row * K) + c)
+                   : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+      const int c = t + i * TPR;
+      if (c < nchunk) {
+        float ci[8], v[8];
+        load_cinv8(cinv_s, c, ci);
+        scale8(raw[i], ci, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+      }
+    }
+    amax = warp_max(amax);
+    if constexpr (WPR > 1) {
+      if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < WPR; ++j) amax = fmaxf(amax, red[local_row * WPR + j]);
+      __syncthreads();  // red is rewritten by the next pass
+    }
+    if (!row_ok) continue;
+
+    float s = 0.0f;
+    const int sid = stream_id[row];
+    if (sid < S) {
+      const float clip = __fmul_rn(__ldg(alpha + step * S + sid), amax);
+      s = __fdiv_rn(clip, static_cast<float>(QMAX));
+    } else if (t == 0) {
+      raise_error(kErrBadStreamId);
+    }
+    if (t == 0) s_tok[row] = s;
+    const float r = s > 0.0f ? __frcp_rn(s) : 0.0f;
+    const bool fast = s > 0.0f && isfinite(r);  // else: zero row, or a tiny scale
+
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+      const int c = t + i * TPR;
+      if (c >= nchunk) continue;
+      float ci[8], v[8];
+      load_cinv8(cinv_s, c, ci);
+      scale8(raw[i], ci, v);
+      uint32_t q[8];  // low byte of each: the code
+      if (fast) {
+        quantize8_recip<QMAX>(v, s, r, q);
       } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ci[e] = 1.0f;
+        for (int e = 0; e < 8; ++e) q[e] = static_cast<uint32_t>(quantize<QMAX>(v[e], s));
       }
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        v[i][2 * e] = __fmul_rn(bf16lo(w[e]), ci[2 * e]);
-        v[i][2 * e + 1] = __fmul_rn(bf16hi(w[e]), ci[2 * e + 1]);
-        amax = fmaxf(amax, fmaxf(fabsf(v[i][2 * e]), fabsf(v[i][2 * e + 1])));
+      if constexpr (ACT_BITS == 8) {
+        const uint2 o = make_uint2(pack_low_bytes(q[0], q[1], q[2], q[3]),
+                                   pack_low_bytes(q[4], q[5], q[6], q[7]));
+        reinterpret_cast<uint2*>(static_cast<int8_t*>(qx) + (size_t)row * K)[c] = o;
+      } else {
+        reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(qx) + (size_t)row * (K / 2))[c] =
+            pack_low_nibbles(q);
       }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[i][e] = 0.0f;
-    }
-  }
-  amax = warp_max(amax);
-  if constexpr (WPR > 1) {
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
-    __syncthreads();
-#pragma unroll
-    for (int j = 0; j < WPR; ++j) amax = fmaxf(amax, red[local_row * WPR + j]);
-  }
-  if (!row_ok) return;
-
-  float s = 0.0f;
-  const int sid = stream_id[row];
-  if (sid < S) {
-    const float clip = __fmul_rn(__ldg(alpha + step * S + sid), amax);
-    s = __fdiv_rn(clip, static_cast<float>(QMAX));
-  } else if (t == 0) {
-    raise_error(kErrBadStreamId);
-  }
-  if (t == 0) s_tok[row] = s;
-  const float r = s > 0.0f ? __frcp_rn(s) : 0.0f;
-  const bool fast = s > 0.0f && isfinite(r);  // else: zero row, or a tiny scale
-
-#pragma unroll
-  for (int i = 0; i < CPT; ++i) {
-    const int c = t + i * TPR;
-    if (c >= nchunk) continue;
-    int q[8];
-    if (fast) {
-      quantize8_recip<QMAX>(v[i], s, r, q);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) q[e] = quantize<QMAX>(v[i][e], s);
-    }
-    if constexpr (ACT_BITS == 8) {
-      uint2 o;
-      o.x = (q[0] & 0xFF) | ((q[1] & 0xFF) << 8) | ((q[2] & 0xFF) << 16) | ((uint32_t)q[3] << 24);
-      o.y = (q[4] & 0xFF) | ((q[5] & 0xFF) << 8) | ((q[6] & 0xFF) << 16) | ((uint32_t)q[7] << 24);
-      reinterpret_cast<uint2*>(static_cast<int8_t*>(qx) + (size_t)row * K)[c] = o;
-    } else {
-      uint32_t o = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o |= (uint32_t)(q[e] & 0xF) << (4 * e);
-      reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(qx) + (size_t)row * (K / 2))[c] = o;
     }
   }
 }
@@ -170,9 +218,23 @@ cudaError_t run_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                           const uint8_t* sid, const float* alpha, int S, int step, void* qx,
                           float* s_tok, cudaStream_t st) {
   constexpr int RPC = 256 / TPR;
-  const int grid = (M + RPC - 1) / RPC;
+  const size_t smem = static_cast<size_t>(K) * sizeof(float);  // cinv copy
+  static int per_sm = 0;  // resident CTAs per SM at the largest K (per template instance)
+  if (per_sm == 0) {
+    if (cudaFuncSetAttribute(act_quant_kernel<ACT_BITS, TPR, CPT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxK * 4) != cudaSuccess)
+      return cudaGetLastError();
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, act_quant_kernel<ACT_BITS, TPR, CPT>,
+                                                  256, smem);
+    if (per_sm < 1) per_sm = 1;
+  }
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int groups = (M + RPC - 1) / RPC;
+  const int grid = groups < per_sm * sms ? groups : per_sm * sms;
   act_quant_kernel<ACT_BITS, TPR, CPT>
-      <<<grid, 256, 0, st>>>(x, M, K, cinv, sid, alpha, S, step, qx, s_tok);
+      <<<grid, 256, smem, st>>>(x, M, K, cinv, sid, alpha, S, step, qx, s_tok);
   return cudaGetLastError();
 }
 
