@@ -71,14 +71,32 @@ wq_status linear(const wq_bf16* x, int M, int K, int N, const float* cinv,
       (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
     return WQ_ERR_ALIGN;
   if (ws_bytes < wq_workspace_bytes(M, K, N, act_bits)) return WQ_ERR_ARG;
+  // workspace: codes | token scales | split-K partial tiles | split-K counters
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* qx = ws;
-  float* s_tok = reinterpret_cast<float*>(ws + round_up(act_bytes(M, K, act_bits)));
+  const size_t off_stok = round_up(act_bytes(M, K, act_bits));
+  float* s_tok = reinterpret_cast<float*>(ws + off_stok);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  wq::SplitScratch scratch{nullptr, nullptr};
+  const int splits = wq::gemm_splits(M, N, K);
+  const size_t off_part = off_stok + round_up(sizeof(float) * static_cast<size_t>(M));
+  const size_t split_bytes = wq::gemm_split_scratch_bytes(M, N, K);
+  if (splits > 1) {
+    const int BN = wq::bn_for(M);
+    const size_t tiles = static_cast<size_t>((M + BN - 1) / BN) * ((N + 127) / 128);
+    const size_t part_bytes = round_up(tiles * BN * 128 * sizeof(int32_t));
+    scratch.partial = reinterpret_cast<int32_t*>(ws + off_part);
+    scratch.counters = reinterpret_cast<int*>(ws + off_part + part_bytes);
+  }
+  // the quantizer also clears the split-K accumulators and counters
   WQ_TRY(from_cuda(wq::launch_act_quant(x, M, K, cinv, stream_id, alpha, S, step, act_bits, qx,
-                                        s_tok, st)));
+                                        s_tok, st, splits > 1 ? ws + off_part : nullptr,
+                                        splits > 1 ? split_bytes : 0)));
   const wq::EpilogueArgs ep{s_tok, stream_id, s_w, bias, beta, S, step};
-  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, y, false, st));
+  // weights may stream while the quantizer runs (it started the GEMM only after
+  // everything before it in the stream had finished)
+  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, y, false,
+                                   splits > 1 ? &scratch : nullptr, st, /*w_prefetch=*/true));
 }
 
 // ------------------------------------------------------------ no-alloc variant
@@ -140,7 +158,8 @@ int wq_version(void) { return 100; }
 size_t wq_workspace_bytes(int M, int K, int N, int act_bits) {
   if ((act_bits != 8 && act_bits != 4) || check_mk(M, K) != WQ_OK || check_n(N) != WQ_OK)
     return 0;
-  return round_up(act_bytes(M, K, act_bits)) + round_up(sizeof(float) * static_cast<size_t>(M));
+  return round_up(act_bytes(M, K, act_bits)) + round_up(sizeof(float) * static_cast<size_t>(M)) +
+         wq::gemm_split_scratch_bytes(M, N, K);
 }
 
 wq_status wq_channel_scale(const wq_bf16* x_cal, int Mcal, const wq_bf16* W, int N, int K,
@@ -181,7 +200,7 @@ wq_status wq_gemm_w4ax(const void* qx, const float* s_tok, int act_bits, int M, 
   WQ_TRY(gemm_checks(qx, s_tok, act_bits, M, K, N, stream_id, beta, S, T, step, qw, s_w, bias,
                      y));
   const wq::EpilogueArgs ep{s_tok, stream_id, s_w, bias, beta, S, step};
-  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, y, false,
+  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, y, false, nullptr,
                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -212,8 +231,10 @@ wq_status wq_debug_gemm_s32(const void* qx, int act_bits, const uint8_t* qw, int
   if (!qx || !qw || !acc) return WQ_ERR_NULL;
   if (!aligned16(qx) || !aligned16(qw) || !aligned16(acc)) return WQ_ERR_ALIGN;
   const wq::EpilogueArgs ep{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 0};
-  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, acc, true,
-                                   reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (wq::gemm_splits(M, N, K) > 1)  // the K splits add into the output
+    WQ_TRY(from_cuda(cudaMemsetAsync(acc, 0, sizeof(int32_t) * static_cast<size_t>(M) * N, st)));
+  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, acc, true, nullptr, st));
 }
 
 wq_status wq_linear_w4a8_noalloc(const wq_bf16* x, int M, int K, int N, const float* cinv,

@@ -38,8 +38,28 @@ struct TileArgs {
   int M, N, K;
   int tiles_m, tiles_n, num_tiles;
   int n_fastest;
+  int splits;     // K ranges per tile (1: no split)
+  int num_units;  // num_tiles * splits work units, unit = tile * splits + split
+  int32_t* partial;  // bf16 split: [tiles][BN][128] int32 sums of the splits (zeroed)
+  int* counters;     // bf16 split: [tiles][8] arrivals per epilogue-warp slice
+  int w_prefetch;    // weights of the first NS K blocks loaded before griddep_wait()
   EpilogueArgs ep;
 };
+
+// K-block range of split `sp` of `splits` (balanced).
+__device__ __forceinline__ void split_range(int num_k, int splits, int sp, int& kb0, int& kb1) {
+  kb0 = (sp * num_k) / splits;
+  kb1 = ((sp + 1) * num_k) / splits;
+}
+
+// Upper bound on the TMA stages in flight per CTA (the shared-memory budget
+// decides below it).
+#ifndef WQ_MAX_STAGES
+#define WQ_MAX_STAGES 8
+#endif
+#ifndef WQ_UNPACK_WARPS_A8
+#define WQ_UNPACK_WARPS_A8 4
+#endif
 
 template <int BN_, int ACT_BITS_, bool OUT_S32_>
 struct Cfg {
@@ -48,13 +68,21 @@ struct Cfg {
   static constexpr bool OUT_S32 = OUT_S32_;
   static constexpr int BM = 128;  // output channels per tile (MMA M)
   static constexpr int BK = 128;  // K elements per pipeline stage
-  static constexpr int UNPACK_WARPS = ACT_BITS == 4 ? 8 : 4;
+  static constexpr int UNPACK_WARPS = ACT_BITS == 4 ? 8 : WQ_UNPACK_WARPS_A8;
   static constexpr int EPI_WARPS = 8;  // two per TMEM lane quadrant
   static constexpr int EPI_THREADS = EPI_WARPS * 32;
-  static constexpr int FIRST_UNPACK_WARP = 2;
-  static constexpr int FIRST_EPI_WARP = FIRST_UNPACK_WARP + UNPACK_WARPS;
-  static constexpr int NUM_WARPS = FIRST_EPI_WARP + EPI_WARPS;
+  // Warp roles: warp 0 issues TMA, warp 1 issues MMAs, then the unpack warps,
+  // then the epilogue warps (two per TMEM lane quadrant, warp % 4).
+  static constexpr int NUM_WARPS = 2 + UNPACK_WARPS + EPI_WARPS;
   static constexpr int THREADS = NUM_WARPS * 32;
+  // index among the unpack warps, or -1
+  __device__ static int unpack_index(int w) {
+    return (w >= 2 && w < 2 + UNPACK_WARPS) ? w - 2 : -1;
+  }
+  // index among the epilogue warps (quadrant w % 4, half e / 4), or -1
+  __device__ static int epi_index(int w) {
+    return (w >= 2 + UNPACK_WARPS && w < NUM_WARPS) ? w - 2 - UNPACK_WARPS : -1;
+  }
 
   static constexpr int WP_BYTES = BM * BK / 2;                               // packed W
   static constexpr int WU_BYTES = BM * BK;                                   // int8 W
@@ -84,7 +112,7 @@ struct Cfg {
   static constexpr int EPI_NBUF = NS_WITH_2 >= 4 ? 2 : 1;
   static constexpr int EPI_BYTES = EPI_WARPS * EPI_NBUF * EPI_BUF_BYTES;
   static constexpr int NS_FIT = (SMEM_LIMIT - FIXED - EPI_BYTES) / STAGE_BYTES;
-  static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
+  static constexpr int NS = NS_FIT > WQ_MAX_STAGES ? WQ_MAX_STAGES : NS_FIT;
   static_assert(NS >= NU && NS >= 2, "the done ring needs NS >= NU");
   static_assert(BN % EPI_CHUNK == 0 && NUM_CHUNKS >= 1, "token tile is a multiple of 16");
 
@@ -221,27 +249,49 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // Every CTA of this grid is resident (at most one per SM): the next kernel may
+  // be launched now; it waits for this one before touching its data.
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     // K block g (counted over all of this CTA's tiles) goes to stage g % NS once
     // the MMA has finished K block g - NS, the previous user of that stage.
     if (lane == 0) {
+      // The first NS stages' weights do not depend on the previous kernel when
+      // the caller says so: start streaming them before waiting for it.
+      uint32_t pre = 0;
+      if (args.w_prefetch) {
+        for (int unit = blockIdx.x; unit < args.num_units && pre < C::NS; unit += gridDim.x) {
+          int n_tile, m_tile, kb0, kb1;
+          decode_tile(args, unit / args.splits, n_tile, m_tile);
+          split_range(num_k, args.splits, unit % args.splits, kb0, kb1);
+          for (int kb = kb0; kb < kb1 && pre < C::NS; ++kb, ++pre) {
+            mbar_arrive_expect_tx(&full[pre], C::STAGE_BYTES);
+            tma_load_2d(smem + C::OFF_WP + pre * C::WP_BYTES, &tm_w, &full[pre],
+                        kb * (C::BK / 2), n_tile * C::BM);
+          }
+        }
+      }
+      griddep_wait();
       uint32_t g = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
-        int n_tile, m_tile;
-        decode_tile(args, tile, n_tile, m_tile);
-        for (int kb = 0; kb < num_k; ++kb, ++g) {
+      for (int unit = blockIdx.x; ok && unit < args.num_units; unit += gridDim.x) {
+        int n_tile, m_tile, kb0, kb1;
+        decode_tile(args, unit / args.splits, n_tile, m_tile);
+        split_range(num_k, args.splits, unit % args.splits, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb, ++g) {
           const uint32_t s = g % C::NS;
-          if (g >= static_cast<uint32_t>(C::NS) &&
-              !mbar_wait(&done[s], ((g / C::NS) - 1) & 1u)) {
-            ok = false;
-            break;
+          if (g >= pre) {  // else: expect_tx and the weight load were issued above
+            if (g >= static_cast<uint32_t>(C::NS) &&
+                !mbar_wait(&done[s], ((g / C::NS) - 1) & 1u)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+            tma_load_2d(smem + C::OFF_WP + s * C::WP_BYTES, &tm_w, &full[s], kb * (C::BK / 2),
+                        n_tile * C::BM);
           }
-          mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-          tma_load_2d(smem + C::OFF_WP + s * C::WP_BYTES, &tm_w, &full[s], kb * (C::BK / 2),
-                      n_tile * C::BM);
           tma_load_2d(smem + C::OFF_XS + s * C::XS_BYTES, &tm_x, &full[s],
                       kb * (C::ACT_BITS == 8 ? C::BK : C::BK / 2), m_tile * C::BN);
         }
@@ -265,11 +315,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       int b = 0;
       uint32_t ph_b = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+      for (int unit = blockIdx.x; ok && unit < args.num_units; unit += gridDim.x) {
+        int kb0, kb1;
+        split_range(num_k, args.splits, unit % args.splits, kb0, kb1);
         if (!mbar_wait(&tempty[b], ph_b ^ 1u)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * C::BN);
-        for (int kb = 0; kb < num_k; ++kb, ++g) {
+        for (int kb = kb0; kb < kb1; ++kb, ++g) {
           const uint32_t s = g % C::NS, u = g % C::NU;
           if (!mbar_wait(&ufull[u], (g / C::NU) & 1u)) { ok = false; break; }
           tc_fence_after();
@@ -280,7 +332,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < C::BK / 32; ++kk)
             mma_i8_ss(d_tmem, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32),
-                      idesc, (kb | kk) != 0 ? 1u : 0u);
+                      idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
           mma_commit(&done[s]);
         }
         if (!ok) break;
@@ -289,16 +341,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
     }
     __syncwarp();
-  } else if (warp < C::FIRST_EPI_WARP) {
+  } else if (C::unpack_index(warp) >= 0) {
     // ------------------------------------------------------------ int4 -> int8
     // K block g: wait for its TMA stage and for the MMA to have finished K block
     // g - NU (the previous user of unpacked buffer g % NU).
-    const int tid = threadIdx.x - C::FIRST_UNPACK_WARP * 32;
+    const int tid = C::unpack_index(warp) * 32 + lane;
     constexpr int NT = C::UNPACK_WARPS * 32;
     uint32_t g = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
-      for (int kb = 0; kb < num_k; ++kb, ++g) {
+    for (int unit = blockIdx.x; ok && unit < args.num_units; unit += gridDim.x) {
+      int kb0, kb1;
+      split_range(num_k, args.splits, unit % args.splits, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb, ++g) {
         const uint32_t s = g % C::NS, u = g % C::NU;
         bool w = mbar_wait(&full[s], (g / C::NS) & 1u);
         if (g >= static_cast<uint32_t>(C::NU)) {
@@ -323,14 +377,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (lane == 0) mbar_arrive(&ufull[u]);
       }
     }
-  } else {
+  } else if (C::epi_index(warp) >= 0) {
     // ------------------------------------------------------------ epilogue
     // Warp e covers TMEM lanes 32q..32q+31 (output channels) and every other
     // 16-column chunk (tokens) of the tile, starting at chunk h.
-    const int e = warp - C::FIRST_EPI_WARP;
+    const int e = C::epi_index(warp);
     const int q = warp & 3;
     const int h = e >> 2;
-    const int et = threadIdx.x - C::FIRST_EPI_WARP * 32;
+    const int et = e * 32 + lane;
     uint8_t* ebuf = smem + C::OFF_EPI + e * C::EPI_NBUF * C::EPI_BUF_BYTES;
     float* tok_s = reinterpret_cast<float*>(smem + C::OFF_TOK);
     uint8_t* tok_id = smem + C::OFF_TOK + 2 * C::BN * 4;
@@ -338,7 +392,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint32_t ph_b = 0;
     const EpilogueArgs& ep = args.ep;
     const bool small_s = ep.S <= 4;
-    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++it) {
+    griddep_wait();  // token scales and split-K scratch come from the previous kernel
+    const bool split = args.splits > 1;
+    for (int unit = blockIdx.x; unit < args.num_units; unit += gridDim.x, ++it) {
+      const int tile = unit / args.splits;
       int n_tile, m_tile;
       decode_tile(args, tile, n_tile, m_tile);
       const int n_base = n_tile * C::BM + q * 32;
@@ -364,30 +421,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             bb[j] = (brow && j < ep.S && small_s) ? __fadd_rn(bs, brow[(size_t)j * args.N]) : bs;
         }
       }
-      // staging visible to every epilogue warp (and the warps kept within one tile)
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tokbar[it & 1]);
-      bool w = mbar_wait(&tokbar[it & 1], (it >> 1) & 1);
-      w = w && mbar_wait(&tfull[b], ph_b);
-      if (!__all_sync(0xFFFFFFFFu, w)) break;  // uniform, and converged for tcgen05.ld
-      tc_fence_after();
-      if (h >= C::NUM_CHUNKS) {  // no chunk for this warp (token tiles of 16)
-        tc_fence_before();
-        if (lane == 0) mbar_arrive(&tempty[b]);
-      }
-      const uint32_t tbase =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * C::BN);
-      for (int c = h; c < C::NUM_CHUNKS; c += 2) {
-        const int j0 = c * C::EPI_CHUNK;
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(tbase + j0, r);
-        tmem_wait_ld();
-        if (c + 2 >= C::NUM_CHUNKS) {  // last chunk of this warp: hand the accumulator back
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[b]);
-        }
-        if (m0 + j0 >= args.M) continue;  // whole chunk beyond the last token
+
+      // y for one 16-column chunk of accumulators (scaled by 2^ACC_SHIFT), through a
+      // shared-memory staging buffer and a TMA store; int32 view for OUT_S32.
+      auto emit = [&](const uint32_t (&r)[16], int j0) {
         uint8_t* sb = ebuf + buf * C::EPI_BUF_BYTES;
         if (lane == 0) {  // this buffer's previous TMA store has read it
           if constexpr (C::EPI_NBUF == 2) bulk_wait_group_read<1>();
@@ -442,6 +479,75 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           bulk_commit_group();
         }
         if constexpr (C::EPI_NBUF == 2) buf ^= 1;
+      };
+
+      // staging visible to every epilogue warp (and the warps kept within one tile)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tokbar[it & 1]);
+      bool w = mbar_wait(&tokbar[it & 1], (it >> 1) & 1);
+      w = w && mbar_wait(&tfull[b], ph_b);
+      if (!__all_sync(0xFFFFFFFFu, w)) break;  // uniform, and converged for tcgen05.ld
+      tc_fence_after();
+      if (h >= C::NUM_CHUNKS) {  // no chunk for this warp (token tiles of 16)
+        tc_fence_before();
+        if (lane == 0) mbar_arrive(&tempty[b]);
+      }
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * C::BN);
+      // split K: the tile's int32 accumulator (2^ACC_SHIFT-scaled), summed by red.add
+      int32_t* tile_acc = split && !C::OUT_S32
+                              ? args.partial + (size_t)tile * C::BN * C::BM + q * 32 + lane
+                              : nullptr;
+      for (int c = h; c < C::NUM_CHUNKS; c += 2) {
+        const int j0 = c * C::EPI_CHUNK;
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tbase + j0, r);
+        tmem_wait_ld();
+        if (c + 2 >= C::NUM_CHUNKS) {  // last chunk of this warp: hand the accumulator back
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[b]);
+        }
+        if (m0 + j0 >= args.M) continue;  // whole chunk beyond the last token
+        if (!split) {
+          emit(r, j0);
+        } else if constexpr (C::OUT_S32) {
+          // int32 view: the splits add into the zeroed output (exact in any order)
+          if (n < args.N) {
+            int32_t* col = static_cast<int32_t*>(args.out) + n;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (m0 + j0 + j < args.M)
+                atomicAdd(col + (size_t)(m0 + j0 + j) * args.N,
+                          static_cast<int32_t>(r[j]) >> C::ACC_SHIFT);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)  // exact in any order; no return value needed
+            atomicAdd(tile_acc + (j0 + j) * C::BM, static_cast<int32_t>(r[j]));
+        }
+      }
+      if (split && !C::OUT_S32 && h < C::NUM_CHUNKS) {
+        // The last of the tile's splits to finish this warp slice sums the
+        // partials (int32: exact in any order) and writes y.
+        __threadfence();
+        __syncwarp();
+        int* counter = args.counters + tile * C::EPI_WARPS + e;
+        int prev = 0;
+        if (lane == 0) prev = atomicAdd(counter, 1);
+        prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
+        if (prev == args.splits - 1) {
+          __threadfence();
+          for (int c = h; c < C::NUM_CHUNKS; c += 2) {
+            const int j0 = c * C::EPI_CHUNK;
+            if (m0 + j0 >= args.M) continue;
+            uint32_t r[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              r[j] = static_cast<uint32_t>(__ldcg(tile_acc + (j0 + j) * C::BM));
+            emit(r, j0);
+          }
+        }
       }
       if (++b == 2) { b = 0; ph_b ^= 1u; }
     }
@@ -500,9 +606,12 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
+int bn_for(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
+
 template <class C>
 cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
-                     const EpilogueArgs& ep, void* out, cudaStream_t st) {
+                     const EpilogueArgs& ep, void* out, const SplitScratch* scratch,
+                     cudaStream_t st, bool w_prefetch) {
   CUtensorMap tm_w, tm_x, tm_out;
   bool ok = make_map(&tm_w, qw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, C::BK / 2, C::BM,
                      CU_TENSOR_MAP_SWIZZLE_64B);
@@ -531,6 +640,11 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
   // Keep the smaller operand resident in L2: sweep output channels fastest when
   // the packed weights fit comfortably, so each activation tile streams once.
   a.n_fastest = (static_cast<size_t>(N) * K / 2) <= (48u << 20) ? 1 : 0;
+  a.splits = (C::OUT_S32 || scratch != nullptr) ? gemm_splits(M, N, K) : 1;
+  a.num_units = a.num_tiles * a.splits;
+  a.partial = scratch ? scratch->partial : nullptr;
+  a.counters = scratch ? scratch->counters : nullptr;
+  a.w_prefetch = w_prefetch ? 1 : 0;
   a.ep = ep;
 
   static bool attr_set = false;  // per template instance
@@ -540,31 +654,56 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int grid = a.num_tiles < sm_count() ? a.num_tiles : sm_count();
-  gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tm_w, tm_x, tm_out, a);
-  return cudaGetLastError();
+  const int grid = a.num_units < sm_count() ? a.num_units : sm_count();
+  return launch_pdl(gemm_kernel<C>, grid, C::THREADS, C::SMEM_BYTES, st, tm_w, tm_x, tm_out, a);
 }
 
 template <int ACT_BITS, bool OUT_S32>
 cudaError_t dispatch_bn(const void* qx, const uint8_t* qw, int M, int N, int K,
-                        const EpilogueArgs& ep, void* out, cudaStream_t st) {
-  if (M <= 16) return run_gemm<Cfg<16, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, st);
-  if (M <= 32) return run_gemm<Cfg<32, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, st);
-  if (M <= 64) return run_gemm<Cfg<64, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, st);
-  if (M <= 128) return run_gemm<Cfg<128, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, st);
-  return run_gemm<Cfg<256, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, st);
+                        const EpilogueArgs& ep, void* out, const SplitScratch* sc,
+                        cudaStream_t st, bool wp) {
+  switch (bn_for(M)) {
+    case 16: return run_gemm<Cfg<16, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, sc, st, wp);
+    case 32: return run_gemm<Cfg<32, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, sc, st, wp);
+    case 64: return run_gemm<Cfg<64, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, sc, st, wp);
+    case 128: return run_gemm<Cfg<128, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, sc, st, wp);
+    default: return run_gemm<Cfg<256, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, sc, st, wp);
+  }
 }
 
 }  // namespace
 
+int gemm_splits(int M, int N, int K) {
+  const int BN = bn_for(M);
+  const int tiles = ((M + BN - 1) / BN) * ((N + 127) / 128);
+  const int num_k = K / 128;
+  if (tiles * 2 > kSplitTargetCtas) return 1;
+  int s = kSplitTargetCtas / tiles;
+  const int cap = num_k / 2 > 1 ? num_k / 2 : 1;  // at least two K blocks per split
+  s = s < cap ? s : cap;
+  return s > 1 ? s : 1;
+}
+
+size_t gemm_split_scratch_bytes(int M, int N, int K) {
+  const int splits = gemm_splits(M, N, K);
+  if (splits == 1) return 0;
+  const int BN = bn_for(M);
+  const size_t tiles = static_cast<size_t>((M + BN - 1) / BN) * ((N + 127) / 128);
+  const size_t partial = tiles * BN * 128 * sizeof(int32_t);
+  const size_t counters = tiles * 8 * sizeof(int);
+  return (partial + 255) / 256 * 256 + (counters + 255) / 256 * 256;
+}
+
 cudaError_t launch_gemm(const void* qx, int act_bits, const uint8_t* qw, int M, int N, int K,
-                        const EpilogueArgs& ep, void* out, bool out_s32, cudaStream_t st) {
+                        const EpilogueArgs& ep, void* out, bool out_s32,
+                        const SplitScratch* scratch, cudaStream_t st, bool w_prefetch) {
   if (M == 0) return cudaSuccess;
+  const bool wp = w_prefetch;
   if (act_bits == 8)
-    return out_s32 ? dispatch_bn<8, true>(qx, qw, M, N, K, ep, out, st)
-                   : dispatch_bn<8, false>(qx, qw, M, N, K, ep, out, st);
-  return out_s32 ? dispatch_bn<4, true>(qx, qw, M, N, K, ep, out, st)
-                 : dispatch_bn<4, false>(qx, qw, M, N, K, ep, out, st);
+    return out_s32 ? dispatch_bn<8, true>(qx, qw, M, N, K, ep, out, scratch, st, wp)
+                   : dispatch_bn<8, false>(qx, qw, M, N, K, ep, out, scratch, st, wp);
+  return out_s32 ? dispatch_bn<4, true>(qx, qw, M, N, K, ep, out, scratch, st, wp)
+                 : dispatch_bn<4, false>(qx, qw, M, N, K, ep, out, scratch, st, wp);
 }
 
 }  // namespace wq

@@ -9,6 +9,25 @@
 
 namespace wq {
 
+// Launch with programmatic stream serialization: the kernel may start while the
+// previous kernel in the stream is still running, and must call griddep_wait()
+// before it touches anything that kernel (or an earlier one) writes.
+template <class... KArgs, class... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Largest K the quantizer keeps in registers (K/8 chunks spread over 256 threads,
 // at most 16 chunks each).
 constexpr int kMaxK = 32768;
@@ -19,9 +38,12 @@ cudaError_t launch_channel_scale(const uint16_t* x_cal, int Mcal, const uint16_t
 cudaError_t launch_pack_int4(const uint16_t* W, const float* c, int N, int K, uint8_t* qw,
                              float* s_w, cudaStream_t st);
 
+// `zero` (16-byte aligned, zero_bytes a multiple of 16) is cleared by the same
+// launch: the fused linear uses it for the GEMM's split-K scratch.
 cudaError_t launch_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                              const uint8_t* stream_id, const float* alpha, int S, int step,
-                             int act_bits, void* qx, float* s_tok, cudaStream_t st);
+                             int act_bits, void* qx, float* s_tok, cudaStream_t st,
+                             void* zero = nullptr, size_t zero_bytes = 0);
 
 // Epilogue inputs of the fused GEMM.
 struct EpilogueArgs {
@@ -34,9 +56,30 @@ struct EpilogueArgs {
   int step;
 };
 
+// Split-K (small token counts): the K blocks of each output tile are spread over
+// `splits` CTAs so that about kSplitTargetCtas CTAs stream the weights.  The
+// bf16 path needs scratch for the int32 partial tiles and one counter per
+// epilogue-warp slice of each tile; the int32 debug path adds its partials
+// atomically into the (zeroed) output instead.
+constexpr int kSplitTargetCtas = 148;
+int gemm_splits(int M, int N, int K);
+size_t gemm_split_scratch_bytes(int M, int N, int K);  // partials + counters, 0 if no split
+
+struct SplitScratch {
+  int32_t* partial;  // [tiles][BN][128] int32 sums of the splits, zero before the launch
+  int* counters;     // [tiles][8], zero before the launch
+};
+
 // y[M][N] (bf16) = epilogue(qx x qw^T) when out_s32 == false; acc[M][N] (int32)
-// when out_s32 == true (the epilogue arguments are then ignored).
+// when out_s32 == true (the epilogue arguments are then ignored).  bf16 with
+// scratch == nullptr never splits K; out_s32 splits into atomics on `out`,
+// which the caller must have zeroed when gemm_splits() > 1.
+// w_prefetch: the packed weights (and nothing else) may be read before the
+// previous kernel in the stream has finished.  Only valid when that kernel is
+// this library's quantizer, which starts its dependents only after everything
+// launched before it has completed.
 cudaError_t launch_gemm(const void* qx, int act_bits, const uint8_t* qw, int M, int N, int K,
-                        const EpilogueArgs& ep, void* out, bool out_s32, cudaStream_t st);
+                        const EpilogueArgs& ep, void* out, bool out_s32,
+                        const SplitScratch* scratch, cudaStream_t st, bool w_prefetch = false);
 
 }  // namespace wq

@@ -124,7 +124,7 @@ template <int ACT_BITS, int TPR, int CPT>
 __global__ void __launch_bounds__(256) act_quant_kernel(
     const uint16_t* __restrict__ x, int M, int K, const float* __restrict__ cinv,
     const uint8_t* __restrict__ stream_id, const float* __restrict__ alpha, int S, int step,
-    void* __restrict__ qx, float* __restrict__ s_tok) {
+    void* __restrict__ qx, float* __restrict__ s_tok, uint4* __restrict__ zero, size_t zero_n16) {
   constexpr int RPC = 256 / TPR;  // rows per CTA pass
   constexpr int WPR = TPR / 32;   // warps per row
   constexpr int QMAX = ACT_BITS == 8 ? 127 : 7;
@@ -132,6 +132,15 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
   float* cinv_s = reinterpret_cast<float*>(cinv_s4);
   __shared__ float red[8];
 
+  // Everything this kernel reads or writes may belong to the previous kernel in
+  // the stream; once that has finished, the GEMM that follows may start its
+  // prologue (and its weight loads) while this one runs.
+  griddep_wait();
+  griddep_launch_dependents();
+  // Clear the next GEMM's split-K accumulators and counters (16-byte words) here
+  // rather than in a separate launch.
+  for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < zero_n16; i += (size_t)gridDim.x * 256)
+    zero[i] = make_uint4(0u, 0u, 0u, 0u);
   for (int k = threadIdx.x * 4; k < K; k += 256 * 4)
     *reinterpret_cast<float4*>(cinv_s + k) =
         cinv ? __ldg(reinterpret_cast<const float4*>(cinv + k)) : make_float4(1.f, 1.f, 1.f, 1.f);
@@ -216,35 +225,41 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
 template <int ACT_BITS, int TPR, int CPT>
 cudaError_t run_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                           const uint8_t* sid, const float* alpha, int S, int step, void* qx,
-                          float* s_tok, cudaStream_t st) {
+                          float* s_tok, uint4* zero, size_t zero_n16, cudaStream_t st) {
   constexpr int RPC = 256 / TPR;
   const size_t smem = static_cast<size_t>(K) * sizeof(float);  // cinv copy
-  static int per_sm = 0;  // resident CTAs per SM at the largest K (per template instance)
-  if (per_sm == 0) {
+  static bool attr_set = false;  // per template instance
+  static int per_sm = 0, per_sm_k = 0;  // resident CTAs per SM at K = per_sm_k
+  if (!attr_set) {
     if (cudaFuncSetAttribute(act_quant_kernel<ACT_BITS, TPR, CPT>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxK * 4) != cudaSuccess)
       return cudaGetLastError();
+    attr_set = true;
+  }
+  if (per_sm_k != K) {
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, act_quant_kernel<ACT_BITS, TPR, CPT>,
                                                   256, smem);
     if (per_sm < 1) per_sm = 1;
+    per_sm_k = K;
   }
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int groups = (M + RPC - 1) / RPC;
   const int grid = groups < per_sm * sms ? groups : per_sm * sms;
-  act_quant_kernel<ACT_BITS, TPR, CPT>
-      <<<grid, 256, smem, st>>>(x, M, K, cinv, sid, alpha, S, step, qx, s_tok);
-  return cudaGetLastError();
+  return launch_pdl(act_quant_kernel<ACT_BITS, TPR, CPT>, grid, 256, smem, st, x, M, K, cinv, sid,
+                    alpha, S, step, qx, s_tok, zero, zero_n16);
 }
 
 template <int ACT_BITS>
 cudaError_t dispatch_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                                const uint8_t* sid, const float* alpha, int S, int step,
-                               void* qx, float* s_tok, cudaStream_t st) {
+                               void* qx, float* s_tok, uint4* zero, size_t zero_n16,
+                               cudaStream_t st) {
   const int nchunk = K / 8;
 #define WQ_AQ(TPR, CPT) \
-  return run_act_quant<ACT_BITS, TPR, CPT>(x, M, K, cinv, sid, alpha, S, step, qx, s_tok, st)
+  return run_act_quant<ACT_BITS, TPR, CPT>(x, M, K, cinv, sid, alpha, S, step, qx, s_tok, zero, \
+                                           zero_n16, st)
   // one warp per row up to K = 2048 (no block-level reduction), 8 chunks of 8
   // channels per thread beyond that
   if (nchunk <= 32) WQ_AQ(32, 1);
@@ -319,11 +334,14 @@ __global__ void channel_scale_kernel(const uint16_t* __restrict__ x_cal, int Mca
 
 cudaError_t launch_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                              const uint8_t* stream_id, const float* alpha, int S, int step,
-                             int act_bits, void* qx, float* s_tok, cudaStream_t st) {
+                             int act_bits, void* qx, float* s_tok, cudaStream_t st,
+                             void* zero, size_t zero_bytes) {
   if (M == 0) return cudaSuccess;
+  uint4* z = static_cast<uint4*>(zero);
+  const size_t n16 = zero ? zero_bytes / 16 : 0;
   if (act_bits == 8)
-    return dispatch_act_quant<8>(x, M, K, cinv, stream_id, alpha, S, step, qx, s_tok, st);
-  return dispatch_act_quant<4>(x, M, K, cinv, stream_id, alpha, S, step, qx, s_tok, st);
+    return dispatch_act_quant<8>(x, M, K, cinv, stream_id, alpha, S, step, qx, s_tok, z, n16, st);
+  return dispatch_act_quant<4>(x, M, K, cinv, stream_id, alpha, S, step, qx, s_tok, z, n16, st);
 }
 
 cudaError_t launch_pack_int4(const uint16_t* W, const float* c, int N, int K, uint8_t* qw,

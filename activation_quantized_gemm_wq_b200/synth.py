@@ -107,6 +107,14 @@ def small_m(parent: Workload, M: int, mix: str, act_bits: int) -> Workload:
                         act_bits=act_bits, T=10)
 
 
+# the small-M batches by name (weights and tables of the parent block)
+for _parent in (BLOCK2048_A8, BLOCK4096_A8):
+    for _bits in (8, 4):
+        for _M in SMALL_M:
+            _w = small_m(_parent, _M, "action", _bits)
+            WORKLOADS[_w.name] = _w
+
+
 def custom(name: str, K: int, N: int, rows: Sequence[Tuple[int, int]], act_bits: int = 8,
            T: int = 1, stds=(1.0, 3.0, 0.5), outlier_frac: float = 0.01,
            outlier_range=(20.0, 50.0)) -> Workload:

@@ -20,6 +20,7 @@ work ("scaling": "weak").  --impl reference times the CPU oracle instead.
 """
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -51,8 +52,12 @@ def parse():
     p.add_argument("--workload", default="block2048_w4a8", choices=sorted(S.WORKLOADS))
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-graph", action="store_true",
+                   help="launch every call from the host instead of replaying one CUDA graph "
+                        "per step")
     p.add_argument("--sweep", action="store_true",
                    help="per-shape table over every configured workload (not the JSON line)")
+    p.add_argument("--sweep-filter", default="", help="only sweep entries whose label has this")
     return p.parse_args()
 
 
@@ -223,44 +228,84 @@ def run_gpu(args, rank, world, local):
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     T = wl.T
+    lin_fn = {8: wq.wq_linear_w4a8, 4: wq.wq_linear_w4a4}
 
-    def step(it, gemm_events=None):
+    def step(it):
+        """One pass of the hot path: the fused public call for every linear."""
+        t = it % T
+        r = it % n_sets
+        for L in layers:
+            lin_fn[L.bits](L.x[r], L.cinv, L.sid, L.alpha, L.beta, t, L.qw, L.s_w, L.bias, L.y,
+                           L.ws)
+
+    def step_split(it, gemm_events):
+        """The same pass as two calls per linear, with events around each GEMM."""
         t = it % T
         r = it % n_sets
         for j, L in enumerate(layers):
             wq.wq_act_quant(L.x[r], L.cinv, L.sid, L.alpha, t, L.bits, L.qx, L.s_tok)
-            if gemm_events is not None:
-                gemm_events[j][0].record(stream)
+            gemm_events[j][0].record(stream)
             wq.wq_gemm_w4ax(L.qx, L.s_tok, L.bits, L.K, L.sid, L.beta, L.S, L.T, t, L.qw, L.s_w,
                             L.bias, L.y)
-            if gemm_events is not None:
-                gemm_events[j][1].record(stream)
+            gemm_events[j][1].record(stream)
+
+    # one CUDA graph per distinct step (denoising step t x activation set r)
+    period = T * n_sets // math.gcd(T, n_sets)
+    for it in range(period):  # first-use setup outside capture
+        step(it)
+    torch.cuda.synchronize()
+    if args.no_graph:
+        run = step
+    else:
+        graphs = []
+        for it in range(period):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(it)
+            graphs.append(g)
+
+        def run(it):
+            graphs[it % period].replay()
 
     for it in range(args.warmup):
-        step(it)
+        run(it)
     torch.cuda.synchronize()
     assert wq.wq_device_status() == ("WQ_OK", 0)
 
     clocks = ClockSampler(local)
     clocks.start()
-    ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-           for _ in layers] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     clocks.t0 = time.time()
     start.record(stream)
     for it in range(args.steps):
-        step(args.warmup + it, ev[it])
+        run(args.warmup + it)
     end.record(stream)
     torch.cuda.synchronize()
     clocks.t1 = time.time()
     barrier(world)
     clocks.stop()
     elapsed_ms = start.elapsed_time(end)
-    gemm_ms = sum(a.elapsed_time(b) for per_step in ev for a, b in per_step)
     status = wq.wq_device_status()
     assert status == ("WQ_OK", 0), status
+
+    # the dominant kernel's launch duration: the same steps again, launched from the
+    # host as quantizer + GEMM calls with an event pair around every GEMM
+    ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+           for _ in layers] for _ in range(args.steps)]
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s0.record(stream)
+    for it in range(args.steps):
+        step_split(args.warmup + it, ev[it])
+    s1.record(stream)
+    torch.cuda.synchronize()
+    split_ms = s0.elapsed_time(s1)
+    gemm_ms = sum(a.elapsed_time(b) for per_step in ev for a, b in per_step)
+    assert wq.wq_device_status() == ("WQ_OK", 0)
+    if not args.no_graph:
+        del graphs
 
     t_max = max_over_ranks(elapsed_ms, world)
     ops_step = sum(L.ops() for L in layers)
@@ -313,8 +358,13 @@ def run_gpu(args, rank, world, local):
             "peak_source": f"{src} bf16 burst {bf16_burst} TFLOP/s x{INT8_PER_BF16} (dense int8 "
                            "/ bf16 nominal ratio); units are int8 tera-ops",
             "gemm_avg_launch_ms": round(gemm_avg_ms, 5),
-            "gemm_share_of_step": round(gemm_ms / (t_max if world == 1 else elapsed_ms), 4),
+            "gemm_share_of_step": round(gemm_ms / split_ms, 4),
+            "measured": "event pair around every GEMM launch in a second pass of the same "
+                        f"{args.steps} steps (quantizer + GEMM calls from the host)",
         },
+        "timing": ("one CUDA graph replay per step (fused wq_linear calls; the GEMM starts "
+                   "under the quantizer by programmatic dependent launch)"
+                   if not args.no_graph else "host launches, fused wq_linear calls"),
         "clocks": clocks.summary(),
         "e2e": e2e,
         "gpu_launches": 2 * len(layers) * args.steps,
@@ -475,11 +525,175 @@ def run_reference(args, rank, world):
     }
 
 
+# ------------------------------------------------------------------ per-config sweep
+
+def _median_ms(torch, fn, warm=5, reps=20):
+    """Median of `reps` event-timed calls after `warm` warm-ups (the pages' protocol:
+    20 timed repetitions after 5 warm-ups)."""
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def _graph_ms(torch, fns, replays=5):
+    """Per-call time of a CUDA graph holding every call in `fns` once."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for f in fns:  # warm-up outside capture (first-use attribute setup)
+            f()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for f in fns:
+            f()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(replays):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / (replays * len(fns))
+    del g
+    return ms
+
+
+def _alg_bytes(M, N, K, bits, S_used=3):
+    """Algorithmic bytes of one linear: K1 (x in, codes and scales out) and K2
+    (codes, packed weights, scales, bias, used beta rows, ids in; y out)."""
+    codes = M * K if bits == 8 else M * K // 2
+    k1 = 2 * M * K + 4 * K + M + codes + 4 * M
+    k2 = codes + 4 * M + M + N * K // 2 + 4 * N + 4 * N + 4 * N * S_used + 2 * M * N
+    return k1, k2
+
+
+def sweep(args):
+    """Every configured workload: GEMM-only and whole-linear throughput per linear, as
+    absolute numbers and as a fraction of the binding roofline."""
+    import torch
+
+    import activation_quantized_gemm_wq_b200 as wq
+
+    bf16_burst, _, hbm, src = peaks()
+    p_int8 = bf16_burst * INT8_PER_BF16 * 1e12  # ops/s
+    bw = hbm * 1e9
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+
+    def dev(a):
+        a = np.ascontiguousarray(a)
+        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
+
+    entries = [("0 tiny", S.TINY, [0])]
+    entries += [("1 block2048 A8", S.BLOCK2048_A8, [0, 1, 2, 3])]
+    entries += [("2 block2048 A4 T10", S.BLOCK2048_A4, [0, 1, 2, 3])]
+    entries += [("3 block4096 A8 T10", S.BLOCK4096_A8, [0, 1, 2, 3])]
+    entries += [("3 block4096 A4 T10", S.BLOCK4096_A4, [0, 1, 2, 3])]
+    for parent in (S.BLOCK2048_A8, S.BLOCK4096_A8):
+        for li in range(4):  # weights outermost: generated once per shape
+            for bits in (8, 4):
+                for M in S.SMALL_M:
+                    entries.append((f"4 small-M {parent.name.split('_')[0]} A{bits} M{M}",
+                                    S.small_m(parent, M, "action", bits), [li]))
+    rows = []
+    cache = {}
+    for label, wl, layers in entries:
+        if args.sweep_filter and args.sweep_filter not in label:
+            continue
+        for li in layers:
+            lin = wl.linears[li]
+            M, K, N, bits = wl.M, lin.K, lin.N, wl.act_bits
+            key = (wl.name.split("_m")[0].split("_w")[0], li)
+            if key not in cache:
+                L = S.layer_inputs(wl, li)
+                c = torch.empty(K, dtype=torch.float32, device="cuda")
+                cinv = torch.empty_like(c)
+                qw = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+                s_w = torch.empty(N, dtype=torch.float32, device="cuda")
+                W = dev(L.W)
+                wq.wq_channel_scale(dev(L.x_cal), W, c, cinv)
+                wq.wq_pack_int4(W, c, qw, s_w)
+                cache.clear()
+                cache[key] = (L, cinv, qw, s_w, W)
+            L, cinv, qw, s_w, W = cache[key]
+            T = wl.T  # tables sized to this workload (values only matter for parity)
+            alpha = dev(np.resize(L.alpha, (T, 3)).astype(np.float32))
+            beta = dev(np.resize(L.beta, (T, 3, N)).astype(np.float32))
+            bias = dev(L.bias)
+            sid = dev(S.stream_ids(wl))
+            # rotate input copies (activations, codes, weights) totalling more than 2x L2
+            per_copy = 2 * M * K + (M * K if bits == 8 else M * K // 2) + N * K // 2
+            ncopy = max(1, int(np.ceil(2 * l2 / per_copy)))
+            xs, qxs, qws = [], [], []
+            for r in range(ncopy):
+                xs.append(dev(S.activations(wl, li, 0, seed=r)) if r < 2 else xs[r % 2].clone())
+                qxs.append(torch.empty((M, K) if bits == 8 else (M, K // 2),
+                                       dtype=torch.int8 if bits == 8 else torch.uint8,
+                                       device="cuda"))
+                qws.append(qw if r == 0 else qw.clone())
+            x = xs[0]
+            s_tok = torch.empty(M, dtype=torch.float32, device="cuda")
+            y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            ws = wq.alloc_workspace(M, K, N, bits)
+            lin_fn = wq.wq_linear_w4a8 if bits == 8 else wq.wq_linear_w4a4
+            step = T - 1
+            for r in range(ncopy):
+                wq.wq_act_quant(xs[r], cinv, sid, alpha, step, bits, qxs[r], s_tok)
+            calls = max(10, ncopy)
+            g_fns = [lambda r=r: wq.wq_gemm_w4ax(qxs[r % ncopy], s_tok, bits, K, sid, beta, 3, T,
+                                                 step, qws[r % ncopy], s_w, bias, y)
+                     for r in range(calls)]
+            l_fns = [lambda r=r: lin_fn(xs[r % ncopy], cinv, sid, alpha, beta, step,
+                                        qws[r % ncopy], s_w, bias, y, ws) for r in range(calls)]
+            t_gemm = _graph_ms(torch, g_fns)
+            t_lin = _graph_ms(torch, l_fns)
+            timing = f"CUDA graph of {calls} calls over {ncopy} input copies"
+            del g_fns, l_fns, qws, qxs
+            xb = x.view(torch.bfloat16)
+            wb = W.view(torch.bfloat16)
+            t_bf16 = _graph_ms(torch, [lambda: torch.nn.functional.linear(xb, wb)] * 10)
+            ops = 2 * M * N * K
+            k1b, k2b = _alg_bytes(M, N, K, bits)
+            roof_gemm = max(ops / p_int8, k2b / bw) * 1e3
+            roof_lin = max(ops / p_int8, (k1b + k2b) / bw) * 1e3
+            bound = "tensor" if ops / p_int8 >= k2b / bw else "hbm"
+            rows.append(dict(config=label, linear=f"{lin.name} {K}->{N}", M=M, bits=bits,
+                             gemm_us=round(t_gemm * 1e3, 2), linear_us=round(t_lin * 1e3, 2),
+                             gemm_tops=round(ops / t_gemm / 1e9, 1),
+                             linear_tops=round(ops / t_lin / 1e9, 1),
+                             gemm_gbs=round(k2b / t_gemm / 1e6, 1),
+                             linear_gbs=round((k1b + k2b) / t_lin / 1e6, 1),
+                             bound=bound, gemm_frac=round(roof_gemm / t_gemm, 3),
+                             linear_frac=round(roof_lin / t_lin, 3),
+                             bf16_us=round(t_bf16 * 1e3, 2), timing=timing))
+            print(json.dumps(rows[-1]), flush=True)
+            del x, xs, y, ws
+        assert wq.wq_device_status() == ("WQ_OK", 0)
+    print(f"# peaks ({src}): int8 {p_int8 / 1e12:.0f} TOPS (bf16 burst x2), HBM {hbm} GB/s")
+    print("| config | linear | M | bits | GEMM us | GEMM TOPS | GEMM GB/s | linear us | "
+          "linear TOPS | bound | GEMM frac | linear frac | torch bf16 us |")
+    print("|---|---|---|---|---|---|---|---|---|---|---|---|---|")
+    for r in rows:
+        print(f"| {r['config']} | {r['linear']} | {r['M']} | {r['bits']} | {r['gemm_us']} | "
+              f"{r['gemm_tops']} | {r['gemm_gbs']} | {r['linear_us']} | {r['linear_tops']} | "
+              f"{r['bound']} | {r['gemm_frac']} | {r['linear_frac']} | {r['bf16_us']} |")
+
+
 def main():
     args = parse()
     if args.sweep:
-        from activation_quantized_gemm_wq_b200 import sweep
-        sweep.main()
+        sweep(args)
         return
     rank, world, local = dist_init(args.gpus)
     try:
