@@ -71,10 +71,13 @@ wq_status linear(const wq_bf16* x, int M, int K, int N, const float* cinv,
       (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
     return WQ_ERR_ALIGN;
   if (ws_bytes < wq_workspace_bytes(M, K, N, act_bits)) return WQ_ERR_ARG;
-  // workspace: codes | token scales | split-K partial tiles | split-K counters
+  // workspace: codes | token scales | split-K partial tiles | split-K counters.
+  // The codes are stored one per int8 byte for both widths: the tensor cores
+  // take int8 operands, so int4 activation codes in bytes feed the int8
+  // mainloop directly instead of being unpacked again for every weight tile.
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* qx = ws;
-  const size_t off_stok = round_up(act_bytes(M, K, act_bits));
+  const size_t off_stok = round_up(act_bytes(M, K, 8));
   float* s_tok = reinterpret_cast<float*>(ws + off_stok);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   wq::SplitScratch scratch{nullptr, nullptr};
@@ -91,11 +94,12 @@ wq_status linear(const wq_bf16* x, int M, int K, int N, const float* cinv,
   // the quantizer also clears the split-K accumulators and counters
   WQ_TRY(from_cuda(wq::launch_act_quant(x, M, K, cinv, stream_id, alpha, S, step, act_bits, qx,
                                         s_tok, st, splits > 1 ? ws + off_part : nullptr,
-                                        splits > 1 ? split_bytes : 0)));
+                                        splits > 1 ? split_bytes : 0, /*bytes_per_code=*/true)));
   const wq::EpilogueArgs ep{s_tok, stream_id, s_w, bias, beta, S, step};
   // weights may stream while the quantizer runs (it started the GEMM only after
   // everything before it in the stream had finished)
-  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, y, false,
+  // int8-stored codes: the int8-activation mainloop (the int32 sums are the same)
+  return from_cuda(wq::launch_gemm(qx, 8, qw, M, N, K, ep, y, false,
                                    splits > 1 ? &scratch : nullptr, st, /*w_prefetch=*/true));
 }
 
@@ -158,7 +162,8 @@ int wq_version(void) { return 100; }
 size_t wq_workspace_bytes(int M, int K, int N, int act_bits) {
   if ((act_bits != 8 && act_bits != 4) || check_mk(M, K) != WQ_OK || check_n(N) != WQ_OK)
     return 0;
-  return round_up(act_bytes(M, K, act_bits)) + round_up(sizeof(float) * static_cast<size_t>(M)) +
+  // codes one per byte for both widths (see linear())
+  return round_up(act_bytes(M, K, 8)) + round_up(sizeof(float) * static_cast<size_t>(M)) +
          wq::gemm_split_scratch_bytes(M, N, K);
 }
 

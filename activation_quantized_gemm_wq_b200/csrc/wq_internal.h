@@ -40,10 +40,13 @@ cudaError_t launch_pack_int4(const uint16_t* W, const float* c, int N, int K, ui
 
 // `zero` (16-byte aligned, zero_bytes a multiple of 16) is cleared by the same
 // launch: the fused linear uses it for the GEMM's split-K scratch.
+// bytes_per_code: int4 codes are written one per int8 byte ([M][K]) instead of
+// packed two per byte ([M][K/2]); int8 codes are always one per byte.
 cudaError_t launch_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                              const uint8_t* stream_id, const float* alpha, int S, int step,
                              int act_bits, void* qx, float* s_tok, cudaStream_t st,
-                             void* zero = nullptr, size_t zero_bytes = 0);
+                             void* zero = nullptr, size_t zero_bytes = 0,
+                             bool bytes_per_code = false);
 
 // Epilogue inputs of the fused GEMM.
 struct EpilogueArgs {

@@ -120,7 +120,9 @@ __device__ __forceinline__ void scale8(const uint4 raw, const float (&ci)[8], fl
 // chunks of 8 channels (128-bit loads, all issued before any use, so x is read
 // from HBM once with CPT loads in flight per thread), then forms x * cinv twice:
 // once for the row maximum and once for the codes, which keeps register use low.
-template <int ACT_BITS, int TPR, int CPT>
+// STORE_BITS: 8 writes one code per int8 byte (the int4 codes too, for the fused
+// linear's workspace), 4 packs two int4 codes per byte (low nibble = even k).
+template <int ACT_BITS, int STORE_BITS, int TPR, int CPT>
 __global__ void __launch_bounds__(256) act_quant_kernel(
     const uint16_t* __restrict__ x, int M, int K, const float* __restrict__ cinv,
     const uint8_t* __restrict__ stream_id, const float* __restrict__ alpha, int S, int step,
@@ -210,7 +212,7 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
 #pragma unroll
         for (int e = 0; e < 8; ++e) q[e] = static_cast<uint32_t>(quantize<QMAX>(v[e], s));
       }
-      if constexpr (ACT_BITS == 8) {
+      if constexpr (STORE_BITS == 8) {
         const uint2 o = make_uint2(pack_low_bytes(q[0], q[1], q[2], q[3]),
                                    pack_low_bytes(q[4], q[5], q[6], q[7]));
         reinterpret_cast<uint2*>(static_cast<int8_t*>(qx) + (size_t)row * K)[c] = o;
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
   }
 }
 
-template <int ACT_BITS, int TPR, int CPT>
+template <int ACT_BITS, int STORE_BITS, int TPR, int CPT>
 cudaError_t run_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                           const uint8_t* sid, const float* alpha, int S, int step, void* qx,
                           float* s_tok, uint4* zero, size_t zero_n16, cudaStream_t st) {
@@ -231,13 +233,13 @@ cudaError_t run_act_quant(const uint16_t* x, int M, int K, const float* cinv,
   static bool attr_set = false;  // per template instance
   static int per_sm = 0, per_sm_k = 0;  // resident CTAs per SM at K = per_sm_k
   if (!attr_set) {
-    if (cudaFuncSetAttribute(act_quant_kernel<ACT_BITS, TPR, CPT>,
+    if (cudaFuncSetAttribute(act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxK * 4) != cudaSuccess)
       return cudaGetLastError();
     attr_set = true;
   }
   if (per_sm_k != K) {
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, act_quant_kernel<ACT_BITS, TPR, CPT>,
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT>,
                                                   256, smem);
     if (per_sm < 1) per_sm = 1;
     per_sm_k = K;
@@ -247,18 +249,19 @@ cudaError_t run_act_quant(const uint16_t* x, int M, int K, const float* cinv,
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int groups = (M + RPC - 1) / RPC;
   const int grid = groups < per_sm * sms ? groups : per_sm * sms;
-  return launch_pdl(act_quant_kernel<ACT_BITS, TPR, CPT>, grid, 256, smem, st, x, M, K, cinv, sid,
+  return launch_pdl(act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT>, grid, 256, smem, st, x, M, K, cinv, sid,
                     alpha, S, step, qx, s_tok, zero, zero_n16);
 }
 
-template <int ACT_BITS>
+template <int ACT_BITS, int STORE_BITS>
 cudaError_t dispatch_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                                const uint8_t* sid, const float* alpha, int S, int step,
                                void* qx, float* s_tok, uint4* zero, size_t zero_n16,
                                cudaStream_t st) {
   const int nchunk = K / 8;
 #define WQ_AQ(TPR, CPT) \
-  return run_act_quant<ACT_BITS, TPR, CPT>(x, M, K, cinv, sid, alpha, S, step, qx, s_tok, zero, \
+  return run_act_quant<ACT_BITS, STORE_BITS, TPR, CPT>(x, M, K, cinv, sid, alpha, S, step, qx, \
+                                                       s_tok, zero, \
                                            zero_n16, st)
   // one warp per row up to K = 2048 (no block-level reduction), 8 chunks of 8
   // channels per thread beyond that
@@ -335,13 +338,17 @@ __global__ void channel_scale_kernel(const uint16_t* __restrict__ x_cal, int Mca
 cudaError_t launch_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                              const uint8_t* stream_id, const float* alpha, int S, int step,
                              int act_bits, void* qx, float* s_tok, cudaStream_t st,
-                             void* zero, size_t zero_bytes) {
+                             void* zero, size_t zero_bytes, bool bytes_per_code) {
   if (M == 0) return cudaSuccess;
   uint4* z = static_cast<uint4*>(zero);
   const size_t n16 = zero ? zero_bytes / 16 : 0;
   if (act_bits == 8)
-    return dispatch_act_quant<8>(x, M, K, cinv, stream_id, alpha, S, step, qx, s_tok, z, n16, st);
-  return dispatch_act_quant<4>(x, M, K, cinv, stream_id, alpha, S, step, qx, s_tok, z, n16, st);
+    return dispatch_act_quant<8, 8>(x, M, K, cinv, stream_id, alpha, S, step, qx, s_tok, z, n16,
+                                    st);
+  if (bytes_per_code)
+    return dispatch_act_quant<4, 8>(x, M, K, cinv, stream_id, alpha, S, step, qx, s_tok, z, n16,
+                                    st);
+  return dispatch_act_quant<4, 4>(x, M, K, cinv, stream_id, alpha, S, step, qx, s_tok, z, n16, st);
 }
 
 cudaError_t launch_pack_int4(const uint16_t* W, const float* c, int N, int K, uint8_t* qw,

@@ -80,8 +80,10 @@ int wq_version(void);
 
 /* Bytes of device workspace wq_linear_w4a8 / wq_linear_w4a4 need for M token
  * rows, K input channels, N output channels: the integer activation codes
- * (M*K bytes for A8, M*K/2 for A4) and the per-token scales (4*M bytes), each
- * rounded up to 256 bytes.  Returns 0 for invalid sizes. */
+ * (M*K bytes: one code per byte for both widths, since the tensor cores take
+ * int8 operands), the per-token scales (4*M bytes) and, for token counts too
+ * small to fill the GPU with output tiles, the split-K scratch, each rounded
+ * up to 256 bytes.  Returns 0 for invalid sizes (act_bits not 8 or 4 included). */
 size_t wq_workspace_bytes(int M, int K, int N, int act_bits);
 
 /* §4.2 (calibration side of the shared diagonal D): for each input channel k,
@@ -130,7 +132,8 @@ wq_status wq_linear_w4a8(const wq_bf16* x, int M, int K, int N, const float* cin
                          wq_stream_t stream);
 
 /* The fused W4A4 linear: as wq_linear_w4a8 with 4-bit activation codes
- * (workspace of wq_workspace_bytes(M, K, N, 4) bytes). */
+ * (qmax 7; workspace of wq_workspace_bytes(M, K, N, 4) bytes, in which the
+ * codes are kept one per byte, not packed as wq_act_quant writes them). */
 wq_status wq_linear_w4a4(const wq_bf16* x, int M, int K, int N, const float* cinv,
                          const uint8_t* stream_id, const float* alpha, const float* beta,
                          int S, int T, int step, const uint8_t* qw, const float* s_w,

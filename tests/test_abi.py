@@ -42,7 +42,8 @@ def test_status_strings_and_version(lib):
 
 def test_workspace_bytes(lib):
     assert wq.wq_workspace_bytes(4288, 2048, 6144, 8) == 4288 * 2048 + 17152
-    assert wq.wq_workspace_bytes(4288, 2048, 6144, 4) == 4288 * 1024 + 17152
+    # int4 codes are kept one per byte in the fused linear's workspace
+    assert wq.wq_workspace_bytes(4288, 2048, 6144, 4) == 4288 * 2048 + 17152
     assert wq.wq_workspace_bytes(1, 128, 16, 8) == 256 + 256
     assert wq.wq_workspace_bytes(64, 100, 256, 8) == 0      # K not a multiple of 128
     assert wq.wq_workspace_bytes(64, 256, 250, 8) == 0      # N not a multiple of 16
