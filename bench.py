@@ -61,6 +61,35 @@ def parse():
     return p.parse_args()
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_traffic_block2048_w4a8.md")
+GEMM_SOURCES = [os.path.join(ROOT, "activation_quantized_gemm_wq_b200", "csrc", f)
+                for f in ("wq_gemm.cuh", "wq_ptx.cuh", "wq_internal.h")]
+
+
+def gemm_traffic(workload):
+    """DRAM bytes per GEMM launch from the committed ncu capture of this workload, or
+    None when there is none or the GEMM sources changed since it was taken."""
+    import hashlib
+    if workload != "block2048_w4a8":
+        return None
+    try:
+        fields = {}
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                if ":" in line and line.startswith("    "):
+                    k, v = line.strip().split(":", 1)
+                    fields[k.strip()] = v.strip()
+        h = hashlib.sha256()
+        for path in GEMM_SOURCES:
+            with open(path, "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != fields.get("source_sha256"):
+            return None
+        return int(fields["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def peaks():
     try:
         with open(PEAKS_FILE) as f:
@@ -354,7 +383,8 @@ def run_gpu(args, rank, world, local):
             "peak": round(peak, 1),
             "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
-            "traffic": None,
+            "traffic": gemm_traffic(wl.name),
+            "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
             "peak_source": f"{src} bf16 burst {bf16_burst} TFLOP/s x{INT8_PER_BF16} (dense int8 "
                            "/ bf16 nominal ratio); units are int8 tera-ops",
             "gemm_avg_launch_ms": round(gemm_avg_ms, 5),

@@ -52,3 +52,20 @@ def test_single_process_needs_no_process_group():
         os.environ.pop(k, None)
     assert bench.dist_init(1) == (0, 1, 0)
     assert bench.max_over_ranks(3.5, 1) == 3.5
+
+
+def test_gemm_traffic_tracks_the_kernel_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed ncu capture only while the GEMM sources
+    hash to the value recorded beside it."""
+    import hashlib
+    src = tmp_path / "k.cuh"
+    src.write_bytes(b"kernel v1")
+    prof = tmp_path / "traffic.md"
+    digest = hashlib.sha256(b"kernel v1").hexdigest()
+    prof.write_text(f"# t\n\n    traffic_bytes_per_launch: 1234\n    source_sha256: {digest}\n")
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(prof))
+    monkeypatch.setattr(bench, "GEMM_SOURCES", [str(src)])
+    assert bench.gemm_traffic("block2048_w4a8") == 1234
+    assert bench.gemm_traffic("block4096_w4a8_t10") is None   # no capture for that workload
+    src.write_bytes(b"kernel v2")                              # the kernel changed since
+    assert bench.gemm_traffic("block2048_w4a8") is None
