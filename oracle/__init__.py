@@ -36,6 +36,8 @@ def _bind(lib):
     lib.oracle_channel_scale.argtypes = [_P, _I, _P, _I, _I, _P, _P]
     lib.oracle_pack_int4.argtypes = [_P, _P, _I, _I, _P, _P]
     lib.oracle_act_quant.argtypes = [_P, _I, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P]
+    lib.oracle_act_quant_static.argtypes = [_P, _I, _I, _P, _P, _P, _P, _I, _I, _I, _I, _P,
+                                            _P]
     lib.oracle_gemm_s32.argtypes = [_P, _I, _P, _I, _I, _I, _P]
     lib.oracle_epilogue.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
     lib.oracle_linear.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P,
@@ -45,7 +47,7 @@ def _bind(lib):
     lib.oracle_double_to_bf16.argtypes = [ctypes.c_double]
     lib.oracle_double_to_bf16.restype = ctypes.c_uint16
     for f in ("oracle_channel_scale", "oracle_pack_int4", "oracle_act_quant",
-              "oracle_gemm_s32", "oracle_epilogue", "oracle_linear"):
+              "oracle_act_quant_static", "oracle_gemm_s32", "oracle_epilogue", "oracle_linear"):
         getattr(lib, f).restype = _I
     return lib
 
@@ -106,6 +108,37 @@ class Oracle:
                                          S, T, step, act_bits, _ptr(qx), _ptr(s_tok)),
                "act_quant")
         return qx, s_tok
+
+    def act_quant_static(self, x, cinv, stream_id, thr, gain, step, act_bits):
+        """Static clipping (shared threshold thr [T], stream gains gain [T][S])."""
+        x = _c(x, np.uint16)
+        cinv = _c(cinv, np.float32)
+        stream_id = _c(stream_id, np.uint8)
+        thr = _c(thr, np.float32)
+        gain = _c(gain, np.float32)
+        T, S = gain.shape
+        M, K = x.shape
+        qx = np.empty((M, K) if act_bits == 8 else (M, K // 2),
+                      np.int8 if act_bits == 8 else np.uint8)
+        s_tok = np.empty(M, np.float32)
+        _check(self.lib.oracle_act_quant_static(_ptr(x), M, K, _ptr(cinv), _ptr(stream_id),
+                                                _ptr(thr), _ptr(gain), S, T, step, act_bits,
+                                                _ptr(qx), _ptr(s_tok)), "act_quant_static")
+        return qx, s_tok
+
+    def linear_static(self, x, cinv, stream_id, thr, gain, beta, step, act_bits, qw, s_w, bias):
+        """The fused linear with static clipping, as the three steps in order:
+        act_quant_static, gemm_s32, epilogue.  Returns (y bf16 bits, qx, s_tok, acc)."""
+        qx, s_tok = self.act_quant_static(x, cinv, stream_id, thr, gain, step, act_bits)
+        acc = self.gemm_s32(qx, act_bits, qw, np.asarray(x).shape[1])
+        if beta is None:  # the epilogue's table shape comes from the gains
+            y = self.epilogue(acc, s_tok, s_w, bias,
+                              np.zeros((np.asarray(gain).shape[0], np.asarray(gain).shape[1],
+                                        np.asarray(qw).shape[0]), np.float32),
+                              stream_id, step)
+        else:
+            y = self.epilogue(acc, s_tok, s_w, bias, beta, stream_id, step)
+        return y, qx, s_tok, acc
 
     def gemm_s32(self, qx, act_bits, qw, K):
         qx = np.ascontiguousarray(qx)

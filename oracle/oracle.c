@@ -178,6 +178,48 @@ int oracle_act_quant(const uint16_t* x, int M, int K, const float* cinv,
   return 0;
 }
 
+/* §4.3 read as static clipping (the layer-step table holds one shared clip
+ * threshold per step and a bounded gain per stream): the token's stream gain g
+ * narrows the threshold thr to clip = thr / g, the scale is clip / qmax, and the
+ * code is the nearest integer to x'/s clamped to +-qmax; the inverse gain stays
+ * inside the scale that the epilogue multiplies back (§4.4).  No row maximum is
+ * involved.  thr [T]; gain [T][S]. */
+int oracle_act_quant_static(const uint16_t* x, int M, int K, const float* cinv,
+                            const uint8_t* stream_id, const float* thr, const float* gain,
+                            int S, int T, int step, int act_bits, void* qx, float* s_tok) {
+  if (!x || !stream_id || !thr || !gain || !qx || !s_tok) return ORACLE_EBADARG;
+  if (M < 0 || K < 2 || (K % 2) != 0 || S < 1 || T < 1 || step < 0 || step >= T)
+    return ORACLE_EBADARG;
+  if (act_bits != 8 && act_bits != 4) return ORACLE_EBADARG;
+  const float qmax = act_bits == 8 ? 127.0f : 7.0f;
+  float* xp = (float*)malloc(sizeof(float) * (size_t)K);
+  if (!xp) return ORACLE_ENOMEM;
+  for (int m = 0; m < M; ++m) {
+    int sid = stream_id[m];
+    if (sid >= S) { free(xp); return ORACLE_EBADARG; }
+    for (int k = 0; k < K; ++k) {
+      float ck = cinv ? cinv[k] : 1.0f;
+      xp[k] = ck * oracle_bf16_to_float(x[(size_t)m * K + k]);
+      if (!isfinite(xp[k])) { free(xp); return ORACLE_ENONFINITE; }
+    }
+    float g = gain[(size_t)step * S + sid];
+    float clip = g > 0.0f ? thr[step] / g : 0.0f;
+    float s = clip / qmax;
+    s_tok[m] = s;
+    if (act_bits == 8) {
+      int8_t* row = (int8_t*)qx + (size_t)m * K;
+      for (int k = 0; k < K; ++k) row[k] = (int8_t)quantize_value(xp[k], s, qmax);
+    } else {
+      uint8_t* row = (uint8_t*)qx + (size_t)m * (K / 2);
+      for (int k = 0; k < K; k += 2)
+        row[k / 2] = pack_pair(quantize_value(xp[k], s, qmax),
+                               quantize_value(xp[k + 1], s, qmax));
+    }
+  }
+  free(xp);
+  return 0;
+}
+
 static int act_code(const void* qx, int act_bits, int K, int m, int k) {
   if (act_bits == 8) return ((const int8_t*)qx)[(size_t)m * K + k];
   uint8_t b = ((const uint8_t*)qx)[(size_t)m * (K / 2) + k / 2];

@@ -58,6 +58,14 @@ int oracle_channel_scale(const uint16_t* x_cal, int Mcal, const uint16_t* W, int
 int oracle_pack_int4(const uint16_t* W, const float* c, int N, int K, uint8_t* qw,
                      float* s_w);
 
+/* §4.3 read as static clipping: one shared clip threshold thr[step] per layer
+ * step and a bounded gain per stream, gain [T][S]; clip = thr[step] / gain (0 when
+ * the gain is not positive), s = clip / qmax, codes as in oracle_act_quant.
+ * Same layouts as oracle_act_quant. */
+int oracle_act_quant_static(const uint16_t* x, int M, int K, const float* cinv,
+                            const uint8_t* stream_id, const float* thr, const float* gain,
+                            int S, int T, int step, int act_bits, void* qx, float* s_tok);
+
 /* §4.4 first kernel (with §4.3 and §4.2 folded in): per-token quantization.
  * x [M][K] bf16; cinv [K] or NULL (=1); stream_id [M]; alpha [T][S] clip ratios;
  * act_bits 8 -> qx int8 [M][K]; act_bits 4 -> qx packed uint8 [M][K/2].

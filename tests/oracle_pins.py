@@ -18,6 +18,9 @@ What pins what:
                     the output equals the fp64 product of the dequantized operands
   requant           re-quantizing dequantized codes returns the same codes
   scale_invariance  doubling a row doubles its scale and keeps its codes
+  static_vs_dynamic static clipping with gain 1 and threshold alpha*amax of the row
+                    gives exactly the dynamic codes and scale (the dynamic path is
+                    pinned by the checks above)
 """
 import numpy as np
 
@@ -80,6 +83,27 @@ def golden_act_quant(orc, golden):
             fails.append(f"act_quant/{case['name']}: packed {qx.tolist()} != {case['packed']}")
         if not np.array_equal(f32_bits(s), f32_bits(case["s_tok"])):
             fails.append(f"act_quant/{case['name']}: s_tok {s.tolist()} != {case['s_tok']}")
+    return fails
+
+
+def golden_act_quant_static(orc, golden):
+    fails = []
+    for case in golden["act_quant_static"]:
+        x = bf16_from_values(case["x"])
+        cinv = None if case["cinv"] is None else np.asarray(case["cinv"], np.float32)
+        qx, s = orc.act_quant_static(x, cinv, np.asarray(case["stream_id"], np.uint8),
+                                     np.asarray(case["thr"], np.float32),
+                                     np.asarray(case["gain"], np.float32), case["step"],
+                                     case["act_bits"])
+        codes = unpack_nibbles(qx) if case["act_bits"] == 4 else qx.astype(np.int16)
+        if not np.array_equal(codes, np.asarray(case["codes"])):
+            fails.append(f"act_quant_static/{case['name']}: codes {codes.tolist()} != "
+                         f"{case['codes']}")
+        if "packed" in case and not np.array_equal(qx, np.asarray(case["packed"], np.uint8)):
+            fails.append(f"act_quant_static/{case['name']}: packed {qx.tolist()}")
+        if not np.array_equal(f32_bits(s), f32_bits(case["s_tok"])):
+            fails.append(f"act_quant_static/{case['name']}: s_tok {s.tolist()} != "
+                         f"{case['s_tok']}")
     return fails
 
 
@@ -356,10 +380,35 @@ def near_ties(orc, seeds=(11, 12)):
     return fails
 
 
+def static_vs_dynamic(orc, seeds=(13,)):
+    """One row at a time: threshold = alpha * amax of the row (binary32 product of the
+    row's exact maximum), gain 1, so clip, scale and codes must equal the dynamic
+    path's bit for bit."""
+    fails = []
+    for seed in seeds:
+        x, cinv, sid, alpha, _, _, _, _ = _tiny_inputs(seed, M=12)
+        step = 1
+        xp = bf16_to_f32(x) * cinv[None, :]
+        for bits in (8, 4):
+            qd, sd = orc.act_quant(x, cinv, sid, alpha, step, bits)
+            for m in range(x.shape[0]):
+                amax = np.float32(np.abs(xp[m]).max())
+                thr = np.zeros(alpha.shape[0], np.float32)
+                thr[step] = np.float32(alpha[step, sid[m]]) * amax
+                gain = np.ones_like(alpha)
+                qs, ss = orc.act_quant_static(x[m:m + 1], cinv, sid[m:m + 1], thr, gain, step,
+                                              bits)
+                if not (np.array_equal(qs[0], qd[m]) and f32_bits(ss[0]) == f32_bits(sd[m])):
+                    fails.append(f"static_vs_dynamic seed {seed} bits {bits} row {m}")
+                    break
+    return fails
+
+
 ALL_CHECKS = (golden_act_quant, golden_pack, golden_channel_scale, golden_linear,
-              golden_bf16_rounding, brute_codes, gemm_vs_matmul, epilogue_fp64, textbook,
-              on_grid, requant, scale_invariance, near_ties)
-GOLDEN_CHECKS = ALL_CHECKS[:5]
+              golden_bf16_rounding, golden_act_quant_static, brute_codes, gemm_vs_matmul,
+              epilogue_fp64, textbook, on_grid, requant, scale_invariance, near_ties,
+              static_vs_dynamic)
+GOLDEN_CHECKS = ALL_CHECKS[:6]
 
 
 def all_failures(orc, golden):

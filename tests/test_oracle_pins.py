@@ -64,6 +64,17 @@ MUTANTS = [
      [("double r = nearbyint(ldexp(a, 8 - e));", "double r = round(ldexp(a, 8 - e));")]),
     ("channel scale inverted", [("if (a > 0.0f && b > 0.0f) ck = sqrtf(a / b);",
                                  "if (a > 0.0f && b > 0.0f) ck = sqrtf(b / a);")]),
+    ("static path: channel scale not folded into activations",
+     [("xp[k] = ck * oracle_bf16_to_float(x[(size_t)m * K + k]);",
+       "xp[k] = oracle_bf16_to_float(x[(size_t)m * K + k]);")]),
+    ("static clip multiplies by the gain",
+     [("float clip = g > 0.0f ? thr[step] / g : 0.0f;",
+       "float clip = g > 0.0f ? thr[step] * g : 0.0f;")]),
+    ("static gain table indexed [stream][step]",
+     [("float g = gain[(size_t)step * S + sid];", "float g = gain[(size_t)sid * T + step];")]),
+    ("static threshold of step 0 for every step",
+     [("float clip = g > 0.0f ? thr[step] / g : 0.0f;",
+       "float clip = g > 0.0f ? thr[0] / g : 0.0f;")]),
 ]
 
 
