@@ -37,6 +37,9 @@ _SIGS = {
                             ctypes.c_size_t, _P]),
     "wq_linear_w4a8_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P,
                                     _P]),
+    "wq_act_quant_static": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
+    "wq_linear_w4ax_static": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P,
+                                   _P, _P, _P, ctypes.c_size_t, _P]),
     "wq_debug_gemm_s32": (_I, [_P, _I, _P, _I, _I, _I, _P, _P]),
     "wq_device_status": (_I, [ctypes.POINTER(ctypes.c_uint)]),
 }
@@ -115,6 +118,23 @@ def wq_act_quant(x, cinv, stream_id, alpha, step, act_bits, qx, s_tok, stream=No
     T, S = alpha.shape
     _call("wq_act_quant", _ptr(x), M, K, _ptr(cinv), _ptr(stream_id), _ptr(alpha), S, T, step,
           act_bits, _ptr(qx), _ptr(s_tok), _stream(stream))
+
+
+def wq_act_quant_static(x, cinv, stream_id, thr, gain, step, act_bits, qx, s_tok, stream=None):
+    M, K = x.shape
+    T, S = gain.shape
+    _call("wq_act_quant_static", _ptr(x), M, K, _ptr(cinv), _ptr(stream_id), _ptr(thr),
+          _ptr(gain), S, T, step, act_bits, _ptr(qx), _ptr(s_tok), _stream(stream))
+
+
+def wq_linear_w4ax_static(x, cinv, stream_id, thr, gain, beta, step, act_bits, qw, s_w, bias, y,
+                          workspace, stream=None):
+    M, K = x.shape
+    N = qw.shape[0]
+    T, S = gain.shape
+    _call("wq_linear_w4ax_static", _ptr(x), M, K, N, _ptr(cinv), _ptr(stream_id), _ptr(thr),
+          _ptr(gain), _ptr(beta), S, T, step, act_bits, _ptr(qw), _ptr(s_w), _ptr(bias), _ptr(y),
+          _ptr(workspace), _nbytes(workspace), _stream(stream))
 
 
 def wq_gemm_w4ax(qx, s_tok, act_bits, K, stream_id, beta, S, T, step, qw, s_w, bias, y,

@@ -57,10 +57,14 @@ wq_status gemm_checks(const void* qx, const float* s_tok, int act_bits, int M, i
   return WQ_OK;
 }
 
+// alpha: the clip ratios [T][S] (dynamic clipping), or, when thr is not NULL, the
+// stream gains [T][S] of static clipping with thresholds thr [T].
 wq_status linear(const wq_bf16* x, int M, int K, int N, const float* cinv,
                  const uint8_t* stream_id, const float* alpha, const float* beta, int S, int T,
                  int step, const uint8_t* qw, const float* s_w, const float* bias, wq_bf16* y,
-                 void* workspace, size_t ws_bytes, wq_stream_t stream, int act_bits) {
+                 void* workspace, size_t ws_bytes, wq_stream_t stream, int act_bits,
+                 const float* thr = nullptr) {
+  if (act_bits != 8 && act_bits != 4) return WQ_ERR_ARG;
   WQ_TRY(check_mk(M, K));
   WQ_TRY(check_n(N));
   WQ_TRY(check_table(S, T, step));
@@ -92,9 +96,15 @@ wq_status linear(const wq_bf16* x, int M, int K, int N, const float* cinv,
     scratch.counters = reinterpret_cast<int*>(ws + off_part + part_bytes);
   }
   // the quantizer also clears the split-K accumulators and counters
-  WQ_TRY(from_cuda(wq::launch_act_quant(x, M, K, cinv, stream_id, alpha, S, step, act_bits, qx,
-                                        s_tok, st, splits > 1 ? ws + off_part : nullptr,
-                                        splits > 1 ? split_bytes : 0, /*bytes_per_code=*/true)));
+  void* zero = splits > 1 ? ws + off_part : nullptr;
+  const size_t zero_bytes = splits > 1 ? split_bytes : 0;
+  if (thr)
+    WQ_TRY(from_cuda(wq::launch_act_quant_static(x, M, K, cinv, stream_id, thr, alpha, S, step,
+                                                 act_bits, qx, s_tok, st, zero, zero_bytes,
+                                                 /*bytes_per_code=*/true)));
+  else
+    WQ_TRY(from_cuda(wq::launch_act_quant(x, M, K, cinv, stream_id, alpha, S, step, act_bits, qx,
+                                          s_tok, st, zero, zero_bytes, /*bytes_per_code=*/true)));
   const wq::EpilogueArgs ep{s_tok, stream_id, s_w, bias, beta, S, step};
   // weights may stream while the quantizer runs (it started the GEMM only after
   // everything before it in the stream had finished)
@@ -196,6 +206,32 @@ wq_status wq_act_quant(const wq_bf16* x, int M, int K, const float* cinv,
   if (!aligned16(x) || !aligned16(qx) || (cinv && !aligned16(cinv))) return WQ_ERR_ALIGN;
   return from_cuda(wq::launch_act_quant(x, M, K, cinv, stream_id, alpha, S, step, act_bits, qx,
                                         s_tok, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_act_quant_static(const wq_bf16* x, int M, int K, const float* cinv,
+                              const uint8_t* stream_id, const float* thr, const float* gain,
+                              int S, int T, int step, int act_bits, void* qx, float* s_tok,
+                              wq_stream_t stream) {
+  if (act_bits != 8 && act_bits != 4) return WQ_ERR_ARG;
+  WQ_TRY(check_mk(M, K));
+  WQ_TRY(check_table(S, T, step));
+  if (M == 0) return WQ_OK;
+  if (!x || !stream_id || !thr || !gain || !qx || !s_tok) return WQ_ERR_NULL;
+  if (!aligned16(x) || !aligned16(qx) || (cinv && !aligned16(cinv))) return WQ_ERR_ALIGN;
+  return from_cuda(wq::launch_act_quant_static(x, M, K, cinv, stream_id, thr, gain, S, step,
+                                               act_bits, qx, s_tok,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_linear_w4ax_static(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                                const uint8_t* stream_id, const float* thr, const float* gain,
+                                const float* beta, int S, int T, int step, int act_bits,
+                                const uint8_t* qw, const float* s_w, const float* bias,
+                                wq_bf16* y, void* workspace, size_t ws_bytes,
+                                wq_stream_t stream) {
+  if (M > 0 && !thr) return WQ_ERR_NULL;
+  return linear(x, M, K, N, cinv, stream_id, gain, beta, S, T, step, qw, s_w, bias, y,
+                workspace, ws_bytes, stream, act_bits, thr);
 }
 
 wq_status wq_gemm_w4ax(const void* qx, const float* s_tok, int act_bits, int M, int K, int N,

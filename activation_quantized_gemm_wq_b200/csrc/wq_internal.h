@@ -48,6 +48,14 @@ cudaError_t launch_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                              void* zero = nullptr, size_t zero_bytes = 0,
                              bool bytes_per_code = false);
 
+// The same quantizer with static clipping: clip = thr[step] / gain[step][stream]
+// (0 when the gain is not positive) instead of alpha * (row maximum).
+cudaError_t launch_act_quant_static(const uint16_t* x, int M, int K, const float* cinv,
+                                    const uint8_t* stream_id, const float* thr,
+                                    const float* gain, int S, int step, int act_bits, void* qx,
+                                    float* s_tok, cudaStream_t st, void* zero = nullptr,
+                                    size_t zero_bytes = 0, bool bytes_per_code = false);
+
 // Epilogue inputs of the fused GEMM.
 struct EpilogueArgs {
   const float* s_tok;        // [M]

@@ -122,11 +122,15 @@ __device__ __forceinline__ void scale8(const uint4 raw, const float (&ci)[8], fl
 // once for the row maximum and once for the codes, which keeps register use low.
 // STORE_BITS: 8 writes one code per int8 byte (the int4 codes too, for the fused
 // linear's workspace), 4 packs two int4 codes per byte (low nibble = even k).
-template <int ACT_BITS, int STORE_BITS, int TPR, int CPT>
+// STATIC: the clip comes from the layer-step table alone (§4.3 read as a shared
+// threshold thr[step] narrowed by the stream gain, clip = thr / gain, with `alpha`
+// holding the gains [T][S]); no row maximum, so x is scaled and quantized once.
+template <int ACT_BITS, int STORE_BITS, int TPR, int CPT, bool STATIC>
 __global__ void __launch_bounds__(256) act_quant_kernel(
     const uint16_t* __restrict__ x, int M, int K, const float* __restrict__ cinv,
-    const uint8_t* __restrict__ stream_id, const float* __restrict__ alpha, int S, int step,
-    void* __restrict__ qx, float* __restrict__ s_tok, uint4* __restrict__ zero, size_t zero_n16) {
+    const uint8_t* __restrict__ stream_id, const float* __restrict__ alpha,
+    const float* __restrict__ thr, int S, int step, void* __restrict__ qx,
+    float* __restrict__ s_tok, uint4* __restrict__ zero, size_t zero_n16) {
   constexpr int RPC = 256 / TPR;  // rows per CTA pass
   constexpr int WPR = TPR / 32;   // warps per row
   constexpr int QMAX = ACT_BITS == 8 ? 127 : 7;
@@ -165,31 +169,39 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
                    : make_uint4(0u, 0u, 0u, 0u);
     }
     float amax = 0.0f;
+    if constexpr (!STATIC) {
 #pragma unroll
-    for (int i = 0; i < CPT; ++i) {
-      const int c = t + i * TPR;
-      if (c < nchunk) {
-        float ci[8], v[8];
-        load_cinv8(cinv_s, c, ci);
-        scale8(raw[i], ci, v);
+      for (int i = 0; i < CPT; ++i) {
+        const int c = t + i * TPR;
+        if (c < nchunk) {
+          float ci[8], v[8];
+          load_cinv8(cinv_s, c, ci);
+          scale8(raw[i], ci, v);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+          for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+        }
       }
-    }
-    amax = warp_max(amax);
-    if constexpr (WPR > 1) {
-      if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
-      __syncthreads();
+      amax = warp_max(amax);
+      if constexpr (WPR > 1) {
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+        __syncthreads();
 #pragma unroll
-      for (int j = 0; j < WPR; ++j) amax = fmaxf(amax, red[local_row * WPR + j]);
-      __syncthreads();  // red is rewritten by the next pass
+        for (int j = 0; j < WPR; ++j) amax = fmaxf(amax, red[local_row * WPR + j]);
+        __syncthreads();  // red is rewritten by the next pass
+      }
     }
     if (!row_ok) continue;
 
     float s = 0.0f;
     const int sid = stream_id[row];
     if (sid < S) {
-      const float clip = __fmul_rn(__ldg(alpha + step * S + sid), amax);
+      float clip;
+      if constexpr (STATIC) {
+        const float g = __ldg(alpha + step * S + sid);
+        clip = g > 0.0f ? __fdiv_rn(__ldg(thr + step), g) : 0.0f;
+      } else {
+        clip = __fmul_rn(__ldg(alpha + step * S + sid), amax);
+      }
       s = __fdiv_rn(clip, static_cast<float>(QMAX));
     } else if (t == 0) {
       raise_error(kErrBadStreamId);
@@ -224,22 +236,23 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
   }
 }
 
-template <int ACT_BITS, int STORE_BITS, int TPR, int CPT>
+template <int ACT_BITS, int STORE_BITS, int TPR, int CPT, bool STATIC>
 cudaError_t run_act_quant(const uint16_t* x, int M, int K, const float* cinv,
-                          const uint8_t* sid, const float* alpha, int S, int step, void* qx,
-                          float* s_tok, uint4* zero, size_t zero_n16, cudaStream_t st) {
+                          const uint8_t* sid, const float* alpha, const float* thr, int S,
+                          int step, void* qx, float* s_tok, uint4* zero, size_t zero_n16,
+                          cudaStream_t st) {
   constexpr int RPC = 256 / TPR;
   const size_t smem = static_cast<size_t>(K) * sizeof(float);  // cinv copy
   static bool attr_set = false;  // per template instance
   static int per_sm = 0, per_sm_k = 0;  // resident CTAs per SM at K = per_sm_k
   if (!attr_set) {
-    if (cudaFuncSetAttribute(act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT>,
+    if (cudaFuncSetAttribute(act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT, STATIC>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxK * 4) != cudaSuccess)
       return cudaGetLastError();
     attr_set = true;
   }
   if (per_sm_k != K) {
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT>,
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT, STATIC>,
                                                   256, smem);
     if (per_sm < 1) per_sm = 1;
     per_sm_k = K;
@@ -249,20 +262,19 @@ cudaError_t run_act_quant(const uint16_t* x, int M, int K, const float* cinv,
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int groups = (M + RPC - 1) / RPC;
   const int grid = groups < per_sm * sms ? groups : per_sm * sms;
-  return launch_pdl(act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT>, grid, 256, smem, st, x, M, K, cinv, sid,
-                    alpha, S, step, qx, s_tok, zero, zero_n16);
+  return launch_pdl(act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT, STATIC>, grid, 256, smem, st, x, M, K, cinv, sid,
+                    alpha, thr, S, step, qx, s_tok, zero, zero_n16);
 }
 
-template <int ACT_BITS, int STORE_BITS>
+template <int ACT_BITS, int STORE_BITS, bool STATIC>
 cudaError_t dispatch_act_quant(const uint16_t* x, int M, int K, const float* cinv,
-                               const uint8_t* sid, const float* alpha, int S, int step,
-                               void* qx, float* s_tok, uint4* zero, size_t zero_n16,
+                               const uint8_t* sid, const float* alpha, const float* thr, int S,
+                               int step, void* qx, float* s_tok, uint4* zero, size_t zero_n16,
                                cudaStream_t st) {
   const int nchunk = K / 8;
 #define WQ_AQ(TPR, CPT) \
-  return run_act_quant<ACT_BITS, STORE_BITS, TPR, CPT>(x, M, K, cinv, sid, alpha, S, step, qx, \
-                                                       s_tok, zero, \
-                                           zero_n16, st)
+  return run_act_quant<ACT_BITS, STORE_BITS, TPR, CPT, STATIC>(x, M, K, cinv, sid, alpha, thr, S, \
+                                                               step, qx, s_tok, zero, zero_n16, st)
   // one warp per row up to K = 2048 (no block-level reduction), 8 chunks of 8
   // channels per thread beyond that
   if (nchunk <= 32) WQ_AQ(32, 1);
@@ -335,20 +347,40 @@ __global__ void channel_scale_kernel(const uint16_t* __restrict__ x_cal, int Mca
 
 }  // namespace
 
-cudaError_t launch_act_quant(const uint16_t* x, int M, int K, const float* cinv,
-                             const uint8_t* stream_id, const float* alpha, int S, int step,
-                             int act_bits, void* qx, float* s_tok, cudaStream_t st,
-                             void* zero, size_t zero_bytes, bool bytes_per_code) {
+template <bool STATIC>
+cudaError_t launch_act_quant_mode(const uint16_t* x, int M, int K, const float* cinv,
+                                  const uint8_t* sid, const float* table, const float* thr,
+                                  int S, int step, int act_bits, void* qx, float* s_tok,
+                                  cudaStream_t st, void* zero, size_t zero_bytes,
+                                  bool bytes_per_code) {
   if (M == 0) return cudaSuccess;
   uint4* z = static_cast<uint4*>(zero);
   const size_t n16 = zero ? zero_bytes / 16 : 0;
   if (act_bits == 8)
-    return dispatch_act_quant<8, 8>(x, M, K, cinv, stream_id, alpha, S, step, qx, s_tok, z, n16,
-                                    st);
+    return dispatch_act_quant<8, 8, STATIC>(x, M, K, cinv, sid, table, thr, S, step, qx, s_tok, z,
+                                            n16, st);
   if (bytes_per_code)
-    return dispatch_act_quant<4, 8>(x, M, K, cinv, stream_id, alpha, S, step, qx, s_tok, z, n16,
-                                    st);
-  return dispatch_act_quant<4, 4>(x, M, K, cinv, stream_id, alpha, S, step, qx, s_tok, z, n16, st);
+    return dispatch_act_quant<4, 8, STATIC>(x, M, K, cinv, sid, table, thr, S, step, qx, s_tok, z,
+                                            n16, st);
+  return dispatch_act_quant<4, 4, STATIC>(x, M, K, cinv, sid, table, thr, S, step, qx, s_tok, z,
+                                          n16, st);
+}
+
+cudaError_t launch_act_quant(const uint16_t* x, int M, int K, const float* cinv,
+                             const uint8_t* stream_id, const float* alpha, int S, int step,
+                             int act_bits, void* qx, float* s_tok, cudaStream_t st,
+                             void* zero, size_t zero_bytes, bool bytes_per_code) {
+  return launch_act_quant_mode<false>(x, M, K, cinv, stream_id, alpha, nullptr, S, step, act_bits,
+                                      qx, s_tok, st, zero, zero_bytes, bytes_per_code);
+}
+
+cudaError_t launch_act_quant_static(const uint16_t* x, int M, int K, const float* cinv,
+                                    const uint8_t* stream_id, const float* thr,
+                                    const float* gain, int S, int step, int act_bits, void* qx,
+                                    float* s_tok, cudaStream_t st, void* zero, size_t zero_bytes,
+                                    bool bytes_per_code) {
+  return launch_act_quant_mode<true>(x, M, K, cinv, stream_id, gain, thr, S, step, act_bits, qx,
+                                     s_tok, st, zero, zero_bytes, bytes_per_code);
 }
 
 cudaError_t launch_pack_int4(const uint16_t* W, const float* c, int N, int K, uint8_t* qw,

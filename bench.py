@@ -66,7 +66,7 @@ def parse():
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_traffic_block2048_w4a8.md")
 GEMM_SOURCES = [os.path.join(ROOT, "activation_quantized_gemm_wq_b200", "csrc", f)
-                for f in ("wq_gemm.cuh", "wq_ptx.cuh", "wq_internal.h")]
+                for f in ("wq_gemm.cuh", "wq_ptx.cuh")]
 
 
 def gemm_traffic(workload):
@@ -646,6 +646,9 @@ def sweep(args):
     entries += [("2 block2048 A4 T10", S.BLOCK2048_A4, [0, 1, 2, 3])]
     entries += [("3 block4096 A8 T10", S.BLOCK4096_A8, [0, 1, 2, 3])]
     entries += [("3 block4096 A4 T10", S.BLOCK4096_A4, [0, 1, 2, 3])]
+    # static clipping (one threshold per step, one gain per stream): no row maximum
+    entries += [("5 static block2048 A8", S.BLOCK2048_A8, [0, 1, 2, 3])]
+    entries += [("5 static block4096 A8 T10", S.BLOCK4096_A8, [0, 1, 2, 3])]
     for parent in (S.BLOCK2048_A8, S.BLOCK4096_A8):
         for li in range(4):  # weights outermost: generated once per shape
             for bits in (8, 4):
@@ -694,6 +697,15 @@ def sweep(args):
             ws = wq.alloc_workspace(M, K, N, bits)
             lin_fn = wq.wq_linear_w4a8 if bits == 8 else wq.wq_linear_w4a4
             step = T - 1
+            if "static" in label:  # threshold: a typical row maximum; gains around 1
+                xp = (S.activations(wl, li, 0).astype(np.uint32) << 16).view(np.float32)
+                thr = dev(np.full(T, np.median(np.abs(xp).max(axis=1)), np.float32))
+                gain = dev(np.resize(L.alpha, (T, 3)).astype(np.float32))
+
+                def lin_fn(x_, cinv_, sid_, alpha_, beta_, step_, qw_, s_w_, bias_, y_, ws_,
+                           thr=thr, gain=gain, bits=bits):
+                    wq.wq_linear_w4ax_static(x_, cinv_, sid_, thr, gain, beta_, step_, bits, qw_,
+                                             s_w_, bias_, y_, ws_)
             for r in range(ncopy):
                 wq.wq_act_quant(xs[r], cinv, sid, alpha, step, bits, qxs[r], s_tok)
             calls = max(10, ncopy)

@@ -140,6 +140,30 @@ wq_status wq_linear_w4a4(const wq_bf16* x, int M, int K, int N, const float* cin
                          const float* bias, wq_bf16* y, void* workspace, size_t ws_bytes,
                          wq_stream_t stream);
 
+/* §4.3, static reading of the layer-step table: one shared clip threshold per
+ * step, thr [T] fp32, narrowed per stream by a bounded gain, gain [T][S] fp32:
+ * clip = thr[step] / gain[step][stream_id[m]] (IEEE division; 0 when the gain is
+ * not positive), s_tok[m] = clip / qmax, and the codes as in wq_act_quant (round
+ * half to even, clamp to +-qmax).  The inverse gain stays inside s_tok, which the
+ * GEMM's epilogue multiplies back (§4.4).  No row maximum is taken, so x is read
+ * and quantized in one pass.  Layouts, preconditions and errors as wq_act_quant;
+ * thr and gain must not be NULL. */
+wq_status wq_act_quant_static(const wq_bf16* x, int M, int K, const float* cinv,
+                              const uint8_t* stream_id, const float* thr, const float* gain,
+                              int S, int T, int step, int act_bits, void* qx, float* s_tok,
+                              wq_stream_t stream);
+
+/* The fused W4A8 (act_bits 8) or W4A4 (act_bits 4) linear with static clipping:
+ * wq_act_quant_static then the GEMM and epilogue, with the workspace of
+ * wq_workspace_bytes(M, K, N, act_bits) bytes (codes one per byte, as in
+ * wq_linear_w4a8 / wq_linear_w4a4).  Other arguments as wq_linear_w4a8. */
+wq_status wq_linear_w4ax_static(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                                const uint8_t* stream_id, const float* thr, const float* gain,
+                                const float* beta, int S, int T, int step, int act_bits,
+                                const uint8_t* qw, const float* s_w, const float* bias,
+                                wq_bf16* y, void* workspace, size_t ws_bytes,
+                                wq_stream_t stream);
+
 /* Debug view of the GEMM's integer core: the same tensor-core mainloop with the
  * epilogue replaced by a raw store of the int32 accumulators acc [M][N]. */
 wq_status wq_debug_gemm_s32(const void* qx, int act_bits, const uint8_t* qw, int M, int N,

@@ -77,3 +77,24 @@ def gpu_gemm_s32(qx, bits, qw, K):
     acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
     wq.wq_debug_gemm_s32(dev(qx), bits, dev(qw), K, acc)
     return host(acc)
+
+
+def gpu_act_quant_static(x, cinv, sid, thr, gain, step, bits):
+    M, K = x.shape
+    qx = torch.empty((M, K) if bits == 8 else (M, K // 2),
+                     dtype=torch.int8 if bits == 8 else torch.uint8, device="cuda")
+    s_tok = torch.empty(M, dtype=torch.float32, device="cuda")
+    wq.wq_act_quant_static(dev(x), None if cinv is None else dev(cinv), dev(sid), dev(thr),
+                           dev(gain), step, bits, qx, s_tok)
+    return host(qx), host(s_tok)
+
+
+def gpu_linear_static(x, cinv, sid, thr, gain, beta, step, bits, qw, s_w, bias):
+    M, K = x.shape
+    N = qw.shape[0]
+    t = lambda a: None if a is None else (a if isinstance(a, torch.Tensor) else dev(a))
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = wq.alloc_workspace(M, K, N, bits)
+    wq.wq_linear_w4ax_static(t(x), t(cinv), t(sid), t(thr), t(gain), t(beta), step, bits, t(qw),
+                             t(s_w), t(bias), y, ws)
+    return host(y.view(torch.int16), np.uint16)

@@ -83,3 +83,29 @@ def test_other_entry_points_reject_on_host(lib):
     assert lib.wq_gemm_w4ax(FAKE, FAKE, 4, 16, 128, 32, FAKE, None, 3, 2, 2, FAKE, FAKE, None,
                             FAKE, None) == 4
     assert lib.wq_channel_scale(None, 4, FAKE, 4, 128, FAKE, FAKE, None) == 1
+
+
+def test_static_clipping_entry_points_reject_on_host(lib):
+    # wq_act_quant_static(x, M, K, cinv, sid, thr, gain, S, T, step, bits, qx, s_tok, st)
+    assert lib.wq_act_quant_static(FAKE, 8, 256, None, FAKE, None, FAKE, 3, 1, 0, 8, FAKE, FAKE,
+                                   None) == 1        # no thresholds
+    assert lib.wq_act_quant_static(FAKE, 8, 256, None, FAKE, FAKE, None, 3, 1, 0, 8, FAKE, FAKE,
+                                   None) == 1        # no gains
+    assert lib.wq_act_quant_static(FAKE, 8, 256, None, FAKE, FAKE, FAKE, 3, 1, 0, 6, FAKE, FAKE,
+                                   None) == 4        # bits
+    assert lib.wq_act_quant_static(FAKE, 8, 200, None, FAKE, FAKE, FAKE, 3, 1, 0, 8, FAKE, FAKE,
+                                   None) == 2        # K
+    assert lib.wq_act_quant_static(FAKE, 8, 256, None, FAKE, FAKE, FAKE, 3, 2, 2, 8, FAKE, FAKE,
+                                   None) == 4        # step outside the table
+    # wq_linear_w4ax_static(x, M, K, N, cinv, sid, thr, gain, beta, S, T, step, bits, qw, s_w,
+    #                       bias, y, ws, ws_bytes, st)
+    args = [FAKE, 64, 256, 256, FAKE, FAKE, FAKE, FAKE, FAKE, 3, 1, 0, 8, FAKE, FAKE, FAKE, FAKE,
+            FAKE, 1 << 30, None]
+    bad = list(args); bad[6] = None
+    assert lib.wq_linear_w4ax_static(*bad) == 1      # no thresholds
+    bad = list(args); bad[7] = None
+    assert lib.wq_linear_w4ax_static(*bad) == 1      # no gains
+    bad = list(args); bad[12] = 5
+    assert lib.wq_linear_w4ax_static(*bad) == 4      # bits
+    bad = list(args); bad[18] = 100
+    assert lib.wq_linear_w4ax_static(*bad) == 4      # workspace too small
