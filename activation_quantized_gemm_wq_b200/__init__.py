@@ -40,6 +40,8 @@ _SIGS = {
     "wq_act_quant_static": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "wq_linear_w4ax_static": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P,
                                    _P, _P, _P, ctypes.c_size_t, _P]),
+    "wq_linear_w4ax_single": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P,
+                                   _P, _P, _P]),
     "wq_debug_gemm_s32": (_I, [_P, _I, _P, _I, _I, _I, _P, _P]),
     "wq_device_status": (_I, [ctypes.POINTER(ctypes.c_uint)]),
 }
@@ -135,6 +137,18 @@ def wq_linear_w4ax_static(x, cinv, stream_id, thr, gain, beta, step, act_bits, q
     _call("wq_linear_w4ax_static", _ptr(x), M, K, N, _ptr(cinv), _ptr(stream_id), _ptr(thr),
           _ptr(gain), _ptr(beta), S, T, step, act_bits, _ptr(qw), _ptr(s_w), _ptr(bias), _ptr(y),
           _ptr(workspace), _nbytes(workspace), _stream(stream))
+
+
+def wq_linear_w4ax_single(x, cinv, stream_id, table, thr, beta, step, act_bits, qw, s_w, bias, y,
+                          stream=None):
+    """The fused linear as one kernel, for M <= 64 tokens (no workspace).  thr None:
+    dynamic clipping, table = alpha; else static clipping, table = the stream gains."""
+    M, K = x.shape
+    N = qw.shape[0]
+    T, S = table.shape
+    _call("wq_linear_w4ax_single", _ptr(x), M, K, N, _ptr(cinv), _ptr(stream_id), _ptr(table),
+          _ptr(thr), _ptr(beta), S, T, step, act_bits, _ptr(qw), _ptr(s_w), _ptr(bias), _ptr(y),
+          _stream(stream))
 
 
 def wq_gemm_w4ax(qx, s_tok, act_bits, K, stream_id, beta, S, T, step, qw, s_w, bias, y,

@@ -234,6 +234,26 @@ wq_status wq_linear_w4ax_static(const wq_bf16* x, int M, int K, int N, const flo
                 workspace, ws_bytes, stream, act_bits, thr);
 }
 
+wq_status wq_linear_w4ax_single(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                                const uint8_t* stream_id, const float* table, const float* thr,
+                                const float* beta, int S, int T, int step, int act_bits,
+                                const uint8_t* qw, const float* s_w, const float* bias,
+                                wq_bf16* y, wq_stream_t stream) {
+  if (act_bits != 8 && act_bits != 4) return WQ_ERR_ARG;
+  WQ_TRY(check_mk(M, K));
+  WQ_TRY(check_n(N));
+  WQ_TRY(check_table(S, T, step));
+  if (M > wq::kSingleKernelMaxM) return WQ_ERR_SHAPE;
+  if (M == 0) return WQ_OK;
+  if (!x || !stream_id || !table || !qw || !s_w || !y) return WQ_ERR_NULL;
+  if (!aligned16(x) || !aligned16(qw) || !aligned16(y) || !aligned16(s_w) ||
+      (cinv && !aligned16(cinv)) || (bias && !aligned16(bias)) || (beta && !aligned16(beta)))
+    return WQ_ERR_ALIGN;
+  const wq::EpilogueArgs ep{nullptr, stream_id, s_w, bias, beta, S, step};
+  return from_cuda(wq::launch_linear_single(x, cinv, table, thr, act_bits, qw, M, N, K, ep, y,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
 wq_status wq_gemm_w4ax(const void* qx, const float* s_tok, int act_bits, int M, int K, int N,
                        const uint8_t* stream_id, const float* beta, int S, int T, int step,
                        const uint8_t* qw, const float* s_w, const float* bias, wq_bf16* y,

@@ -29,6 +29,7 @@
 
 #include "wq_internal.h"
 #include "wq_ptx.cuh"
+#include "wq_quant.cuh"
 
 namespace wq {
 namespace {
@@ -43,6 +44,12 @@ struct TileArgs {
   int32_t* partial;  // bf16 split: [tiles][BN][128] int32 sums of the splits (zeroed)
   int* counters;     // bf16 split: [tiles][8] arrivals per epilogue-warp slice
   int w_prefetch;    // weights of the first NS K blocks loaded before griddep_wait()
+  // single-kernel linear (Cfg QBITS > 0): the bf16 activations, the channel
+  // scale [K] (or null) and the clip ratios [T][S] the kernel quantizes with
+  const uint16_t* q_x;
+  const float* q_cinv;
+  const float* q_alpha;  // clip ratios [T][S]; with q_thr, the stream gains [T][S]
+  const float* q_thr;    // static clipping thresholds [T], or null (dynamic)
   EpilogueArgs ep;
 };
 
@@ -61,11 +68,20 @@ __device__ __forceinline__ void split_range(int num_k, int splits, int sp, int& 
 #define WQ_UNPACK_WARPS_A8 4
 #endif
 
-template <int BN_, int ACT_BITS_, bool OUT_S32_>
+// QBITS > 0: the single-kernel linear for token counts that fit one tile.  The
+// producer also stages the bf16 activation tile; the epilogue warps compute each
+// token's scale once (its row maximum over all of K) before the first tile; the
+// unpack warps quantize every K block (qmax 127 or 7) straight into the int8
+// tile the MMA reads.  No codes go through HBM.
+template <int BN_, int ACT_BITS_, bool OUT_S32_, int QBITS_ = 0>
 struct Cfg {
   static constexpr int BN = BN_;
   static constexpr int ACT_BITS = ACT_BITS_;
   static constexpr bool OUT_S32 = OUT_S32_;
+  static constexpr int QBITS = QBITS_;
+  static constexpr int QMAX = QBITS == 4 ? 7 : 127;
+  static_assert(QBITS == 0 || (ACT_BITS == 8 && !OUT_S32 && BN <= 64),
+                "the single-kernel linear quantizes into the int8 mainloop, one token tile");
   static constexpr int BM = 128;  // output channels per tile (MMA M)
   static constexpr int BK = 128;  // K elements per pipeline stage
   static constexpr int UNPACK_WARPS = ACT_BITS == 4 ? 8 : WQ_UNPACK_WARPS_A8;
@@ -88,7 +104,9 @@ struct Cfg {
   static constexpr int WU_BYTES = BM * BK;                                   // int8 W
   static constexpr int XS_BYTES = ACT_BITS == 8 ? BN * BK : BN * BK / 2;     // staged x
   static constexpr int XU_BYTES = ACT_BITS == 8 ? 0 : BN * BK;               // int8 x (A4)
-  static constexpr int STAGE_BYTES = WP_BYTES + XS_BYTES;
+  static constexpr int XB_BYTES = QBITS ? BN * BK * 2 : 0;                  // staged bf16 x
+  static constexpr int STAGE_BYTES = WP_BYTES + (QBITS ? XB_BYTES : XS_BYTES);  // TMA bytes
+  static constexpr int STAGE_SMEM = WP_BYTES + XS_BYTES + XB_BYTES;
   // Pipeline: NS TMA stages (packed weights + activation tile), NU unpacked
   // buffers, and one "MMA done with K block g" barrier per stage (a ring of NS).
   // The single MMA-issuing thread does one wait and one commit per K block: it
@@ -102,28 +120,30 @@ struct Cfg {
   static constexpr int EPI_CHUNK = 16;  // token columns per TMEM load / TMA store
   static constexpr int NUM_CHUNKS = BN / EPI_CHUNK;
   static constexpr int EPI_BUF_BYTES = EPI_CHUNK * 32 * EPI_ELEM;
-  static constexpr int TOK_BYTES = 2 * BN * 4 + 2 * BN;  // staged s_tok and stream ids, x2
+  // staged s_tok and stream ids, x2; then (QBITS) each token's scale and its reciprocal
+  static constexpr int TOK_BYTES = 2 * BN * 4 + 2 * BN + (QBITS ? 2 * BN * 4 : 0);
   static constexpr int SMEM_LIMIT = 232448;  // 227 KB opt-in per CTA
   static constexpr int RESERVED = 1024 /*alignment slack*/ + 512 /*barriers*/;
   static constexpr int FIXED = RESERVED + NU * (WU_BYTES + XU_BYTES) + TOK_BYTES;
   // double-buffered epilogue staging unless that would cost a TMA stage below 4
   static constexpr int NS_WITH_2 =
-      (SMEM_LIMIT - FIXED - EPI_WARPS * 2 * EPI_BUF_BYTES) / STAGE_BYTES;
+      (SMEM_LIMIT - FIXED - EPI_WARPS * 2 * EPI_BUF_BYTES) / STAGE_SMEM;
   static constexpr int EPI_NBUF = NS_WITH_2 >= 4 ? 2 : 1;
   static constexpr int EPI_BYTES = EPI_WARPS * EPI_NBUF * EPI_BUF_BYTES;
-  static constexpr int NS_FIT = (SMEM_LIMIT - FIXED - EPI_BYTES) / STAGE_BYTES;
+  static constexpr int NS_FIT = (SMEM_LIMIT - FIXED - EPI_BYTES) / STAGE_SMEM;
   static constexpr int NS = NS_FIT > WQ_MAX_STAGES ? WQ_MAX_STAGES : NS_FIT;
   static_assert(NS >= NU && NS >= 2, "the done ring needs NS >= NU");
   static_assert(BN % EPI_CHUNK == 0 && NUM_CHUNKS >= 1, "token tile is a multiple of 16");
 
   static constexpr int OFF_WP = 0;
   static constexpr int OFF_XS = OFF_WP + NS * WP_BYTES;
-  static constexpr int OFF_WU = OFF_XS + NS * XS_BYTES;
+  static constexpr int OFF_XB = OFF_XS + NS * XS_BYTES;
+  static constexpr int OFF_WU = OFF_XB + NS * XB_BYTES;
   static constexpr int OFF_XU = OFF_WU + NU * WU_BYTES;
   static constexpr int OFF_EPI = OFF_XU + NU * XU_BYTES;
   static constexpr int OFF_TOK = OFF_EPI + EPI_BYTES;
   static constexpr int OFF_BAR = OFF_TOK + TOK_BYTES;
-  static constexpr int NUM_BARS = 2 * NS + NU + 6;
+  static constexpr int NUM_BARS = 2 * NS + NU + 7;
   static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
   static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
   static_assert(OFF_XS % 1024 == 0 && XS_BYTES % 512 == 0 && OFF_WU % 1024 == 0 &&
@@ -216,7 +236,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* tfull = ufull + C::NU;
   uint64_t* tempty = tfull + 2;
   uint64_t* tokbar = tempty + 2;  // epilogue warps: token staging of buffer i complete
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tokbar + 2);
+  uint64_t* qready = tokbar + 2;  // QBITS: every token scale of the tile is in shared memory
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qready + 1);
+  float* q_s = reinterpret_cast<float*>(smem + C::OFF_TOK + 2 * C::BN * 4 + 2 * C::BN);
+  float* q_r = q_s + C::BN;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -233,6 +256,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_init(&tempty[b], C::EPI_WARPS);
       mbar_init(&tokbar[b], C::EPI_WARPS);
     }
+    mbar_init(qready, C::EPI_WARPS);
     fence_mbar_init();
     fence_proxy_async_smem();
   }
@@ -292,8 +316,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             tma_load_2d(smem + C::OFF_WP + s * C::WP_BYTES, &tm_w, &full[s], kb * (C::BK / 2),
                         n_tile * C::BM);
           }
-          tma_load_2d(smem + C::OFF_XS + s * C::XS_BYTES, &tm_x, &full[s],
-                      kb * (C::ACT_BITS == 8 ? C::BK : C::BK / 2), m_tile * C::BN);
+          if constexpr (C::QBITS > 0) {  // bf16 x, two boxes of 64 channels
+            tma_load_2d(smem + C::OFF_XB + s * C::XB_BYTES, &tm_x, &full[s], kb * C::BK,
+                        m_tile * C::BN);
+            tma_load_2d(smem + C::OFF_XB + s * C::XB_BYTES + C::BN * 128, &tm_x, &full[s],
+                        kb * C::BK + 64, m_tile * C::BN);
+          } else {
+            tma_load_2d(smem + C::OFF_XS + s * C::XS_BYTES, &tm_x, &full[s],
+                        kb * (C::ACT_BITS == 8 ? C::BK : C::BK / 2), m_tile * C::BN);
+          }
         }
       }
       // Drain: the copies of every issued stage must have landed before the CTA
@@ -349,6 +380,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     constexpr int NT = C::UNPACK_WARPS * 32;
     uint32_t g = 0;
     bool ok = true;
+    if constexpr (C::QBITS > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(qready, 0));
     for (int unit = blockIdx.x; ok && unit < args.num_units; unit += gridDim.x) {
       int kb0, kb1;
       split_range(num_k, args.splits, unit % args.splits, kb0, kb1);
@@ -372,6 +404,41 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           unpack_tile<C::BN, NT, false>(smem + C::OFF_XS + s * C::XS_BYTES,
                                         smem + C::OFF_XU + u * C::XU_BYTES, tid);
         }
+        if constexpr (C::QBITS > 0) {
+          // chunk i: token row i / 16, channels 8*(i % 16) .. +7 of this K block
+          const uint8_t* xb = smem + C::OFF_XB + s * C::XB_BYTES;
+          uint8_t* xs = smem + C::OFF_XS + s * C::XS_BYTES;
+          for (int i = tid; i < C::BN * 16; i += NT) {
+            const int m = i >> 4, j = i & 15;
+            const uint4 raw = *reinterpret_cast<const uint4*>(xb + (j >> 3) * (C::BN * 128) +
+                                                               m * 128 + (j & 7) * 16);
+            const int k0 = kb * C::BK + 8 * j;
+            float ci[8];
+            if (args.q_cinv) {
+              const float4 a = __ldg(reinterpret_cast<const float4*>(args.q_cinv + k0));
+              const float4 b = __ldg(reinterpret_cast<const float4*>(args.q_cinv + k0 + 4));
+              ci[0] = a.x; ci[1] = a.y; ci[2] = a.z; ci[3] = a.w;
+              ci[4] = b.x; ci[5] = b.y; ci[6] = b.z; ci[7] = b.w;
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) ci[e] = 1.0f;
+            }
+            float v[8];
+            scale8(raw, ci, v);
+            const float sm = q_s[m], rm = q_r[m];
+            uint32_t q[8];
+            if (sm > 0.0f && isfinite(rm)) {
+              quantize8_recip<C::QMAX>(v, sm, rm, q);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) q[e] = static_cast<uint32_t>(quantize<C::QMAX>(v[e], sm));
+            }
+            // 8 codes -> bytes 8*(j%2) .. of 16-byte chunk j/2 of row m (128-byte swizzle)
+            *reinterpret_cast<uint2*>(xs + m * 128 + (((j >> 1) ^ (m & 7)) << 4) + (j & 1) * 8) =
+                make_uint2(pack_low_bytes(q[0], q[1], q[2], q[3]),
+                           pack_low_bytes(q[4], q[5], q[6], q[7]));
+          }
+        }
         fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
         __syncwarp();
         if (lane == 0) mbar_arrive(&ufull[u]);
@@ -393,6 +460,60 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const EpilogueArgs& ep = args.ep;
     const bool small_s = ep.S <= 4;
     griddep_wait();  // token scales and split-K scratch come from the previous kernel
+    if constexpr (C::QBITS > 0) {
+      // Token scales of the (single) token tile: the 256 epilogue threads split
+      // into BN groups of 256/BN lanes (within one warp), one token row per group;
+      // s = alpha[step][stream] * max_k |x * cinv| / qmax, over all of K.
+      constexpr int TPR = C::EPI_THREADS / C::BN;  // 4, 8 or 16 lanes per row
+      const int m = et / TPR, part = et % TPR;
+      const int nchunk = args.K >> 3;
+      float amax = 0.0f;
+      if (m < args.M && args.q_thr == nullptr) {  // static clipping needs no row maximum
+        const uint4* xr = reinterpret_cast<const uint4*>(args.q_x + (size_t)m * args.K);
+#pragma unroll 4
+        for (int c = part; c < nchunk; c += TPR) {
+          float ci[8], v[8];
+          if (args.q_cinv) {
+            const float4 a = __ldg(reinterpret_cast<const float4*>(args.q_cinv) + 2 * c);
+            const float4 b = __ldg(reinterpret_cast<const float4*>(args.q_cinv) + 2 * c + 1);
+            ci[0] = a.x; ci[1] = a.y; ci[2] = a.z; ci[3] = a.w;
+            ci[4] = b.x; ci[5] = b.y; ci[6] = b.z; ci[7] = b.w;
+          } else {
+#pragma unroll
+            for (int t = 0; t < 8; ++t) ci[t] = 1.0f;
+          }
+          scale8(__ldg(xr + c), ci, v);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) amax = fmaxf(amax, fabsf(v[t]));
+        }
+      }
+#pragma unroll
+      for (int o = TPR / 2; o > 0; o >>= 1)  // within the row's lane group
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      if (part == 0) {
+        float s_m = 0.0f;
+        if (m < args.M) {
+          const int sid = ep.stream_id[m];
+          if (sid < ep.S) {
+            const float tab = __ldg(args.q_alpha + ep.step * ep.S + sid);
+            float clip;
+            if (args.q_thr)  // clip = threshold / stream gain (0 when the gain is not positive)
+              clip = tab > 0.0f ? __fdiv_rn(__ldg(args.q_thr + ep.step), tab) : 0.0f;
+            else
+              clip = __fmul_rn(tab, amax);
+            s_m = __fdiv_rn(clip, static_cast<float>(C::QMAX));
+          } else {
+            raise_error(kErrBadStreamId);
+          }
+        }
+        q_s[m] = s_m;
+        q_r[m] = s_m > 0.0f ? __frcp_rn(s_m) : 0.0f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qready);
+      // every row's scale staged (after a timeout the waits below give up too)
+      __all_sync(0xFFFFFFFFu, mbar_wait(qready, 0));
+    }
     const bool split = args.splits > 1;
     for (int unit = blockIdx.x; unit < args.num_units; unit += gridDim.x, ++it) {
       const int tile = unit / args.splits;
@@ -409,7 +530,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (!C::OUT_S32) {
         for (int i = et; i < C::BN; i += C::EPI_THREADS) {
           const int m = m0 + i;
-          sts[i] = m < args.M ? ep.s_tok[m] : 0.0f;
+          if constexpr (C::QBITS > 0) sts[i] = q_s[i];  // the single token tile
+          else sts[i] = m < args.M ? ep.s_tok[m] : 0.0f;
           sds[i] = m < args.M ? ep.stream_id[m] : 0;
         }
         if (n < args.N) {
@@ -608,14 +730,25 @@ int sm_count() {
 
 int bn_for(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
 
+// Inputs of the single-kernel linear (Cfg QBITS > 0).
+struct SingleArgs {
+  const uint16_t* x;   // bf16 [M][K]
+  const float* cinv;   // [K] or null
+  const float* table;  // clip ratios [T][S], or the stream gains [T][S] with thr
+  const float* thr;    // static clipping thresholds [T], or null
+};
+
 template <class C>
 cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
                      const EpilogueArgs& ep, void* out, const SplitScratch* scratch,
-                     cudaStream_t st, bool w_prefetch) {
+                     cudaStream_t st, bool w_prefetch, const SingleArgs* single = nullptr) {
   CUtensorMap tm_w, tm_x, tm_out;
   bool ok = make_map(&tm_w, qw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, C::BK / 2, C::BM,
                      CU_TENSOR_MAP_SWIZZLE_64B);
-  if (C::ACT_BITS == 8)
+  if (C::QBITS > 0)  // bf16 activations, boxes of 64 channels x BN tokens
+    ok = ok && single && make_map(&tm_x, single->x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, 64,
+                                  C::BN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  else if (C::ACT_BITS == 8)
     ok = ok && make_map(&tm_x, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, C::BK, C::BN,
                         CU_TENSOR_MAP_SWIZZLE_128B);
   else
@@ -645,6 +778,10 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
   a.partial = scratch ? scratch->partial : nullptr;
   a.counters = scratch ? scratch->counters : nullptr;
   a.w_prefetch = w_prefetch ? 1 : 0;
+  a.q_x = single ? single->x : nullptr;
+  a.q_cinv = single ? single->cinv : nullptr;
+  a.q_alpha = single ? single->table : nullptr;
+  a.q_thr = single ? single->thr : nullptr;
   a.ep = ep;
 
   static bool attr_set = false;  // per template instance
@@ -671,7 +808,30 @@ cudaError_t dispatch_bn(const void* qx, const uint8_t* qw, int M, int N, int K,
   }
 }
 
+template <int QBITS>
+cudaError_t dispatch_single(const SingleArgs& sa, const uint8_t* qw, int M, int N, int K,
+                            const EpilogueArgs& ep, void* y, cudaStream_t st) {
+  switch (bn_for(M)) {
+    case 16: return run_gemm<Cfg<16, 8, false, QBITS>>(nullptr, qw, M, N, K, ep, y, nullptr, st,
+                                                       false, &sa);
+    case 32: return run_gemm<Cfg<32, 8, false, QBITS>>(nullptr, qw, M, N, K, ep, y, nullptr, st,
+                                                       false, &sa);
+    default: return run_gemm<Cfg<64, 8, false, QBITS>>(nullptr, qw, M, N, K, ep, y, nullptr, st,
+                                                       false, &sa);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_linear_single(const uint16_t* x, const float* cinv, const float* table,
+                                 const float* thr, int act_bits, const uint8_t* qw, int M, int N,
+                                 int K, const EpilogueArgs& ep, void* y, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  if (M > kSingleKernelMaxM) return cudaErrorInvalidValue;
+  const SingleArgs sa{x, cinv, table, thr};
+  return act_bits == 8 ? dispatch_single<8>(sa, qw, M, N, K, ep, y, st)
+                       : dispatch_single<4>(sa, qw, M, N, K, ep, y, st);
+}
 
 int gemm_splits(int M, int N, int K) {
   const int BN = bn_for(M);

@@ -67,6 +67,16 @@ struct EpilogueArgs {
   int step;
 };
 
+// The single-kernel linear (token counts up to kSingleKernelMaxM, one token tile):
+// the GEMM quantizes the bf16 activations itself (qmax 127 for act_bits 8, 7 for
+// 4) into its shared-memory operand tiles.  Dynamic clipping with table = alpha
+// [T][S] when thr is null; static clipping (clip = thr[step] / gain) with table =
+// the gains [T][S] otherwise.  ep.s_tok is unused.
+constexpr int kSingleKernelMaxM = 64;
+cudaError_t launch_linear_single(const uint16_t* x, const float* cinv, const float* table,
+                                 const float* thr, int act_bits, const uint8_t* qw, int M, int N,
+                                 int K, const EpilogueArgs& ep, void* y, cudaStream_t st);
+
 // Split-K (small token counts): the K blocks of each output tile are spread over
 // `splits` CTAs so that about kSplitTargetCtas CTAs stream the weights.  The
 // bf16 path needs scratch for the int32 partial tiles and one counter per

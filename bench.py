@@ -655,6 +655,15 @@ def sweep(args):
                 for M in S.SMALL_M:
                     entries.append((f"4 small-M {parent.name.split('_')[0]} A{bits} M{M}",
                                     S.small_m(parent, M, "action", bits), [li]))
+    # the single-kernel linear (quantization inside the GEMM) at token counts <= 64
+    for parent in (S.BLOCK2048_A8, S.BLOCK4096_A8):
+        for M in (16, 64):
+            for mode in ("dynamic", "static"):
+                entries.append((f"6 single-kernel {mode} {parent.name.split('_')[0]} A8 M{M}",
+                                S.small_m(parent, M, "action", 8), [0, 1, 2, 3]))
+                if mode == "static":  # the two-kernel static linear beside it
+                    entries.append((f"6 two-kernel static {parent.name.split('_')[0]} A8 M{M}",
+                                    S.small_m(parent, M, "action", 8), [0, 1, 2, 3]))
     rows = []
     cache = {}
     for label, wl, layers in entries:
@@ -706,9 +715,18 @@ def sweep(args):
                            thr=thr, gain=gain, bits=bits):
                     wq.wq_linear_w4ax_static(x_, cinv_, sid_, thr, gain, beta_, step_, bits, qw_,
                                              s_w_, bias_, y_, ws_)
+            if "single-kernel" in label:
+                def lin_fn(x_, cinv_, sid_, alpha_, beta_, step_, qw_, s_w_, bias_, y_, ws_,
+                           bits=bits, static=("static" in label)):
+                    if static:
+                        wq.wq_linear_w4ax_single(x_, cinv_, sid_, gain, thr, beta_, step_, bits,
+                                                 qw_, s_w_, bias_, y_)
+                    else:
+                        wq.wq_linear_w4ax_single(x_, cinv_, sid_, alpha_, None, beta_, step_,
+                                                 bits, qw_, s_w_, bias_, y_)
             for r in range(ncopy):
                 wq.wq_act_quant(xs[r], cinv, sid, alpha, step, bits, qxs[r], s_tok)
-            calls = max(10, ncopy)
+            calls = max(100 if M <= 256 else 10, ncopy)  # small M: at least 100 calls
             g_fns = [lambda r=r: wq.wq_gemm_w4ax(qxs[r % ncopy], s_tok, bits, K, sid, beta, 3, T,
                                                  step, qws[r % ncopy], s_w, bias, y)
                      for r in range(calls)]

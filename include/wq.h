@@ -164,6 +164,25 @@ wq_status wq_linear_w4ax_static(const wq_bf16* x, int M, int K, int N, const flo
                                 wq_bf16* y, void* workspace, size_t ws_bytes,
                                 wq_stream_t stream);
 
+/* The fused linear as ONE kernel, for token counts that fit one token tile
+ * (1 <= M <= 64; larger M returns WQ_ERR_SHAPE): the quantization (qmax 127 for
+ * act_bits 8, 7 for act_bits 4) runs inside the GEMM, which stages the bf16
+ * activations next to the weights and quantizes each K block into its
+ * shared-memory operand tile, so no codes pass through device memory and no
+ * workspace is needed.
+ *   thr == NULL: dynamic clipping as wq_linear_w4a8 / w4a4, table = alpha [T][S].
+ *     Every CTA first reads the tile's rows in full for their maxima.
+ *   thr != NULL: static clipping as wq_linear_w4ax_static, table = gain [T][S]
+ *     and thresholds thr [T]; no row maximum is needed.
+ * The pages split the linear into two kernels (§4.4); this single-kernel form is
+ * an option for tiny batches (action tokens).  Results equal the two-kernel
+ * calls bit for bit.  Other arguments as wq_linear_w4a8. */
+wq_status wq_linear_w4ax_single(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                                const uint8_t* stream_id, const float* table, const float* thr,
+                                const float* beta, int S, int T, int step, int act_bits,
+                                const uint8_t* qw, const float* s_w, const float* bias,
+                                wq_bf16* y, wq_stream_t stream);
+
 /* Debug view of the GEMM's integer core: the same tensor-core mainloop with the
  * epilogue replaced by a raw store of the int32 accumulators acc [M][N]. */
 wq_status wq_debug_gemm_s32(const void* qx, int act_bits, const uint8_t* qw, int M, int N,

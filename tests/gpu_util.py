@@ -98,3 +98,13 @@ def gpu_linear_static(x, cinv, sid, thr, gain, beta, step, bits, qw, s_w, bias):
     wq.wq_linear_w4ax_static(t(x), t(cinv), t(sid), t(thr), t(gain), t(beta), step, bits, t(qw),
                              t(s_w), t(bias), y, ws)
     return host(y.view(torch.int16), np.uint16)
+
+
+def gpu_linear_single(x, cinv, sid, table, beta, step, bits, qw, s_w, bias, thr=None):
+    M, K = x.shape
+    N = qw.shape[0]
+    t = lambda a: None if a is None else (a if isinstance(a, torch.Tensor) else dev(a))
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    wq.wq_linear_w4ax_single(t(x), t(cinv), t(sid), t(table), t(thr), t(beta), step, bits, t(qw),
+                             t(s_w), t(bias), y)
+    return host(y.view(torch.int16), np.uint16)

@@ -109,3 +109,19 @@ def test_static_clipping_entry_points_reject_on_host(lib):
     assert lib.wq_linear_w4ax_static(*bad) == 4      # bits
     bad = list(args); bad[18] = 100
     assert lib.wq_linear_w4ax_static(*bad) == 4      # workspace too small
+
+
+def test_single_kernel_linear_rejects_on_host(lib):
+    # (x, M, K, N, cinv, sid, table, thr, beta, S, T, step, bits, qw, s_w, bias, y, st)
+    args = [FAKE, 64, 256, 256, FAKE, FAKE, FAKE, None, FAKE, 3, 1, 0, 8, FAKE, FAKE, FAKE, FAKE,
+            None]
+    bad = list(args); bad[1] = 65
+    assert lib.wq_linear_w4ax_single(*bad) == 2      # more tokens than one tile
+    bad = list(args); bad[6] = None
+    assert lib.wq_linear_w4ax_single(*bad) == 1      # no clip table
+    bad = list(args); bad[12] = 6
+    assert lib.wq_linear_w4ax_single(*bad) == 4      # bits
+    bad = list(args); bad[0] = MIS
+    assert lib.wq_linear_w4ax_single(*bad) == 3      # misaligned x
+    bad = list(args); bad[1] = 0
+    assert lib.wq_linear_w4ax_single(*bad) == 0      # empty batch: nothing to do
