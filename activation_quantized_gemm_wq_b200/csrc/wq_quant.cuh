@@ -105,6 +105,19 @@ __device__ __forceinline__ void load_cinv8(const float* cinv_s, int c, float (&c
   ci[4] = b.x; ci[5] = b.y; ci[6] = b.z; ci[7] = b.w;
 }
 
+// cinv chunk c through L1, or all ones when there is no channel scale.
+__device__ __forceinline__ void load_cinv8_global(const float* cinv, int c, float (&ci)[8]) {
+  if (cinv == nullptr) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ci[e] = 1.0f;
+    return;
+  }
+  const float4 a = __ldg(reinterpret_cast<const float4*>(cinv) + 2 * c);
+  const float4 b = __ldg(reinterpret_cast<const float4*>(cinv) + 2 * c + 1);
+  ci[0] = a.x; ci[1] = a.y; ci[2] = a.z; ci[3] = a.w;
+  ci[4] = b.x; ci[5] = b.y; ci[6] = b.z; ci[7] = b.w;
+}
+
 // x' = x * cinv for one chunk of 8 channels (bf16 widening is exact).
 __device__ __forceinline__ void scale8(const uint4 raw, const float (&ci)[8], float (&v)[8]) {
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -266,11 +279,132 @@ cudaError_t run_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                     alpha, thr, S, step, qx, s_tok, zero, zero_n16);
 }
 
+// One warp per token row, no block-level synchronisation: pass 1 streams the row
+// for its maximum (absent with static clipping), pass 2 reads it again (from L2)
+// and writes the codes.  Warps progress independently, so one warp's loads
+// overlap other warps' arithmetic.
+template <int ACT_BITS, int STORE_BITS, bool STATIC>
+__global__ void __launch_bounds__(256) act_quant_row_kernel(
+    const uint16_t* __restrict__ x, int M, int K, const float* __restrict__ cinv,
+    const uint8_t* __restrict__ stream_id, const float* __restrict__ alpha,
+    const float* __restrict__ thr, int S, int step, void* __restrict__ qx,
+    float* __restrict__ s_tok, uint4* __restrict__ zero, size_t zero_n16) {
+  constexpr int QMAX = ACT_BITS == 8 ? 127 : 7;
+  constexpr int U = 4;  // chunks in flight per lane
+  griddep_wait();
+  griddep_launch_dependents();
+  for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < zero_n16; i += (size_t)gridDim.x * 256)
+    zero[i] = make_uint4(0u, 0u, 0u, 0u);
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * 8;
+  const int nchunk = K >> 3;
+  for (int row = blockIdx.x * 8 + (threadIdx.x >> 5); row < M; row += nwarps) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * K);
+    float amax = 0.0f;
+    if constexpr (!STATIC) {
+      for (int c0 = lane; c0 < nchunk; c0 += 32 * U) {
+        uint4 raw[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int c = c0 + 32 * u;
+          raw[u] = c < nchunk ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int c = c0 + 32 * u;
+          if (c < nchunk) {
+            float ci[8], v[8];
+            load_cinv8_global(cinv, c, ci);
+            scale8(raw[u], ci, v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+          }
+        }
+      }
+      amax = warp_max(amax);
+    }
+    float s = 0.0f;
+    const int sid = stream_id[row];
+    if (sid < S) {
+      float clip;
+      if constexpr (STATIC) {
+        const float g = __ldg(alpha + step * S + sid);
+        clip = g > 0.0f ? __fdiv_rn(__ldg(thr + step), g) : 0.0f;
+      } else {
+        clip = __fmul_rn(__ldg(alpha + step * S + sid), amax);
+      }
+      s = __fdiv_rn(clip, static_cast<float>(QMAX));
+    } else if (lane == 0) {
+      raise_error(kErrBadStreamId);
+    }
+    if (lane == 0) s_tok[row] = s;
+    const float r = s > 0.0f ? __frcp_rn(s) : 0.0f;
+    const bool fast = s > 0.0f && isfinite(r);
+    for (int c0 = lane; c0 < nchunk; c0 += 32 * U) {
+      uint4 raw[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + 32 * u;
+        raw[u] = c < nchunk ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + 32 * u;
+        if (c >= nchunk) continue;
+        float ci[8], v[8];
+        load_cinv8_global(cinv, c, ci);
+        scale8(raw[u], ci, v);
+        uint32_t q[8];
+        if (fast) {
+          quantize8_recip<QMAX>(v, s, r, q);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) q[e] = static_cast<uint32_t>(quantize<QMAX>(v[e], s));
+        }
+        if constexpr (STORE_BITS == 8) {
+          reinterpret_cast<uint2*>(static_cast<int8_t*>(qx) + (size_t)row * K)[c] =
+              make_uint2(pack_low_bytes(q[0], q[1], q[2], q[3]),
+                         pack_low_bytes(q[4], q[5], q[6], q[7]));
+        } else {
+          reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(qx) + (size_t)row * (K / 2))[c] =
+              pack_low_nibbles(q);
+        }
+      }
+    }
+  }
+}
+
+template <int ACT_BITS, int STORE_BITS, bool STATIC>
+cudaError_t run_act_quant_rows(const uint16_t* x, int M, int K, const float* cinv,
+                               const uint8_t* sid, const float* alpha, const float* thr, int S,
+                               int step, void* qx, float* s_tok, uint4* zero, size_t zero_n16,
+                               cudaStream_t st) {
+  static int per_sm = 0;  // per template instance
+  if (per_sm == 0) {
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+        &per_sm, act_quant_row_kernel<ACT_BITS, STORE_BITS, STATIC>, 256, 0);
+    if (per_sm < 1) per_sm = 1;
+  }
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int want = (M + 7) / 8;  // one warp per row
+  const int grid = want < per_sm * sms ? want : per_sm * sms;
+  return launch_pdl(act_quant_row_kernel<ACT_BITS, STORE_BITS, STATIC>, grid, 256, 0, st, x, M,
+                    K, cinv, sid, alpha, thr, S, step, qx, s_tok, zero, zero_n16);
+}
+
 template <int ACT_BITS, int STORE_BITS, bool STATIC>
 cudaError_t dispatch_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                                const uint8_t* sid, const float* alpha, const float* thr, int S,
                                int step, void* qx, float* s_tok, uint4* zero, size_t zero_n16,
                                cudaStream_t st) {
+  // Many rows of moderate length: independent warps, one per row (measured faster
+  // for M = 4288 and 8512 at K = 2048 and 4096).  Few rows, or long rows, keep a
+  // CTA's threads on each row (measured faster for M <= 256, and for K >= 8192).
+  if (M >= 1024 && K <= 4096)
+    return run_act_quant_rows<ACT_BITS, STORE_BITS, STATIC>(x, M, K, cinv, sid, alpha, thr, S,
+                                                            step, qx, s_tok, zero, zero_n16, st);
   const int nchunk = K / 8;
 #define WQ_AQ(TPR, CPT) \
   return run_act_quant<ACT_BITS, STORE_BITS, TPR, CPT, STATIC>(x, M, K, cinv, sid, alpha, thr, S, \

@@ -50,7 +50,9 @@ def test_channel_scale_and_pack_bit_exact(oracle, wl, layer):
 
 # ------------------------------------------------------------------ activation codes
 
-AQ_SHAPES = [(64, 256), (37, 384), (300, 2048), (16, 8192), (9, 16384), (3, 32768), (1, 128)]
+# M >= 1024 with K <= 4096 takes the one-warp-per-row kernel, the rest the CTA-per-rows one
+AQ_SHAPES = [(64, 256), (37, 384), (300, 2048), (16, 8192), (9, 16384), (3, 32768), (1, 128),
+             (1100, 256), (1030, 4096), (2048, 2048)]
 
 
 @pytest.mark.parametrize("bits", [8, 4])
@@ -70,6 +72,19 @@ def test_act_quant_bit_exact(oracle, M, K, bits):
         q, s = gpu_act_quant(x, ci, sid, alpha, step, bits)
         assert np.array_equal(_f32bits(s), _f32bits(s_ref))
         assert np.array_equal(q.view(np.uint8), q_ref.view(np.uint8))
+
+
+@pytest.mark.parametrize("bits,qmax", [(8, 127), (4, 7)])
+def test_act_quant_near_ties_many_rows(oracle, bits, qmax):
+    """Near-tie rows tiled to 1024 rows (the one-warp-per-row kernel)."""
+    x1, cinv = P.near_tie_inputs(21, K=4096, qmax=qmax)
+    x = np.ascontiguousarray(np.repeat(x1, 1024, axis=0))
+    sid = np.zeros(x.shape[0], np.uint8)
+    alpha = np.ones((1, 1), np.float32)
+    q_ref, s_ref = oracle.act_quant(x1, cinv, sid[:1], alpha, 0, bits)
+    q, s = gpu_act_quant(x, cinv, sid, alpha, 0, bits)
+    assert np.array_equal(_f32bits(s), np.repeat(_f32bits(s_ref), x.shape[0]))
+    assert np.array_equal(q.view(np.uint8), np.repeat(q_ref.view(np.uint8), x.shape[0], axis=0))
 
 
 @pytest.mark.parametrize("bits,qmax", [(8, 127), (4, 7)])

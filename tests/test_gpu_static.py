@@ -38,7 +38,8 @@ def _tables(g, T, Sn, x, cinv, qmax):
 
 
 @pytest.mark.parametrize("bits,qmax", [(8, 127), (4, 7)])
-@pytest.mark.parametrize("M,K", [(64, 256), (300, 2048), (16, 8192), (3, 32768), (37, 384)])
+@pytest.mark.parametrize("M,K", [(64, 256), (300, 2048), (16, 8192), (3, 32768), (37, 384),
+                                 (1200, 2048)])
 def test_act_quant_static_bit_exact(oracle, M, K, bits, qmax):
     g = np.random.default_rng(M * 13 + K)
     wl = S.custom(f"st{M}x{K}", K, 16, ((0, M),), act_bits=bits, T=3)
