@@ -52,7 +52,7 @@ def test_channel_scale_and_pack_bit_exact(oracle, wl, layer):
 
 # M >= 1024 with K <= 4096 takes the one-warp-per-row kernel, the rest the CTA-per-rows one
 AQ_SHAPES = [(64, 256), (37, 384), (300, 2048), (16, 8192), (9, 16384), (3, 32768), (1, 128),
-             (1100, 256), (1030, 4096), (2048, 2048)]
+             (1100, 256), (1030, 4096), (2048, 2048), (1050, 8192), (1025, 32768)]
 
 
 @pytest.mark.parametrize("bits", [8, 4])
