@@ -784,13 +784,9 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
   a.q_thr = single ? single->thr : nullptr;
   a.ep = ep;
 
-  static bool attr_set = false;  // per template instance
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static bool attr_set[kAttrDevices] = {};  // per template instance and device
+  const cudaError_t e = set_smem_once(gemm_kernel<C>, C::SMEM_BYTES, attr_set);
+  if (e != cudaSuccess) return e;
   const int grid = a.num_units < sm_count() ? a.num_units : sm_count();
   return launch_pdl(gemm_kernel<C>, grid, C::THREADS, C::SMEM_BYTES, st, tm_w, tm_x, tm_out, a);
 }

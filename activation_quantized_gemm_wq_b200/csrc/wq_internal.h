@@ -28,6 +28,22 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t sme
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// Set a kernel's shared-memory limit once per device: function attributes belong
+// to each device's context, so a process that drives several GPUs sets them on
+// each.  `done` is the caller's per-kernel flag array.
+constexpr int kAttrDevices = 64;
+template <class Kernel>
+cudaError_t set_smem_once(Kernel kernel, int bytes, bool (&done)[kAttrDevices]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaGetLastError();
+  const bool cached = dev >= 0 && dev < kAttrDevices;
+  if (cached && done[dev]) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && cached) done[dev] = true;
+  return e;
+}
+
 // Largest K the quantizer keeps in registers (K/8 chunks spread over 256 threads,
 // at most 16 chunks each).
 constexpr int kMaxK = 32768;

@@ -256,17 +256,15 @@ cudaError_t run_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                           cudaStream_t st) {
   constexpr int RPC = 256 / TPR;
   const size_t smem = static_cast<size_t>(K) * sizeof(float);  // cinv copy
-  static bool attr_set = false;  // per template instance
+  static bool attr_set[kAttrDevices] = {};  // per template instance and device
   static int per_sm = 0, per_sm_k = 0;  // resident CTAs per SM at K = per_sm_k
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT, STATIC>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxK * 4) != cudaSuccess)
-      return cudaGetLastError();
-    attr_set = true;
-  }
+  // cinv's shared-memory copy: up to kMaxK floats
+  const cudaError_t ea = set_smem_once(act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT, STATIC>,
+                                       kMaxK * 4, attr_set);
+  if (ea != cudaSuccess) return ea;
   if (per_sm_k != K) {
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT, STATIC>,
-                                                  256, smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+        &per_sm, act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT, STATIC>, 256, smem);
     if (per_sm < 1) per_sm = 1;
     per_sm_k = K;
   }
