@@ -67,12 +67,25 @@ def parse():
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_traffic_block2048_w4a8.md")
 GEMM_SOURCES = [os.path.join(ROOT, "activation_quantized_gemm_wq_b200", "csrc", f)
                 for f in ("wq_gemm.cuh", "wq_ptx.cuh")]
+HOST_SIDE_MARKER = b"// ------------------------------------------------------------------ host side"
+
+
+def gemm_device_source_hash(paths=None):
+    """sha256 of the GEMM kernel's device code: each source file up to its host-side
+    marker (the whole file when it has none), concatenated in order."""
+    import hashlib
+    h = hashlib.sha256()
+    for path in paths or GEMM_SOURCES:
+        with open(path, "rb") as f:
+            data = f.read()
+        cut = data.find(HOST_SIDE_MARKER)
+        h.update(data if cut < 0 else data[:cut])
+    return h.hexdigest()
 
 
 def gemm_traffic(workload):
     """DRAM bytes per GEMM launch from the committed ncu capture of this workload, or
     None when there is none or the GEMM sources changed since it was taken."""
-    import hashlib
     if workload != "block2048_w4a8":
         return None
     try:
@@ -82,11 +95,7 @@ def gemm_traffic(workload):
                 if ":" in line and line.startswith("    "):
                     k, v = line.strip().split(":", 1)
                     fields[k.strip()] = v.strip()
-        h = hashlib.sha256()
-        for path in GEMM_SOURCES:
-            with open(path, "rb") as f:
-                h.update(f.read())
-        if h.hexdigest() != fields.get("source_sha256"):
+        if gemm_device_source_hash() != fields.get("source_sha256"):
             return None
         return int(fields["traffic_bytes_per_launch"])
     except (OSError, KeyError, ValueError):

@@ -69,3 +69,20 @@ def test_gemm_traffic_tracks_the_kernel_source(tmp_path, monkeypatch):
     assert bench.gemm_traffic("block4096_w4a8_t10") is None   # no capture for that workload
     src.write_bytes(b"kernel v2")                              # the kernel changed since
     assert bench.gemm_traffic("block2048_w4a8") is None
+
+
+def test_gemm_traffic_ignores_host_side_edits(tmp_path, monkeypatch):
+    """Only the device code before the host-side marker identifies the kernel."""
+    marker = bench.HOST_SIDE_MARKER.decode()
+    src = tmp_path / "g.cuh"
+    src.write_text(f"__global__ void k() {{}}\n{marker}\nint host_a();\n")
+    digest = bench.gemm_device_source_hash([str(src)])
+    prof = tmp_path / "traffic.md"
+    prof.write_text(f"    traffic_bytes_per_launch: 77\n    source_sha256: {digest}\n")
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(prof))
+    monkeypatch.setattr(bench, "GEMM_SOURCES", [str(src)])
+    assert bench.gemm_traffic("block2048_w4a8") == 77
+    src.write_text(f"__global__ void k() {{}}\n{marker}\nint host_b();\n")   # host side only
+    assert bench.gemm_traffic("block2048_w4a8") == 77
+    src.write_text(f"__global__ void k() {{ int x; }}\n{marker}\nint host_b();\n")  # device
+    assert bench.gemm_traffic("block2048_w4a8") is None
