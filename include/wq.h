@@ -33,6 +33,10 @@
  *   - bf16 tensors are passed as raw 16-bit patterns (wq_bf16).
  *   - Calls are asynchronous on `stream` (NULL = the legacy default stream).
  *     Argument errors are returned synchronously before anything is launched.
+ *   - Kernels are launched with programmatic stream serialization: one may start
+ *     while the previous kernel in the stream finishes, but it waits for that
+ *     kernel before touching memory, so stream order is preserved (and the calls
+ *     can be captured in CUDA graphs).
  *   - Nothing throws or aborts across this boundary.
  *   - Preconditions checked on the host: M >= 0 (M == 0 returns WQ_OK at once
  *     after the size and table checks; token tensors may then be NULL), K a
@@ -184,7 +188,8 @@ wq_status wq_linear_w4ax_single(const wq_bf16* x, int M, int K, int N, const flo
                                 wq_bf16* y, wq_stream_t stream);
 
 /* Debug view of the GEMM's integer core: the same tensor-core mainloop with the
- * epilogue replaced by a raw store of the int32 accumulators acc [M][N]. */
+ * epilogue replaced by a raw store of the int32 accumulators acc [M][N] (every
+ * element is overwritten).  qx as in wq_gemm_w4ax. */
 wq_status wq_debug_gemm_s32(const void* qx, int act_bits, const uint8_t* qw, int M, int N,
                             int K, int32_t* acc, wq_stream_t stream);
 
