@@ -5,8 +5,13 @@ Argument marshalling only: every step runs in the CUDA library.  Tensors are
 torch CUDA tensors (device memory and streams come from PyTorch); bf16 tensors
 may be torch.bfloat16 or raw 16-bit integer tensors.  Each function has the
 name and argument order of its C entry point, with sizes taken from the tensor
-shapes.  There is no CPU fallback: if libwq.so is missing or fails to load,
-importing the functions raises.
+shapes.  The C entry points take plain pointers and cannot see how large a
+buffer is, so before each call the binding checks every tensor against what the
+call will read or write there: on the current CUDA device, contiguous, of the
+element type the header names, and holding at least that many elements.  A
+tensor that fails raises here (TypeError for the type, ValueError otherwise)
+instead of reaching a kernel that would run past its end.  There is no CPU
+fallback: if libwq.so is missing or fails to load, calling the functions raises.
 """
 import ctypes
 import os
@@ -69,14 +74,42 @@ def lib():
     return _lib
 
 
-def _ptr(t):
+# element types the header names for each kind of tensor
+_BF16 = frozenset({"torch.bfloat16", "torch.int16", "torch.uint16"})
+_F32 = frozenset({"torch.float32"})
+_BYTES = frozenset({"torch.uint8", "torch.int8"})
+_I32 = frozenset({"torch.int32"})
+
+
+def _current_device():
+    import torch
+    return torch.cuda.current_device()
+
+
+def _ptr(t, name, kinds=None, count=0):
+    """Device address of tensor `t`, which the C call reads or writes as `count`
+    elements of one of the element types `kinds` (None: any type, e.g. the
+    workspace).  None passes through: the library decides which pointers may be
+    NULL and returns WQ_ERR_NULL for the others."""
     if t is None:
         return None
     if not t.is_cuda:
-        raise ValueError("libwq takes device tensors")
+        raise ValueError(f"{name}: libwq takes device tensors")
     if not t.is_contiguous():
-        raise ValueError("libwq takes contiguous tensors")
+        raise ValueError(f"{name}: libwq takes contiguous tensors")
+    if kinds is not None and str(t.dtype) not in kinds:
+        raise TypeError(f"{name}: element type {t.dtype}, expected one of {sorted(kinds)}")
+    if t.numel() < count:
+        raise ValueError(f"{name}: {t.numel()} elements, the call uses {count}")
+    if t.get_device() != _current_device():
+        raise ValueError(f"{name}: on cuda:{t.get_device()}, the current device is "
+                         f"cuda:{_current_device()}")
     return t.data_ptr()
+
+
+def _codes_per_row(K, act_bits):
+    """Bytes per token row of activation codes: K int8 codes, or K/2 packed int4."""
+    return K // 2 if act_bits == 4 else K
 
 
 def _stream(stream):
@@ -106,65 +139,86 @@ def wq_workspace_bytes(M, K, N, act_bits):
 
 def wq_channel_scale(x_cal, W, c, cinv, stream=None):
     Mcal, K = x_cal.shape
-    _call("wq_channel_scale", _ptr(x_cal), Mcal, _ptr(W), W.shape[0], K, _ptr(c), _ptr(cinv),
+    N = W.shape[0]
+    _call("wq_channel_scale", _ptr(x_cal, "x_cal", _BF16, Mcal * K), Mcal,
+          _ptr(W, "W", _BF16, N * K), N, K, _ptr(c, "c", _F32, K), _ptr(cinv, "cinv", _F32, K),
           _stream(stream))
 
 
 def wq_pack_int4(W, c, qw, s_w, stream=None):
     N, K = W.shape
-    _call("wq_pack_int4", _ptr(W), _ptr(c), N, K, _ptr(qw), _ptr(s_w), _stream(stream))
+    _call("wq_pack_int4", _ptr(W, "W", _BF16, N * K), _ptr(c, "c", _F32, K), N, K,
+          _ptr(qw, "qw", _BYTES, N * (K // 2)), _ptr(s_w, "s_w", _F32, N), _stream(stream))
 
 
 def wq_act_quant(x, cinv, stream_id, alpha, step, act_bits, qx, s_tok, stream=None):
     M, K = x.shape
     T, S = alpha.shape
-    _call("wq_act_quant", _ptr(x), M, K, _ptr(cinv), _ptr(stream_id), _ptr(alpha), S, T, step,
-          act_bits, _ptr(qx), _ptr(s_tok), _stream(stream))
+    _call("wq_act_quant", _ptr(x, "x", _BF16, M * K), M, K, _ptr(cinv, "cinv", _F32, K),
+          _ptr(stream_id, "stream_id", _BYTES, M), _ptr(alpha, "alpha", _F32, T * S), S, T, step,
+          act_bits, _ptr(qx, "qx", _BYTES, M * _codes_per_row(K, act_bits)),
+          _ptr(s_tok, "s_tok", _F32, M), _stream(stream))
 
 
 def wq_act_quant_static(x, cinv, stream_id, thr, gain, step, act_bits, qx, s_tok, stream=None):
     M, K = x.shape
     T, S = gain.shape
-    _call("wq_act_quant_static", _ptr(x), M, K, _ptr(cinv), _ptr(stream_id), _ptr(thr),
-          _ptr(gain), S, T, step, act_bits, _ptr(qx), _ptr(s_tok), _stream(stream))
+    _call("wq_act_quant_static", _ptr(x, "x", _BF16, M * K), M, K, _ptr(cinv, "cinv", _F32, K),
+          _ptr(stream_id, "stream_id", _BYTES, M), _ptr(thr, "thr", _F32, T),
+          _ptr(gain, "gain", _F32, T * S), S, T, step, act_bits,
+          _ptr(qx, "qx", _BYTES, M * _codes_per_row(K, act_bits)),
+          _ptr(s_tok, "s_tok", _F32, M), _stream(stream))
+
+
+def _token_and_weight_args(x, cinv, stream_id, beta, S, T, qw, s_w, bias, y):
+    """The pointers every fused linear takes, checked for x [M][K], qw [N][K/2]."""
+    M, K = x.shape
+    N = qw.shape[0]
+    return dict(M=M, K=K, N=N,
+                x=_ptr(x, "x", _BF16, M * K), cinv=_ptr(cinv, "cinv", _F32, K),
+                sid=_ptr(stream_id, "stream_id", _BYTES, M),
+                beta=_ptr(beta, "beta", _F32, T * S * N), qw=_ptr(qw, "qw", _BYTES, N * (K // 2)),
+                s_w=_ptr(s_w, "s_w", _F32, N), bias=_ptr(bias, "bias", _F32, N),
+                y=_ptr(y, "y", _BF16, M * N))
 
 
 def wq_linear_w4ax_static(x, cinv, stream_id, thr, gain, beta, step, act_bits, qw, s_w, bias, y,
                           workspace, stream=None):
-    M, K = x.shape
-    N = qw.shape[0]
     T, S = gain.shape
-    _call("wq_linear_w4ax_static", _ptr(x), M, K, N, _ptr(cinv), _ptr(stream_id), _ptr(thr),
-          _ptr(gain), _ptr(beta), S, T, step, act_bits, _ptr(qw), _ptr(s_w), _ptr(bias), _ptr(y),
-          _ptr(workspace), _nbytes(workspace), _stream(stream))
+    a = _token_and_weight_args(x, cinv, stream_id, beta, S, T, qw, s_w, bias, y)
+    _call("wq_linear_w4ax_static", a["x"], a["M"], a["K"], a["N"], a["cinv"], a["sid"],
+          _ptr(thr, "thr", _F32, T), _ptr(gain, "gain", _F32, T * S), a["beta"], S, T, step,
+          act_bits, a["qw"], a["s_w"], a["bias"], a["y"], _ptr(workspace, "workspace"),
+          _nbytes(workspace), _stream(stream))
 
 
 def wq_linear_w4ax_single(x, cinv, stream_id, table, thr, beta, step, act_bits, qw, s_w, bias, y,
                           stream=None):
     """The fused linear as one kernel, for M <= 64 tokens (no workspace).  thr None:
     dynamic clipping, table = alpha; else static clipping, table = the stream gains."""
-    M, K = x.shape
-    N = qw.shape[0]
     T, S = table.shape
-    _call("wq_linear_w4ax_single", _ptr(x), M, K, N, _ptr(cinv), _ptr(stream_id), _ptr(table),
-          _ptr(thr), _ptr(beta), S, T, step, act_bits, _ptr(qw), _ptr(s_w), _ptr(bias), _ptr(y),
-          _stream(stream))
+    a = _token_and_weight_args(x, cinv, stream_id, beta, S, T, qw, s_w, bias, y)
+    _call("wq_linear_w4ax_single", a["x"], a["M"], a["K"], a["N"], a["cinv"], a["sid"],
+          _ptr(table, "table", _F32, T * S), _ptr(thr, "thr", _F32, T), a["beta"], S, T, step,
+          act_bits, a["qw"], a["s_w"], a["bias"], a["y"], _stream(stream))
 
 
 def wq_gemm_w4ax(qx, s_tok, act_bits, K, stream_id, beta, S, T, step, qw, s_w, bias, y,
                  stream=None):
     M, N = y.shape
-    _call("wq_gemm_w4ax", _ptr(qx), _ptr(s_tok), act_bits, M, K, N, _ptr(stream_id), _ptr(beta),
-          S, T, step, _ptr(qw), _ptr(s_w), _ptr(bias), _ptr(y), _stream(stream))
+    _call("wq_gemm_w4ax", _ptr(qx, "qx", _BYTES, M * _codes_per_row(K, act_bits)),
+          _ptr(s_tok, "s_tok", _F32, M), act_bits, M, K, N,
+          _ptr(stream_id, "stream_id", _BYTES, M), _ptr(beta, "beta", _F32, T * S * N), S, T,
+          step, _ptr(qw, "qw", _BYTES, N * (K // 2)), _ptr(s_w, "s_w", _F32, N),
+          _ptr(bias, "bias", _F32, N), _ptr(y, "y", _BF16, M * N), _stream(stream))
 
 
 def _linear(name, x, cinv, stream_id, alpha, beta, step, qw, s_w, bias, y, workspace, stream):
-    M, K = x.shape
-    N = qw.shape[0]
     T, S = alpha.shape
-    _call(name, _ptr(x), M, K, N, _ptr(cinv), _ptr(stream_id), _ptr(alpha), _ptr(beta), S, T,
-          step, _ptr(qw), _ptr(s_w), _ptr(bias), _ptr(y), _ptr(workspace), _nbytes(workspace),
-          _stream(stream))
+    a = _token_and_weight_args(x, cinv, stream_id, beta, S, T, qw, s_w, bias, y)
+    _call(name, a["x"], a["M"], a["K"], a["N"], a["cinv"], a["sid"],
+          _ptr(alpha, "alpha", _F32, T * S), a["beta"], S, T, step, a["qw"], a["s_w"], a["bias"],
+          a["y"], _ptr(workspace, "workspace"), _nbytes(workspace), _stream(stream))
 
 
 def wq_linear_w4a8(x, cinv, stream_id, alpha, beta, step, qw, s_w, bias, y, workspace,
@@ -183,16 +237,18 @@ def wq_linear_w4a8_noalloc(x, cinv, stream_id, alpha, beta, step, qw, s_w, bias,
                            stream=None):
     """wq_linear_w4a8 without a workspace: for callers that cannot allocate device
     memory while they run.  Uses the library's fixed 16 MiB scratch (see wq.h)."""
-    M, K = x.shape
-    N = qw.shape[0]
     T, S = alpha.shape
-    _call("wq_linear_w4a8_noalloc", _ptr(x), M, K, N, _ptr(cinv), _ptr(stream_id), _ptr(alpha),
-          _ptr(beta), S, T, step, _ptr(qw), _ptr(s_w), _ptr(bias), _ptr(y), _stream(stream))
+    a = _token_and_weight_args(x, cinv, stream_id, beta, S, T, qw, s_w, bias, y)
+    _call("wq_linear_w4a8_noalloc", a["x"], a["M"], a["K"], a["N"], a["cinv"], a["sid"],
+          _ptr(alpha, "alpha", _F32, T * S), a["beta"], S, T, step, a["qw"], a["s_w"],
+          a["bias"], a["y"], _stream(stream))
 
 
 def wq_debug_gemm_s32(qx, act_bits, qw, K, acc, stream=None):
     M, N = acc.shape
-    _call("wq_debug_gemm_s32", _ptr(qx), act_bits, _ptr(qw), M, N, K, _ptr(acc), _stream(stream))
+    _call("wq_debug_gemm_s32", _ptr(qx, "qx", _BYTES, M * _codes_per_row(K, act_bits)),
+          act_bits, _ptr(qw, "qw", _BYTES, N * (K // 2)), M, N, K, _ptr(acc, "acc", _I32, M * N),
+          _stream(stream))
 
 
 def wq_device_status():
