@@ -52,7 +52,8 @@ wq_status gemm_checks(const void* qx, const float* s_tok, int act_bits, int M, i
   if (M == 0) return WQ_OK;
   if (!qx || !s_tok || !stream_id || !qw || !s_w || !y) return WQ_ERR_NULL;
   if (!aligned16(qx) || !aligned16(qw) || !aligned16(y) || !aligned16(s_tok) ||
-      !aligned16(s_w) || (bias && !aligned16(bias)) || (beta && !aligned16(beta)))
+      !aligned16(stream_id) || !aligned16(s_w) || (bias && !aligned16(bias)) ||
+      (beta && !aligned16(beta)))
     return WQ_ERR_ALIGN;
   return WQ_OK;
 }
@@ -71,6 +72,7 @@ wq_status linear(const wq_bf16* x, int M, int K, int N, const float* cinv,
   if (M == 0) return WQ_OK;  // empty batch: token tensors may be NULL
   if (!x || !stream_id || !alpha || !qw || !s_w || !y || !workspace) return WQ_ERR_NULL;
   if (!aligned16(x) || !aligned16(qw) || !aligned16(y) || !aligned16(s_w) ||
+      !aligned16(stream_id) || !aligned16(alpha) || (thr && !aligned16(thr)) ||
       (cinv && !aligned16(cinv)) || (bias && !aligned16(bias)) || (beta && !aligned16(beta)) ||
       (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
     return WQ_ERR_ALIGN;
@@ -181,6 +183,7 @@ wq_status wq_channel_scale(const wq_bf16* x_cal, int Mcal, const wq_bf16* W, int
                            float* c, float* cinv, wq_stream_t stream) {
   if (Mcal < 1 || N < 1 || K < 1) return WQ_ERR_SHAPE;
   if (!x_cal || !W || !c || !cinv) return WQ_ERR_NULL;
+  if (!aligned16(x_cal) || !aligned16(W) || !aligned16(c) || !aligned16(cinv)) return WQ_ERR_ALIGN;
   return from_cuda(wq::launch_channel_scale(x_cal, Mcal, W, N, K, c, cinv,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -203,7 +206,9 @@ wq_status wq_act_quant(const wq_bf16* x, int M, int K, const float* cinv,
   WQ_TRY(check_table(S, T, step));
   if (M == 0) return WQ_OK;
   if (!x || !stream_id || !alpha || !qx || !s_tok) return WQ_ERR_NULL;
-  if (!aligned16(x) || !aligned16(qx) || (cinv && !aligned16(cinv))) return WQ_ERR_ALIGN;
+  if (!aligned16(x) || !aligned16(qx) || !aligned16(s_tok) || !aligned16(stream_id) ||
+      !aligned16(alpha) || (cinv && !aligned16(cinv)))
+    return WQ_ERR_ALIGN;
   return from_cuda(wq::launch_act_quant(x, M, K, cinv, stream_id, alpha, S, step, act_bits, qx,
                                         s_tok, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -217,7 +222,9 @@ wq_status wq_act_quant_static(const wq_bf16* x, int M, int K, const float* cinv,
   WQ_TRY(check_table(S, T, step));
   if (M == 0) return WQ_OK;
   if (!x || !stream_id || !thr || !gain || !qx || !s_tok) return WQ_ERR_NULL;
-  if (!aligned16(x) || !aligned16(qx) || (cinv && !aligned16(cinv))) return WQ_ERR_ALIGN;
+  if (!aligned16(x) || !aligned16(qx) || !aligned16(s_tok) || !aligned16(stream_id) ||
+      !aligned16(thr) || !aligned16(gain) || (cinv && !aligned16(cinv)))
+    return WQ_ERR_ALIGN;
   return from_cuda(wq::launch_act_quant_static(x, M, K, cinv, stream_id, thr, gain, S, step,
                                                act_bits, qx, s_tok,
                                                reinterpret_cast<cudaStream_t>(stream)));
@@ -247,6 +254,7 @@ wq_status wq_linear_w4ax_single(const wq_bf16* x, int M, int K, int N, const flo
   if (M == 0) return WQ_OK;
   if (!x || !stream_id || !table || !qw || !s_w || !y) return WQ_ERR_NULL;
   if (!aligned16(x) || !aligned16(qw) || !aligned16(y) || !aligned16(s_w) ||
+      !aligned16(stream_id) || !aligned16(table) || (thr && !aligned16(thr)) ||
       (cinv && !aligned16(cinv)) || (bias && !aligned16(bias)) || (beta && !aligned16(beta)))
     return WQ_ERR_ALIGN;
   const wq::EpilogueArgs ep{nullptr, stream_id, s_w, bias, beta, S, step};

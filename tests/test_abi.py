@@ -125,3 +125,41 @@ def test_single_kernel_linear_rejects_on_host(lib):
     assert lib.wq_linear_w4ax_single(*bad) == 3      # misaligned x
     bad = list(args); bad[1] = 0
     assert lib.wq_linear_w4ax_single(*bad) == 0      # empty batch: nothing to do
+
+
+def test_every_pointer_is_checked_for_alignment(lib):
+    """A table, stream-id or scale pointer off a 16-byte boundary is rejected like the others."""
+    # wq_act_quant(x, M, K, cinv, sid, alpha, S, T, step, bits, qx, s_tok, st)
+    aq = [FAKE, 8, 256, None, FAKE, FAKE, 3, 1, 0, 8, FAKE, FAKE, None]
+    for i in (4, 5, 11):                   # stream_id, alpha, s_tok
+        bad = list(aq); bad[i] = MIS
+        assert lib.wq_act_quant(*bad) == 3, i
+    # wq_act_quant_static(x, M, K, cinv, sid, thr, gain, S, T, step, bits, qx, s_tok, st)
+    st = [FAKE, 8, 256, None, FAKE, FAKE, FAKE, 3, 1, 0, 8, FAKE, FAKE, None]
+    for i in (4, 5, 6, 12):                # stream_id, thr, gain, s_tok
+        bad = list(st); bad[i] = MIS
+        assert lib.wq_act_quant_static(*bad) == 3, i
+    for kw in (dict(sid=MIS), dict(alpha=MIS)):
+        assert _linear(lib, **kw) == 3, kw
+    # wq_linear_w4ax_static: thr (index 6) and gain (index 7)
+    ls = [FAKE, 64, 256, 256, FAKE, FAKE, FAKE, FAKE, FAKE, 3, 1, 0, 8, FAKE, FAKE, FAKE, FAKE,
+          FAKE, 1 << 30, None]
+    for i in (5, 6, 7):
+        bad = list(ls); bad[i] = MIS
+        assert lib.wq_linear_w4ax_static(*bad) == 3, i
+    # wq_linear_w4ax_single: stream_id, table, thr
+    one = [FAKE, 64, 256, 256, FAKE, FAKE, FAKE, FAKE, FAKE, 3, 1, 0, 8, FAKE, FAKE, FAKE, FAKE,
+           None]
+    for i in (5, 6, 7):
+        bad = list(one); bad[i] = MIS
+        assert lib.wq_linear_w4ax_single(*bad) == 3, i
+    # wq_gemm_w4ax(qx, s_tok, bits, M, K, N, sid, beta, S, T, step, qw, s_w, bias, y, st)
+    gm = [FAKE, FAKE, 8, 16, 128, 32, FAKE, None, 3, 1, 0, FAKE, FAKE, None, FAKE, None]
+    for i in (0, 1, 6, 11, 12, 14):
+        bad = list(gm); bad[i] = MIS
+        assert lib.wq_gemm_w4ax(*bad) == 3, i
+    # wq_channel_scale(x_cal, Mcal, W, N, K, c, cinv, st)
+    cs = [FAKE, 4, FAKE, 4, 128, FAKE, FAKE, None]
+    for i in (0, 2, 5, 6):
+        bad = list(cs); bad[i] = MIS
+        assert lib.wq_channel_scale(*bad) == 3, i
