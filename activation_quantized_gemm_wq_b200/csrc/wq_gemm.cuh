@@ -784,7 +784,7 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
   a.q_thr = single ? single->thr : nullptr;
   a.ep = ep;
 
-  static bool attr_set[kAttrDevices] = {};  // per template instance and device
+  static std::atomic<bool> attr_set[kAttrDevices] = {};  // per template instance and device
   const cudaError_t e = set_smem_once(gemm_kernel<C>, C::SMEM_BYTES, attr_set);
   if (e != cudaSuccess) return e;
   const int grid = a.num_units < sm_count() ? a.num_units : sm_count();

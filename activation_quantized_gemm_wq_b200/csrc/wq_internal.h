@@ -2,6 +2,7 @@
 // kernels.  Arguments are assumed validated by the caller.
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
@@ -32,15 +33,17 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t sme
 // to each device's context, so a process that drives several GPUs sets them on
 // each.  `done` is the caller's per-kernel flag array.
 constexpr int kAttrDevices = 64;
+// (The flags are atomic: host threads may launch concurrently; two threads that
+// both find a flag clear just set the same attribute twice.)
 template <class Kernel>
-cudaError_t set_smem_once(Kernel kernel, int bytes, bool (&done)[kAttrDevices]) {
+cudaError_t set_smem_once(Kernel kernel, int bytes, std::atomic<bool> (&done)[kAttrDevices]) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaGetLastError();
   const bool cached = dev >= 0 && dev < kAttrDevices;
-  if (cached && done[dev]) return cudaSuccess;
+  if (cached && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
   const cudaError_t e =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && cached) done[dev] = true;
+  if (e == cudaSuccess && cached) done[dev].store(true, std::memory_order_release);
   return e;
 }
 

@@ -256,17 +256,23 @@ cudaError_t run_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                           cudaStream_t st) {
   constexpr int RPC = 256 / TPR;
   const size_t smem = static_cast<size_t>(K) * sizeof(float);  // cinv copy
-  static bool attr_set[kAttrDevices] = {};  // per template instance and device
-  static int per_sm = 0, per_sm_k = 0;  // resident CTAs per SM at K = per_sm_k
+  static std::atomic<bool> attr_set[kAttrDevices] = {};  // per template instance and device
+  // resident CTAs per SM for the last K seen, packed with that K into one word so
+  // concurrent callers never pair one K with another K's count: (K << 32) | CTAs
+  static std::atomic<uint64_t> occupancy{0};
   // cinv's shared-memory copy: up to kMaxK floats
   const cudaError_t ea = set_smem_once(act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT, STATIC>,
                                        kMaxK * 4, attr_set);
   if (ea != cudaSuccess) return ea;
-  if (per_sm_k != K) {
+  const uint64_t occ = occupancy.load(std::memory_order_relaxed);
+  int per_sm = static_cast<int>(occ & 0xFFFFFFFFu);
+  if (static_cast<int>(occ >> 32) != K) {
+    per_sm = 0;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(
         &per_sm, act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT, STATIC>, 256, smem);
     if (per_sm < 1) per_sm = 1;
-    per_sm_k = K;
+    occupancy.store((static_cast<uint64_t>(K) << 32) | static_cast<uint32_t>(per_sm),
+                    std::memory_order_relaxed);
   }
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
@@ -377,12 +383,12 @@ cudaError_t run_act_quant_rows(const uint16_t* x, int M, int K, const float* cin
                                const uint8_t* sid, const float* alpha, const float* thr, int S,
                                int step, void* qx, float* s_tok, uint4* zero, size_t zero_n16,
                                cudaStream_t st) {
-  static int per_sm = 0;  // per template instance
-  if (per_sm == 0) {
+  static const int per_sm = [] {  // per template instance; thread-safe initialisation
+    int n = 0;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-        &per_sm, act_quant_row_kernel<ACT_BITS, STORE_BITS, STATIC>, 256, 0);
-    if (per_sm < 1) per_sm = 1;
-  }
+        &n, act_quant_row_kernel<ACT_BITS, STORE_BITS, STATIC>, 256, 0);
+    return n < 1 ? 1 : n;
+  }();
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
