@@ -36,6 +36,7 @@ import numpy as np  # noqa: E402
 from activation_quantized_gemm_wq_b200 import synth as S  # noqa: E402
 
 METRIC = "fused W4A8/W4A4 linear TOPS (and GB/s at small M) vs roofline; vs oracle"
+DATA = "synthetic (seeded; stream-structured token rows, outlier channels)"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
@@ -219,6 +220,32 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ the GPU path
 
+def activation_sets(wl):
+    """(bytes of activations + packed weights per step, rotating activation sets): at
+    least two sets, and enough that the sets together exceed twice the L2, so every
+    step reads its inputs from HBM."""
+    in_bytes = sum(l.K * wl.M * 2 + l.N * l.K // 2 for l in wl.linears)
+    n_sets = 2 if in_bytes > L2_BYTES else max(2, -(-2 * L2_BYTES // in_bytes))
+    return in_bytes, n_sets
+
+
+def workload_config(wl, world):
+    """The `config` object of the JSON line, the same for the GPU and reference arms."""
+    in_bytes, n_sets = activation_sets(wl)
+    return {
+        "workload": wl.name,
+        "linears": [f"{l.name} {l.K}->{l.N}" for l in wl.linears],
+        "M": wl.M,
+        "token_rows": {"video": dict(wl.rows).get(0, 0), "proprio": dict(wl.rows).get(1, 0),
+                       "action": dict(wl.rows).get(2, 0)},
+        "act_bits": wl.act_bits,
+        "denoising_steps_in_table": wl.T,
+        "l2": f"inputs larger than L2: {in_bytes / 2**20:.0f} MiB of activations+weights "
+              f"per step, {n_sets} rotating activation sets",
+        "parallelism": f"replicas x{world}",
+    }
+
+
 class Layer:
     """Device-resident inputs of one linear: packed weights, tables, activations."""
 
@@ -263,8 +290,7 @@ def run_gpu(args, rank, world, local):
         a = np.ascontiguousarray(a)
         return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
 
-    in_bytes = sum(l.K * wl.M * 2 + l.N * l.K // 2 for l in wl.linears)
-    n_sets = 2 if in_bytes > L2_BYTES else max(2, -(-2 * L2_BYTES // in_bytes))
+    _, n_sets = activation_sets(wl)
     layers = [Layer(wl, i, n_sets, wq, torch, dev) for i in range(len(wl.linears))]
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
@@ -375,19 +401,8 @@ def run_gpu(args, rank, world, local):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "int8",
-        "data": "synthetic (seeded; stream-structured token rows, outlier channels)",
-        "config": {
-            "workload": wl.name,
-            "linears": [f"{l.name} {l.K}->{l.N}" for l in wl.linears],
-            "M": wl.M,
-            "token_rows": {"video": dict(wl.rows).get(0, 0), "proprio": dict(wl.rows).get(1, 0),
-                           "action": dict(wl.rows).get(2, 0)},
-            "act_bits": wl.act_bits,
-            "denoising_steps_in_table": T,
-            "l2": f"inputs larger than L2: {in_bytes / 2**20:.0f} MiB of activations+weights "
-                  f"per step, {n_sets} rotating activation sets",
-            "parallelism": f"replicas x{world}",
-        },
+        "data": DATA,
+        "config": workload_config(wl, world),
         "roofline": {
             "bound": "tensor",
             "kernel": "gemm_kernel (tcgen05 kind::i8)",
@@ -577,9 +592,8 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-        "data": "synthetic (seeded)",
-        "config": {"workload": wl.name, "M": wl.M, "act_bits": wl.act_bits,
-                   "linears": [f"{l.name} {l.K}->{l.N}" for l in wl.linears]},
+        "data": DATA,
+        "config": workload_config(wl, world),
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle",
                          "sample": f"each step: oracle_linear on {rows} of {wl.M} token rows "
                                    f"of every linear, rows split over {cores} host threads "
