@@ -42,6 +42,10 @@ def _bind(lib):
     lib.oracle_epilogue.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
     lib.oracle_linear.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P,
                                   _P, _P, _P, _P, _P]
+    lib.oracle_gelu.argtypes = [ctypes.c_double]
+    lib.oracle_gelu.restype = ctypes.c_double
+    lib.oracle_gelu_bf16.argtypes = [_P, ctypes.c_size_t, _P]
+    lib.oracle_gelu_bf16.restype = _I
     lib.oracle_bf16_to_float.argtypes = [ctypes.c_uint16]
     lib.oracle_bf16_to_float.restype = ctypes.c_float
     lib.oracle_double_to_bf16.argtypes = [ctypes.c_double]
@@ -191,6 +195,32 @@ class Oracle:
                                       _ptr(bias), _ptr(y), _ptr(qx), _ptr(s_tok), _ptr(acc)),
                "linear")
         return y, qx, s_tok, acc
+
+
+    def gelu(self, v):
+        """GELU(v) in fp64 (App. D keeps GELU in BF16; exact erf form)."""
+        return float(self.lib.oracle_gelu(float(v)))
+
+    def gelu_bf16(self, v):
+        """bf16(GELU(v)) elementwise for raw bf16 patterns v, one rounding."""
+        v = _c(v, np.uint16)
+        h = np.empty_like(v)
+        _check(self.lib.oracle_gelu_bf16(_ptr(v), v.size, _ptr(h)), "gelu_bf16")
+        return h
+
+    def linear_gelu_quant_static(self, x, cinv, stream_id, alpha, beta, step, act_bits, qw,
+                                 s_w, bias, cinv_next, thr_next, gain_next, act_bits_next):
+        """An FFN up-projection whose output is quantized for the down-projection:
+        y = the fused linear (bf16, App. D keeps the linear's output in BF16),
+        h = bf16(GELU(y)), then h quantized as the next linear's activation with its
+        channel scale cinv_next and static clipping (thr_next [T], gain_next [T][S]:
+        one shared threshold per step, a gain per stream; no row maximum, so each
+        code depends only on its own element).  Returns (codes, s_next, h, y)."""
+        y = self.linear(x, cinv, stream_id, alpha, beta, step, act_bits, qw, s_w, bias)[0]
+        h = self.gelu_bf16(y)
+        codes, s_next = self.act_quant_static(h, cinv_next, stream_id, thr_next, gain_next,
+                                              step, act_bits_next)
+        return codes, s_next, h, y
 
 
 def bf16_bits_to_f32(bits):

@@ -290,3 +290,17 @@ int oracle_linear(const uint16_t* x, int M, int K, int N, const float* cinv,
   if (!acc_out) free(acc);
   return rc;
 }
+
+/* App. D (GELU in BF16): GELU(v) = v * Phi(v) with Phi(v) = 0.5 * erfc(-v / sqrt(2)),
+ * in fp64; the bf16 result is rounded once from that value. */
+double oracle_gelu(double v) { return v * 0.5 * erfc(-v / sqrt(2.0)); }
+
+int oracle_gelu_bf16(const uint16_t* v, size_t n, uint16_t* h) {
+  if (n > 0 && (!v || !h)) return ORACLE_EBADARG;
+  for (size_t i = 0; i < n; ++i) {
+    double a = (double)oracle_bf16_to_float(v[i]);
+    if (!isfinite(a)) return ORACLE_ENONFINITE;
+    h[i] = oracle_double_to_bf16(oracle_gelu(a));
+  }
+  return 0;
+}

@@ -42,6 +42,7 @@
 #ifndef WQ_ORACLE_H
 #define WQ_ORACLE_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -91,6 +92,16 @@ int oracle_linear(const uint16_t* x, int M, int K, int N, const float* cinv,
                   int S, int T, int step, int act_bits, const uint8_t* qw,
                   const float* s_w, const float* bias, uint16_t* y, void* qx_out,
                   float* s_tok_out, int32_t* acc_out);
+
+/* App. D keeps GELU in BF16 between the FFN up- and down-projections; fusing the
+ * down-projection's activation quantization into the up-projection's epilogue is
+ * an extension of the pages' two-kernel split.  GELU is read as the exact form
+ * GELU(v) = v * Phi(v), Phi the standard normal distribution function, evaluated
+ * in fp64 as v * 0.5 * erfc(-v / sqrt(2)) (erfc keeps Phi accurate for negative v).
+ * oracle_gelu_bf16: h[i] = bf16(GELU(v[i])) for bf16 inputs v [n], one rounding
+ * (half to even).  Non-finite inputs are rejected. */
+double oracle_gelu(double v);
+int oracle_gelu_bf16(const uint16_t* v, size_t n, uint16_t* h);
 
 /* Helpers exposed for the pin tests. */
 float oracle_bf16_to_float(uint16_t b);

@@ -21,7 +21,12 @@ What pins what:
   static_vs_dynamic static clipping with gain 1 and threshold alpha*amax of the row
                     gives exactly the dynamic codes and scale (the dynamic path is
                     pinned by the checks above)
+  gelu_quadrature   GELU(v) = v * Phi(v) with Phi integrated numerically from the
+                    normal density (no erf or erfc), and its bf16 rounding done here
+  gelu_odd_part     GELU(v) - GELU(-v) = v, since Phi(v) + Phi(-v) = 1
 """
+import math
+
 import numpy as np
 
 from activation_quantized_gemm_wq_b200.synth import f32_to_bf16_bits
@@ -104,6 +109,42 @@ def golden_act_quant_static(orc, golden):
         if not np.array_equal(f32_bits(s), f32_bits(case["s_tok"])):
             fails.append(f"act_quant_static/{case['name']}: s_tok {s.tolist()} != "
                          f"{case['s_tok']}")
+    return fails
+
+
+def golden_gelu(orc, golden):
+    fails = []
+    for case in golden["gelu_bf16"]:
+        h = orc.gelu_bf16(bf16_from_values(case["v"]))
+        if h.tolist() != case["h_bits"]:
+            fails.append(f"gelu_bf16/{case['name']}: {[hex(b) for b in h.tolist()]}")
+    return fails
+
+
+def golden_linear_gelu_quant_static(orc, golden):
+    fails = []
+    for case in golden["linear_gelu_quant_static"]:
+        w = np.asarray(case["w"], np.float32)
+        s_w = np.abs(w) / np.float32(7.0)  # binary32 quotients |w|/7
+        sid = np.asarray(case["stream_id"], np.uint8)
+        thr = np.asarray(case["thr_next"], np.float32)
+        gain = np.asarray(case["gain_next"], np.float32)
+        codes, s_next, h, y = orc.linear_gelu_quant_static(
+            bf16_from_values(case["x"]), None, sid, np.asarray(case["alpha"], np.float32), None,
+            case["step"], case["act_bits"], np.asarray(case["qw_packed"], np.uint8), s_w, None,
+            np.asarray(case["cinv_next"], np.float32), thr, gain, case["act_bits_next"])
+        name = f"linear_gelu_quant_static/{case['name']}"
+        if not np.array_equal(y, bf16_from_values(case["y"])):
+            fails.append(f"{name}: y {bf16_to_f32(y).tolist()}")
+        if h.tolist() != case["h_bits"]:
+            fails.append(f"{name}: h {[[hex(b) for b in r] for r in h.tolist()]}")
+        if not np.array_equal(codes.astype(np.int16), np.asarray(case["codes"])):
+            fails.append(f"{name}: codes {codes.tolist()}")
+        qmax = np.float32(127.0 if case["act_bits_next"] == 8 else 7.0)
+        step = case["step"]
+        want = [(thr[step] / gain[step, g]) / qmax for g in sid]  # binary32 operations
+        if not np.array_equal(f32_bits(s_next), f32_bits(want)):
+            fails.append(f"{name}: scales {s_next.tolist()}")
     return fails
 
 
@@ -404,11 +445,75 @@ def static_vs_dynamic(orc, seeds=(13,)):
     return fails
 
 
-ALL_CHECKS = (golden_act_quant, golden_pack, golden_channel_scale, golden_linear,
-              golden_bf16_rounding, golden_act_quant_static, brute_codes, gemm_vs_matmul,
-              epilogue_fp64, textbook, on_grid, requant, scale_invariance, near_ties,
-              static_vs_dynamic)
-GOLDEN_CHECKS = ALL_CHECKS[:6]
+def _phi_by_quadrature(v):
+    """Standard normal distribution function by numerical integration of the density
+    (the left tail integrated from -inf directly, so no cancellation)."""
+    from scipy.integrate import quad
+
+    def density(t):
+        return math.exp(-0.5 * t * t) / math.sqrt(2.0 * math.pi)
+    if v >= 0.0:
+        return 0.5 + quad(density, 0.0, v, epsabs=0.0, epsrel=1e-13, limit=200)[0]
+    return quad(density, -math.inf, v, epsabs=0.0, epsrel=1e-13, limit=200)[0]
+
+
+def _nearest_bf16_bits(g):
+    """bf16 pattern nearest to the double g (nonzero, normal range), or None when g
+    lies within 1e-6 of a quantum of a rounding tie (then the check skips it)."""
+    e = math.floor(math.log2(abs(g)))
+    r = abs(g) / 2.0 ** (e - 7)  # in [128, 256)
+    if abs(r - math.floor(r) - 0.5) < 1e-6:
+        return None
+    n = int(math.floor(r + 0.5))
+    if n == 256:
+        n, e = 128, e + 1
+    return (0x8000 if g < 0 else 0) | ((e + 127) << 7) | (n - 128)
+
+
+def gelu_quadrature(orc, seed=14):
+    """GELU(v) against v * Phi(v), Phi from quadrature, on a grid of eighths in
+    [-8, 8] and random bf16 values with |v| in [2^-10, 8]; the oracle's bf16 results
+    against that value rounded to nearest bf16 here."""
+    g = np.random.default_rng(seed)
+    grid = np.arange(-64, 65) / 8.0
+    mags = 2.0 ** g.uniform(-10, 3, 600)
+    rand = bf16_to_f32(f32_to_bf16_bits((mags * g.choice([-1.0, 1.0], 600)).astype(np.float32)))
+    vs = np.concatenate([grid, rand.astype(np.float64)])
+    fails = []
+    h = orc.gelu_bf16(f32_to_bf16_bits(vs.astype(np.float32)))
+    for v, hb in zip(vs.tolist(), h.tolist()):
+        ref = v * _phi_by_quadrature(v)
+        got = orc.gelu(v)
+        if abs(got - ref) > 1e-12 * abs(ref):
+            fails.append(f"gelu({v}) = {got}, quadrature {ref}")
+        elif ref != 0.0:
+            want = _nearest_bf16_bits(ref)
+            if want is not None and hb != want:
+                fails.append(f"bf16 gelu({v}) = {hex(hb)}, nearest to {ref} is {hex(want)}")
+        if len(fails) > 5:
+            break
+    return fails
+
+
+def gelu_odd_part(orc, seed=15):
+    """GELU(v) - GELU(-v) = v (Phi(v) + Phi(-v) = 1), to a few fp64 roundings."""
+    g = np.random.default_rng(seed)
+    fails = []
+    for v in g.uniform(-8.0, 8.0, 400).tolist():
+        d = orc.gelu(v) - orc.gelu(-v)
+        if abs(d - v) > 4e-16 * max(abs(v), 1.0):
+            fails.append(f"gelu({v}) - gelu({-v}) = {d}")
+            break
+    return fails
+
+
+GOLDEN_CHECKS = (golden_act_quant, golden_pack, golden_channel_scale, golden_linear,
+                 golden_bf16_rounding, golden_act_quant_static, golden_gelu,
+                 golden_linear_gelu_quant_static)
+PROPERTY_CHECKS = (brute_codes, gemm_vs_matmul, epilogue_fp64, textbook, on_grid, requant,
+                   scale_invariance, near_ties, static_vs_dynamic, gelu_quadrature,
+                   gelu_odd_part)
+ALL_CHECKS = GOLDEN_CHECKS + PROPERTY_CHECKS
 
 
 def all_failures(orc, golden):

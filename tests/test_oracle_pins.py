@@ -75,6 +75,14 @@ MUTANTS = [
     ("static threshold of step 0 for every step",
      [("float clip = g > 0.0f ? thr[step] / g : 0.0f;",
        "float clip = g > 0.0f ? thr[0] / g : 0.0f;")]),
+    ("GELU distribution function at the wrong scale",
+     [("erfc(-v / sqrt(2.0))", "erfc(-v / 2.0)")]),
+    ("GELU with the upper tail 1 - Phi", [("erfc(-v / sqrt(2.0))", "erfc(v / sqrt(2.0))")]),
+    ("GELU without the one half", [("v * 0.5 * erfc", "v * erfc")]),
+    ("GELU as v * erf without the leading one",
+     [("return v * 0.5 * erfc(-v / sqrt(2.0));", "return v * 0.5 * erf(v / sqrt(2.0));")]),
+    ("GELU skipped before the bf16 rounding",
+     [("h[i] = oracle_double_to_bf16(oracle_gelu(a));", "h[i] = oracle_double_to_bf16(a);")]),
 ]
 
 
