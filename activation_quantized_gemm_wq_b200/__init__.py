@@ -47,7 +47,12 @@ _SIGS = {
                                    _P, _P, _P, ctypes.c_size_t, _P]),
     "wq_linear_w4ax_single": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P,
                                    _P, _P, _P]),
-    "wq_debug_gemm_s32": (_I, [_P, _I, _P, _I, _I, _I, _P, _P]),
+    "wq_debug_gemm_s32": (_I, [_P, _I, _P, _I, _I, _I, _P, _P, ctypes.c_size_t, _P]),
+    "wq_debug_linear_s32": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P,
+                                 _P, _P, _P, ctypes.c_size_t, _P]),
+    "wq_linear_gelu_quant": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P,
+                                  _P, _P, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "wq_debug_inject_stall": (_I, [_I, ctypes.c_uint]),
     "wq_device_status": (_I, [ctypes.POINTER(ctypes.c_uint)]),
 }
 
@@ -244,11 +249,51 @@ def wq_linear_w4a8_noalloc(x, cinv, stream_id, alpha, beta, step, qw, s_w, bias,
           a["bias"], a["y"], _stream(stream))
 
 
-def wq_debug_gemm_s32(qx, act_bits, qw, K, acc, stream=None):
+def wq_debug_gemm_s32(qx, act_bits, qw, K, acc, workspace=None, stream=None):
+    """The product GEMM's int32 accumulators on codes qx.  workspace: as for the
+    fused linear (wq_workspace_bytes); only needed when K is split (few tokens)."""
     M, N = acc.shape
     _call("wq_debug_gemm_s32", _ptr(qx, "qx", _BYTES, M * _codes_per_row(K, act_bits)),
           act_bits, _ptr(qw, "qw", _BYTES, N * (K // 2)), M, N, K, _ptr(acc, "acc", _I32, M * N),
+          _ptr(workspace, "workspace"), 0 if workspace is None else _nbytes(workspace),
           _stream(stream))
+
+
+def wq_debug_linear_s32(x, cinv, stream_id, alpha, beta, step, act_bits, qw, s_w, bias, y, acc,
+                        workspace, stream=None):
+    """wq_linear_w4a8 / w4a4 (by act_bits) with the int32 accumulators also written."""
+    T, S = alpha.shape
+    a = _token_and_weight_args(x, cinv, stream_id, beta, S, T, qw, s_w, bias, y)
+    _call("wq_debug_linear_s32", a["x"], a["M"], a["K"], a["N"], a["cinv"], a["sid"],
+          _ptr(alpha, "alpha", _F32, T * S), a["beta"], S, T, step, act_bits, a["qw"], a["s_w"],
+          a["bias"], a["y"], _ptr(acc, "acc", _I32, a["M"] * a["N"]),
+          _ptr(workspace, "workspace"), _nbytes(workspace), _stream(stream))
+
+
+def wq_linear_gelu_quant(x, cinv, stream_id, alpha, beta, step, act_bits, qw, s_w, bias,
+                         cinv_next, thr_next, gain_next, act_bits_next, codes_next, s_next, h,
+                         workspace, stream=None):
+    """FFN up-projection whose epilogue writes the down-projection's codes:
+    codes_next int8 [M][N] and s_next [M] (static clipping thr_next [T], gain_next
+    [T][S]); h [M][N] bf16 (debug copy of bf16(GELU(y))) may be None."""
+    T, S = alpha.shape
+    M, K = x.shape
+    N = qw.shape[0]
+    _call("wq_linear_gelu_quant", _ptr(x, "x", _BF16, M * K), M, K, N,
+          _ptr(cinv, "cinv", _F32, K), _ptr(stream_id, "stream_id", _BYTES, M),
+          _ptr(alpha, "alpha", _F32, T * S), _ptr(beta, "beta", _F32, T * S * N), S, T, step,
+          act_bits, _ptr(qw, "qw", _BYTES, N * (K // 2)), _ptr(s_w, "s_w", _F32, N),
+          _ptr(bias, "bias", _F32, N), _ptr(cinv_next, "cinv_next", _F32, N),
+          _ptr(thr_next, "thr_next", _F32, T), _ptr(gain_next, "gain_next", _F32, T * S),
+          act_bits_next, _ptr(codes_next, "codes_next", _BYTES, M * N),
+          _ptr(s_next, "s_next", _F32, M), _ptr(h, "h", _BF16, M * N),
+          _ptr(workspace, "workspace"), _nbytes(workspace), _stream(stream))
+
+
+def wq_debug_inject_stall(enable, limit_us=0):
+    """Test hook: make every later GEMM launch stall on its first stage and give up
+    after limit_us (enable=True), or restore the defaults (enable=False)."""
+    _call("wq_debug_inject_stall", 1 if enable else 0, int(limit_us))
 
 
 def wq_device_status():

@@ -58,61 +58,95 @@ wq_status gemm_checks(const void* qx, const float* s_tok, int act_bits, int M, i
   return WQ_OK;
 }
 
-// alpha: the clip ratios [T][S] (dynamic clipping), or, when thr is not NULL, the
-// stream gains [T][S] of static clipping with thresholds thr [T].
-wq_status linear(const wq_bf16* x, int M, int K, int N, const float* cinv,
-                 const uint8_t* stream_id, const float* alpha, const float* beta, int S, int T,
-                 int step, const uint8_t* qw, const float* s_w, const float* bias, wq_bf16* y,
-                 void* workspace, size_t ws_bytes, wq_stream_t stream, int act_bits,
-                 const float* thr = nullptr) {
+// The workspace of a fused linear: codes | token scales | split-K partial tiles |
+// split-K counters.  The codes are stored one per int8 byte for both widths: the
+// tensor cores take int8 operands, so int4 activation codes in bytes feed the int8
+// mainloop directly instead of being unpacked again for every weight tile.
+struct Workspace {
+  void* qx;
+  float* s_tok;
+  wq::SplitScratch scratch;  // partial == nullptr: K is not split
+  void* zero;                // the split-K scratch, cleared by the quantizer's launch
+  size_t zero_bytes;
+};
+
+Workspace carve(void* workspace, int M, int K, int N) {
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  Workspace w{};
+  w.qx = ws;
+  const size_t off_stok = round_up(act_bytes(M, K, 8));
+  w.s_tok = reinterpret_cast<float*>(ws + off_stok);
+  const size_t off_part = off_stok + round_up(sizeof(float) * static_cast<size_t>(M));
+  if (wq::gemm_splits(M, N, K) > 1) {
+    const int BN = wq::bn_for(M);
+    const size_t tiles = static_cast<size_t>((M + BN - 1) / BN) * ((N + 127) / 128);
+    const size_t part_bytes = round_up(tiles * BN * 128 * sizeof(int32_t));
+    w.scratch.partial = reinterpret_cast<int32_t*>(ws + off_part);
+    w.scratch.counters = reinterpret_cast<int*>(ws + off_part + part_bytes);
+    w.zero = ws + off_part;
+    w.zero_bytes = wq::gemm_split_scratch_bytes(M, N, K);
+  }
+  return w;
+}
+
+// Host-side checks shared by the fused linears.
+wq_status linear_checks(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                        const uint8_t* stream_id, const float* alpha, const float* beta, int S,
+                        int T, int step, const uint8_t* qw, const float* s_w, const float* bias,
+                        const void* out, void* workspace, size_t ws_bytes, int act_bits,
+                        const float* thr) {
   if (act_bits != 8 && act_bits != 4) return WQ_ERR_ARG;
   WQ_TRY(check_mk(M, K));
   WQ_TRY(check_n(N));
   WQ_TRY(check_table(S, T, step));
   if (M == 0) return WQ_OK;  // empty batch: token tensors may be NULL
-  if (!x || !stream_id || !alpha || !qw || !s_w || !y || !workspace) return WQ_ERR_NULL;
-  if (!aligned16(x) || !aligned16(qw) || !aligned16(y) || !aligned16(s_w) ||
+  if (!x || !stream_id || !alpha || !qw || !s_w || !out || !workspace) return WQ_ERR_NULL;
+  if (!aligned16(x) || !aligned16(qw) || !aligned16(out) || !aligned16(s_w) ||
       !aligned16(stream_id) || !aligned16(alpha) || (thr && !aligned16(thr)) ||
       (cinv && !aligned16(cinv)) || (bias && !aligned16(bias)) || (beta && !aligned16(beta)) ||
       (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
     return WQ_ERR_ALIGN;
   if (ws_bytes < wq_workspace_bytes(M, K, N, act_bits)) return WQ_ERR_ARG;
-  // workspace: codes | token scales | split-K partial tiles | split-K counters.
-  // The codes are stored one per int8 byte for both widths: the tensor cores
-  // take int8 operands, so int4 activation codes in bytes feed the int8
-  // mainloop directly instead of being unpacked again for every weight tile.
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  void* qx = ws;
-  const size_t off_stok = round_up(act_bytes(M, K, 8));
-  float* s_tok = reinterpret_cast<float*>(ws + off_stok);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  wq::SplitScratch scratch{nullptr, nullptr};
-  const int splits = wq::gemm_splits(M, N, K);
-  const size_t off_part = off_stok + round_up(sizeof(float) * static_cast<size_t>(M));
-  const size_t split_bytes = wq::gemm_split_scratch_bytes(M, N, K);
-  if (splits > 1) {
-    const int BN = wq::bn_for(M);
-    const size_t tiles = static_cast<size_t>((M + BN - 1) / BN) * ((N + 127) / 128);
-    const size_t part_bytes = round_up(tiles * BN * 128 * sizeof(int32_t));
-    scratch.partial = reinterpret_cast<int32_t*>(ws + off_part);
-    scratch.counters = reinterpret_cast<int*>(ws + off_part + part_bytes);
-  }
-  // the quantizer also clears the split-K accumulators and counters
-  void* zero = splits > 1 ? ws + off_part : nullptr;
-  const size_t zero_bytes = splits > 1 ? split_bytes : 0;
+  return WQ_OK;
+}
+
+// The first kernel of a fused linear: codes and token scales into the workspace
+// (and the split-K scratch cleared).  alpha: the clip ratios [T][S] (dynamic
+// clipping), or, when thr is not NULL, the stream gains [T][S] of static clipping
+// with thresholds thr [T].
+wq_status quantize_into(const Workspace& w, const wq_bf16* x, int M, int K, const float* cinv,
+                        const uint8_t* stream_id, const float* alpha, int S, int step,
+                        int act_bits, const float* thr, cudaStream_t st) {
   if (thr)
-    WQ_TRY(from_cuda(wq::launch_act_quant_static(x, M, K, cinv, stream_id, thr, alpha, S, step,
-                                                 act_bits, qx, s_tok, st, zero, zero_bytes,
-                                                 /*bytes_per_code=*/true)));
-  else
-    WQ_TRY(from_cuda(wq::launch_act_quant(x, M, K, cinv, stream_id, alpha, S, step, act_bits, qx,
-                                          s_tok, st, zero, zero_bytes, /*bytes_per_code=*/true)));
-  const wq::EpilogueArgs ep{s_tok, stream_id, s_w, bias, beta, S, step};
+    return from_cuda(wq::launch_act_quant_static(x, M, K, cinv, stream_id, thr, alpha, S, step,
+                                                 act_bits, w.qx, w.s_tok, st, w.zero,
+                                                 w.zero_bytes, /*bytes_per_code=*/true));
+  return from_cuda(wq::launch_act_quant(x, M, K, cinv, stream_id, alpha, S, step, act_bits,
+                                        w.qx, w.s_tok, st, w.zero, w.zero_bytes,
+                                        /*bytes_per_code=*/true));
+}
+
+wq_status linear(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                 const uint8_t* stream_id, const float* alpha, const float* beta, int S, int T,
+                 int step, const uint8_t* qw, const float* s_w, const float* bias, wq_bf16* y,
+                 void* workspace, size_t ws_bytes, wq_stream_t stream, int act_bits,
+                 const float* thr = nullptr, int32_t* acc_out = nullptr) {
+  WQ_TRY(linear_checks(x, M, K, N, cinv, stream_id, alpha, beta, S, T, step, qw, s_w, bias, y,
+                       workspace, ws_bytes, act_bits, thr));
+  if (M == 0) return WQ_OK;
+  if (acc_out && !aligned16(acc_out)) return WQ_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Workspace w = carve(workspace, M, K, N);
+  WQ_TRY(quantize_into(w, x, M, K, cinv, stream_id, alpha, S, step, act_bits, thr, st));
+  const wq::EpilogueArgs ep{w.s_tok, stream_id, s_w, bias, beta, S, step};
+  wq::GemmExtras ex;
+  ex.acc_out = acc_out;
   // weights may stream while the quantizer runs (it started the GEMM only after
-  // everything before it in the stream had finished)
-  // int8-stored codes: the int8-activation mainloop (the int32 sums are the same)
-  return from_cuda(wq::launch_gemm(qx, 8, qw, M, N, K, ep, y, false,
-                                   splits > 1 ? &scratch : nullptr, st, /*w_prefetch=*/true));
+  // everything before it in the stream had finished); int8-stored codes: the
+  // int8-activation mainloop (the int32 sums are the same)
+  return from_cuda(wq::launch_gemm(w.qx, 8, qw, M, N, K, ep, y,
+                                   w.scratch.partial ? &w.scratch : nullptr, st,
+                                   /*w_prefetch=*/true, acc_out ? &ex : nullptr));
 }
 
 // ------------------------------------------------------------ no-alloc variant
@@ -269,7 +303,7 @@ wq_status wq_gemm_w4ax(const void* qx, const float* s_tok, int act_bits, int M, 
   WQ_TRY(gemm_checks(qx, s_tok, act_bits, M, K, N, stream_id, beta, S, T, step, qw, s_w, bias,
                      y));
   const wq::EpilogueArgs ep{s_tok, stream_id, s_w, bias, beta, S, step};
-  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, y, false, nullptr,
+  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, y, nullptr,
                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -292,18 +326,85 @@ wq_status wq_linear_w4a4(const wq_bf16* x, int M, int K, int N, const float* cin
 }
 
 wq_status wq_debug_gemm_s32(const void* qx, int act_bits, const uint8_t* qw, int M, int N,
-                            int K, int32_t* acc, wq_stream_t stream) {
+                            int K, int32_t* acc, void* workspace, size_t ws_bytes,
+                            wq_stream_t stream) {
   if (act_bits != 8 && act_bits != 4) return WQ_ERR_ARG;
   WQ_TRY(check_mk(M, K));
   WQ_TRY(check_n(N));
   if (M == 0) return WQ_OK;
   if (!qx || !qw || !acc) return WQ_ERR_NULL;
   if (!aligned16(qx) || !aligned16(qw) || !aligned16(acc)) return WQ_ERR_ALIGN;
-  const wq::EpilogueArgs ep{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 0};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (wq::gemm_splits(M, N, K) > 1)  // the K splits add into the output
-    WQ_TRY(from_cuda(cudaMemsetAsync(acc, 0, sizeof(int32_t) * static_cast<size_t>(M) * N, st)));
-  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, acc, true, nullptr, st));
+  const wq::EpilogueArgs ep{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 0};
+  wq::GemmExtras ex;
+  ex.acc_out = acc;
+  const size_t split_bytes = wq::gemm_split_scratch_bytes(M, N, K);
+  wq::SplitScratch sc{nullptr, nullptr};
+  if (split_bytes > 0) {  // the fused linear's split of K, through the caller's scratch
+    if (!workspace) return WQ_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return WQ_ERR_ALIGN;
+    if (ws_bytes < split_bytes) return WQ_ERR_ARG;
+    const int BN = wq::bn_for(M);
+    const size_t tiles = static_cast<size_t>((M + BN - 1) / BN) * ((N + 127) / 128);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    sc.partial = reinterpret_cast<int32_t*>(ws);
+    sc.counters = reinterpret_cast<int*>(ws + round_up(tiles * BN * 128 * sizeof(int32_t)));
+    WQ_TRY(from_cuda(cudaMemsetAsync(workspace, 0, split_bytes, st)));
+  }
+  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, nullptr,
+                                   split_bytes > 0 ? &sc : nullptr, st, false, &ex));
+}
+
+wq_status wq_debug_linear_s32(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                              const uint8_t* stream_id, const float* alpha, const float* beta,
+                              int S, int T, int step, int act_bits, const uint8_t* qw,
+                              const float* s_w, const float* bias, wq_bf16* y, int32_t* acc,
+                              void* workspace, size_t ws_bytes, wq_stream_t stream) {
+  if (M > 0 && !acc) return WQ_ERR_NULL;
+  return linear(x, M, K, N, cinv, stream_id, alpha, beta, S, T, step, qw, s_w, bias, y,
+                workspace, ws_bytes, stream, act_bits, nullptr, acc);
+}
+
+wq_status wq_linear_gelu_quant(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                               const uint8_t* stream_id, const float* alpha, const float* beta,
+                               int S, int T, int step, int act_bits, const uint8_t* qw,
+                               const float* s_w, const float* bias, const float* cinv_next,
+                               const float* thr_next, const float* gain_next, int act_bits_next,
+                               int8_t* codes_next, float* s_next, wq_bf16* h, void* workspace,
+                               size_t ws_bytes, wq_stream_t stream) {
+  if (act_bits_next != 8 && act_bits_next != 4) return WQ_ERR_ARG;
+  WQ_TRY(linear_checks(x, M, K, N, cinv, stream_id, alpha, beta, S, T, step, qw, s_w, bias,
+                       codes_next, workspace, ws_bytes, act_bits, nullptr));
+  if (M == 0) return WQ_OK;
+  if (!thr_next || !gain_next || !s_next) return WQ_ERR_NULL;
+  if (!aligned16(thr_next) || !aligned16(gain_next) || !aligned16(s_next) ||
+      (cinv_next && !aligned16(cinv_next)) || (h && !aligned16(h)))
+    return WQ_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Workspace w = carve(workspace, M, K, N);
+  WQ_TRY(quantize_into(w, x, M, K, cinv, stream_id, alpha, S, step, act_bits, nullptr, st));
+  const wq::EpilogueArgs ep{w.s_tok, stream_id, s_w, bias, beta, S, step};
+  wq::GemmExtras ex;
+  ex.next_thr = thr_next;
+  ex.next_gain = gain_next;
+  ex.next_cinv = cinv_next;
+  ex.next_s = s_next;
+  ex.h = h;
+  return from_cuda(wq::launch_gemm_gelu_quant(w.qx, qw, M, N, K, ep, act_bits_next, codes_next,
+                                              w.scratch.partial ? &w.scratch : nullptr, st,
+                                              /*w_prefetch=*/true, ex));
+}
+
+wq_status wq_debug_inject_stall(int enable, unsigned limit_us) {
+  const int kblock = enable ? 0 : -1;
+  const unsigned long long limit =
+      enable ? static_cast<unsigned long long>(limit_us) * 1000ull : wq::kWaitLimitNs;
+  if (enable && limit_us == 0) return WQ_ERR_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return WQ_ERR_CUDA;
+  if (cudaMemcpyToSymbol(wq::g_wait_limit_ns, &limit, sizeof limit) != cudaSuccess ||
+      cudaMemcpyToSymbol(wq::g_stall_kblock, &kblock, sizeof kblock) != cudaSuccess)
+    return WQ_ERR_CUDA;
+  return cudaDeviceSynchronize() == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
 }
 
 wq_status wq_linear_w4a8_noalloc(const wq_bf16* x, int M, int K, int N, const float* cinv,

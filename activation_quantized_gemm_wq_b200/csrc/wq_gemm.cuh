@@ -16,7 +16,11 @@
 //               activations when they are int4)
 //   epilogue    tcgen05.ld of the accumulator, y = bf16((s_tok*s_w)*acc + bias +
 //   warps       beta[step][stream][n]), staged in shared memory and written with
-//               TMA stores (tails clipped by the tensor map)
+//               TMA stores (tails clipped by the tensor map).  A second instance
+//               (EPI = 8 or 4) continues from y: h = bf16(GELU(y)), then h is
+//               quantized as the NEXT linear's activation (its channel scale and
+//               static clip), and int8 codes are stored instead of y.  Any instance
+//               can also copy the raw int32 accumulators to a debug buffer.
 // The output-channel dimension is the MMA's M ("swap AB"), so the same kernel
 // serves any token count from 1 to the full batch, with token tiles of 16..256.
 //
@@ -51,6 +55,15 @@ struct TileArgs {
   const float* q_alpha;  // clip ratios [T][S]; with q_thr, the stream gains [T][S]
   const float* q_thr;    // static clipping thresholds [T], or null (dynamic)
   EpilogueArgs ep;
+  int has_y;             // 0: no y / codes store (the int32 debug view alone)
+  int32_t* acc_out;      // int32 [M][N] copy of the accumulators (debug), or null
+  // EPI > 0: the next linear's static clipping (thr [T], gain [T][S]), its channel
+  // scale [N] (or null), the codes' scales s_next [M] out, h [M][N] bf16 out or null
+  const float* g_thr;
+  const float* g_gain;
+  const float* g_cinv;
+  float* g_s;
+  uint16_t* g_h;
 };
 
 // K-block range of split `sp` of `splits` (balanced).
@@ -73,15 +86,20 @@ __device__ __forceinline__ void split_range(int num_k, int splits, int sp, int& 
 // token's scale once (its row maximum over all of K) before the first tile; the
 // unpack warps quantize every K block (qmax 127 or 7) straight into the int8
 // tile the MMA reads.  No codes go through HBM.
-template <int BN_, int ACT_BITS_, bool OUT_S32_, int QBITS_ = 0>
+// EPI > 0: the up-projection of an FFN whose epilogue emits the down-projection's
+// activation codes (qmax 127 for EPI 8, 7 for EPI 4) instead of y.
+template <int BN_, int ACT_BITS_, int QBITS_ = 0, int EPI_ = 0>
 struct Cfg {
   static constexpr int BN = BN_;
   static constexpr int ACT_BITS = ACT_BITS_;
-  static constexpr bool OUT_S32 = OUT_S32_;
   static constexpr int QBITS = QBITS_;
   static constexpr int QMAX = QBITS == 4 ? 7 : 127;
-  static_assert(QBITS == 0 || (ACT_BITS == 8 && !OUT_S32 && BN <= 64),
+  static constexpr int EPI = EPI_;
+  static constexpr int QMAX_NEXT = EPI == 4 ? 7 : 127;
+  static_assert(QBITS == 0 || (ACT_BITS == 8 && BN <= 64),
                 "the single-kernel linear quantizes into the int8 mainloop, one token tile");
+  static_assert(EPI == 0 || ((EPI == 8 || EPI == 4) && QBITS == 0 && ACT_BITS == 8),
+                "the GELU-and-quantize epilogue follows the int8-activation mainloop");
   static constexpr int BM = 128;  // output channels per tile (MMA M)
   static constexpr int BK = 128;  // K elements per pipeline stage
   static constexpr int UNPACK_WARPS = ACT_BITS == 4 ? 8 : WQ_UNPACK_WARPS_A8;
@@ -113,15 +131,18 @@ struct Cfg {
   // can queue barely one instruction ahead of the tensor pipe, so its per-block
   // overhead, not the pipeline depth alone, decides whether the pipe stays fed.
   static constexpr int NU = ACT_BITS == 8 ? 3 : 2;
-  static constexpr int EPI_ELEM = OUT_S32 ? 4 : 2;
+  static constexpr int EPI_ELEM = 2;  // bf16 y (the codes of EPI > 0 use half of it)
   // The tensor cores accumulate 16x (int8 activations) or 256x (both operands
   // unpacked from int4) the code products; see unpack32.
   static constexpr int ACC_SHIFT = ACT_BITS == 8 ? 4 : 8;
   static constexpr int EPI_CHUNK = 16;  // token columns per TMEM load / TMA store
   static constexpr int NUM_CHUNKS = BN / EPI_CHUNK;
   static constexpr int EPI_BUF_BYTES = EPI_CHUNK * 32 * EPI_ELEM;
-  // staged s_tok and stream ids, x2; then (QBITS) each token's scale and its reciprocal
-  static constexpr int TOK_BYTES = 2 * BN * 4 + 2 * BN + (QBITS ? 2 * BN * 4 : 0);
+  // staged s_tok and stream ids, x2; then (QBITS) each token's scale and its
+  // reciprocal; then (EPI) the next linear's token scales and reciprocals, x2
+  static constexpr int TOK_BYTES =
+      2 * BN * 4 + 2 * BN + (QBITS ? 2 * BN * 4 : 0) + (EPI ? 2 * 2 * BN * 4 : 0);
+  static constexpr int OFF_TOK_NEXT = 2 * BN * 4 + 2 * BN + (QBITS ? 2 * BN * 4 : 0);
   static constexpr int SMEM_LIMIT = 232448;  // 227 KB opt-in per CTA
   static constexpr int RESERVED = 1024 /*alignment slack*/ + 512 /*barriers*/;
   static constexpr int FIXED = RESERVED + NU * (WU_BYTES + XU_BYTES) + TOK_BYTES;
@@ -143,7 +164,7 @@ struct Cfg {
   static constexpr int OFF_EPI = OFF_XU + NU * XU_BYTES;
   static constexpr int OFF_TOK = OFF_EPI + EPI_BYTES;
   static constexpr int OFF_BAR = OFF_TOK + TOK_BYTES;
-  static constexpr int NUM_BARS = 2 * NS + NU + 7;
+  static constexpr int NUM_BARS = 2 * NS + NU + 8;
   static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
   static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
   static_assert(OFF_XS % 1024 == 0 && XS_BYTES % 512 == 0 && OFF_WU % 1024 == 0 &&
@@ -237,7 +258,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* tokbar = tempty + 2;  // epilogue warps: token staging of buffer i complete
   uint64_t* qready = tokbar + 2;  // QBITS: every token scale of the tile is in shared memory
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qready + 1);
+  uint64_t* mma_drained = qready + 1;  // every MMA this CTA issued has completed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_drained + 1);
   float* q_s = reinterpret_cast<float*>(smem + C::OFF_TOK + 2 * C::BN * 4 + 2 * C::BN);
   float* q_r = q_s + C::BN;
 
@@ -257,6 +279,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_init(&tokbar[b], C::EPI_WARPS);
     }
     mbar_init(qready, C::EPI_WARPS);
+    mbar_init(mma_drained, 1);
     fence_mbar_init();
     fence_proxy_async_smem();
   }
@@ -298,6 +321,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
       }
       griddep_wait();
+      // test hook (normally -1): K block whose activation copy CTA 0 leaves out
+      const int stall = blockIdx.x == 0 ? *reinterpret_cast<volatile int*>(&g_stall_kblock) : -1;
       uint32_t g = 0;
       bool ok = true;
       for (int unit = blockIdx.x; ok && unit < args.num_units; unit += gridDim.x) {
@@ -316,7 +341,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             tma_load_2d(smem + C::OFF_WP + s * C::WP_BYTES, &tm_w, &full[s], kb * (C::BK / 2),
                         n_tile * C::BM);
           }
-          if constexpr (C::QBITS > 0) {  // bf16 x, two boxes of 64 channels
+          if (static_cast<int>(g) == stall) {
+            // leave the stage one copy short: its phase never completes
+          } else if constexpr (C::QBITS > 0) {  // bf16 x, two boxes of 64 channels
             tma_load_2d(smem + C::OFF_XB + s * C::XB_BYTES, &tm_x, &full[s], kb * C::BK,
                         m_tile * C::BN);
             tma_load_2d(smem + C::OFF_XB + s * C::XB_BYTES + C::BN * 128, &tm_x, &full[s],
@@ -328,10 +355,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
       }
       // Drain: the copies of every issued stage must have landed before the CTA
-      // exits (normally all were consumed already and these waits return at once).
+      // exits (normally all were consumed already and these waits return at once;
+      // after an error elsewhere they still wait, bounded, for copies in flight).
+      // The stage the test hook left short never completes and is not waited for.
       for (uint32_t i = 0; i < static_cast<uint32_t>(C::NS) && i < g; ++i) {
         const uint32_t j = g - 1 - i;
-        mbar_wait(&full[j % C::NS], (j / C::NS) & 1u);
+        if (static_cast<int>(j) != stall) mbar_wait_drain(&full[j % C::NS], (j / C::NS) & 1u);
       }
     }
     __syncwarp();
@@ -370,6 +399,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         mma_commit(&tfull[b]);
         if (++b == 2) { b = 0; ph_b ^= 1u; }
       }
+      // Every MMA issued has completed before the TMEM is freed (after an error the
+      // epilogue may not have waited for the last ones).
+      mma_commit(mma_drained);
+      mbar_wait_drain(mma_drained, 0);
     }
     __syncwarp();
   } else if (C::unpack_index(warp) >= 0) {
@@ -515,6 +548,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       __all_sync(0xFFFFFFFFu, mbar_wait(qready, 0));
     }
     const bool split = args.splits > 1;
+    // y (or the next linear's codes) is written unless this is the int32 debug view
+    const bool has_out = args.has_y != 0;
+    float* nxt_s = reinterpret_cast<float*>(smem + C::OFF_TOK + C::OFF_TOK_NEXT);  // EPI
     for (int unit = blockIdx.x; unit < args.num_units; unit += gridDim.x, ++it) {
       const int tile = unit / args.splits;
       int n_tile, m_tile;
@@ -524,76 +560,63 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const int m0 = m_tile * C::BN;
       float* sts = tok_s + (it & 1) * C::BN;
       uint8_t* sds = tok_id + (it & 1) * C::BN;
+      float* g_s = nxt_s + (it & 1) * 2 * C::BN;  // EPI: next scale [BN], reciprocal [BN]
       // per-lane channel constants; bias and the compensation of each stream
-      // combined once per tile
-      float sw = 0.0f, bb[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      if (!C::OUT_S32) {
+      // combined once per tile.  A stream id >= S (a precondition violation the
+      // quantizer reports) gets the bias alone: no table row is read for it.
+      float sw = 0.0f, bs = 0.0f, bb[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      float g_ci = 1.0f;  // EPI: the next linear's channel scale at channel n
+      if (has_out) {
         for (int i = et; i < C::BN; i += C::EPI_THREADS) {
           const int m = m0 + i;
           if constexpr (C::QBITS > 0) sts[i] = q_s[i];  // the single token tile
           else sts[i] = m < args.M ? ep.s_tok[m] : 0.0f;
-          sds[i] = m < args.M ? ep.stream_id[m] : 0;
+          const int sd = m < args.M ? ep.stream_id[m] : 0;
+          sds[i] = static_cast<uint8_t>(sd);
+          if constexpr (C::EPI > 0) {
+            // static clip of the next linear: thr[step] / gain[step][stream]
+            float sn = 0.0f;
+            if (m < args.M && sd < ep.S) {
+              const float gn = __ldg(args.g_gain + ep.step * ep.S + sd);
+              const float clip = gn > 0.0f ? __fdiv_rn(__ldg(args.g_thr + ep.step), gn) : 0.0f;
+              sn = __fdiv_rn(clip, static_cast<float>(C::QMAX_NEXT));
+            }
+            g_s[i] = sn;
+            g_s[C::BN + i] = sn > 0.0f ? __frcp_rn(sn) : 0.0f;
+            if (n_tile == 0 && unit % args.splits == 0 && m < args.M) args.g_s[m] = sn;
+          }
         }
         if (n < args.N) {
           sw = ldexpf(ep.s_w[n], -C::ACC_SHIFT);  // exact power-of-two rescale
-          const float bs = ep.bias ? ep.bias[n] : 0.0f;
+          bs = ep.bias ? ep.bias[n] : 0.0f;
           const float* brow = ep.beta ? ep.beta + (size_t)ep.step * ep.S * args.N + n : nullptr;
 #pragma unroll
           for (int j = 0; j < 4; ++j)
             bb[j] = (brow && j < ep.S && small_s) ? __fadd_rn(bs, brow[(size_t)j * args.N]) : bs;
+          if constexpr (C::EPI > 0) g_ci = args.g_cinv ? args.g_cinv[n] : 1.0f;
         }
       }
 
-      // y for one 16-column chunk of accumulators (scaled by 2^ACC_SHIFT), through a
-      // shared-memory staging buffer and a TMA store; int32 view for OUT_S32.
-      auto emit = [&](const uint32_t (&r)[16], int j0) {
+      // bias + compensation of token stream sd at this lane's channel
+      auto offset = [&](int sd) -> float {
+        if (sd >= ep.S) return bs;
+        if (small_s) return sd == 0 ? bb[0] : sd == 1 ? bb[1] : sd == 2 ? bb[2] : bb[3];
+        return (ep.beta && n < args.N)
+                   ? __fadd_rn(bs, ep.beta[((size_t)ep.step * ep.S + sd) * args.N + n])
+                   : bs;
+      };
+
+      // This chunk's staging buffer, once its previous TMA store has read it.
+      auto stage_buf = [&]() -> uint8_t* {
         uint8_t* sb = ebuf + buf * C::EPI_BUF_BYTES;
-        if (lane == 0) {  // this buffer's previous TMA store has read it
+        if (lane == 0) {
           if constexpr (C::EPI_NBUF == 2) bulk_wait_group_read<1>();
           else bulk_wait_group_read<0>();
         }
         __syncwarp();
-        if constexpr (C::OUT_S32) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)  // exact: the scaled sums are multiples of 2^ACC_SHIFT
-            reinterpret_cast<int32_t*>(sb)[j * 32 + lane] = static_cast<int32_t>(r[j]) >> C::ACC_SHIFT;
-        } else {
-          __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(sb);
-          const float4* st4 = reinterpret_cast<const float4*>(sts + j0);
-          const int sd_l = sds[j0 + (lane & 15)];
-          const int sd0 = sds[j0];
-          if (small_s && __all_sync(0xFFFFFFFFu, sd_l == sd0)) {
-            // one stream in the whole chunk (the common case: streams are runs of rows)
-            const float bsel = sd0 == 0 ? bb[0] : sd0 == 1 ? bb[1] : sd0 == 2 ? bb[2] : bb[3];
-#pragma unroll
-            for (int j4 = 0; j4 < 4; ++j4) {
-              const float4 t = st4[j4];
-              const float tv[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const int j = 4 * j4 + k;
-                const float v =
-                    fmaf(tv[k] * sw, __int2float_rn(static_cast<int>(r[j])), bsel);
-                ob[j * 32 + lane] = __float2bfloat16_rn(v);
-              }
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int sd = sds[j0 + j];
-              float bv;
-              if (small_s) {
-                bv = sd == 0 ? bb[0] : sd == 1 ? bb[1] : sd == 2 ? bb[2] : bb[3];
-              } else {
-                bv = n < args.N ? (ep.bias ? ep.bias[n] : 0.0f) : 0.0f;
-                if (ep.beta && n < args.N)
-                  bv = __fadd_rn(bv, ep.beta[((size_t)ep.step * ep.S + sd) * args.N + n]);
-              }
-              const float v = fmaf(sts[j0 + j] * sw, __int2float_rn(static_cast<int>(r[j])), bv);
-              ob[j * 32 + lane] = __float2bfloat16_rn(v);
-            }
-          }
-        }
+        return sb;
+      };
+      auto store_buf = [&](uint8_t* sb, int j0) {
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && n_base < args.N) {
@@ -601,6 +624,78 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           bulk_commit_group();
         }
         if constexpr (C::EPI_NBUF == 2) buf ^= 1;
+      };
+
+      // y for one 16-column chunk of accumulators (scaled by 2^ACC_SHIFT), through a
+      // shared-memory staging buffer and a TMA store.
+      auto emit_y = [&](const uint32_t (&r)[16], int j0) {
+        uint8_t* sb = stage_buf();
+        __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(sb);
+        const float4* st4 = reinterpret_cast<const float4*>(sts + j0);
+        const int sd_l = sds[j0 + (lane & 15)];
+        const int sd0 = sds[j0];
+        if (small_s && __all_sync(0xFFFFFFFFu, sd_l == sd0)) {
+          // one stream in the whole chunk (the common case: streams are runs of rows)
+          const float bsel = offset(sd0);
+#pragma unroll
+          for (int j4 = 0; j4 < 4; ++j4) {
+            const float4 t = st4[j4];
+            const float tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int j = 4 * j4 + k;
+              const float v = fmaf(tv[k] * sw, __int2float_rn(static_cast<int>(r[j])), bsel);
+              ob[j * 32 + lane] = __float2bfloat16_rn(v);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float v =
+                fmaf(sts[j0 + j] * sw, __int2float_rn(static_cast<int>(r[j])), offset(sds[j0 + j]));
+            ob[j * 32 + lane] = __float2bfloat16_rn(v);
+          }
+        }
+        store_buf(sb, j0);
+      };
+
+      // EPI > 0: y as above, then h = bf16(GELU(y)) and the next linear's code of
+      // h * cinv_next[n] with its static scale, staged as int8 [16 tokens][32
+      // channels] and written with a TMA store; h itself only to the debug buffer.
+      auto emit_codes = [&](const uint32_t (&r)[16], int j0) {
+        uint8_t* sb = stage_buf();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float v =
+              fmaf(sts[j0 + j] * sw, __int2float_rn(static_cast<int>(r[j])), offset(sds[j0 + j]));
+          const float yv = __bfloat162float(__float2bfloat16_rn(v));
+          const __nv_bfloat16 hb = __float2bfloat16_rn(gelu_f32(yv));
+          const int m = m0 + j0 + j;
+          if (args.g_h != nullptr && n < args.N && m < args.M)
+            args.g_h[(size_t)m * args.N + n] = __bfloat16_as_ushort(hb);
+          const float xv = __fmul_rn(__bfloat162float(hb), g_ci);
+          const float sn = g_s[j0 + j], rn = g_s[C::BN + j0 + j];
+          const uint32_t code = (sn > 0.0f && isfinite(rn))
+                                    ? quantize1_recip<C::QMAX_NEXT>(xv, sn, rn)
+                                    : static_cast<uint32_t>(quantize<C::QMAX_NEXT>(xv, sn));
+          sb[j * 32 + lane] = static_cast<uint8_t>(code);
+        }
+        store_buf(sb, j0);
+      };
+
+      // Everything one chunk of finished accumulators produces.
+      auto finish = [&](const uint32_t (&r)[16], int j0) {
+        if (args.acc_out != nullptr && n < args.N) {
+          // int32 debug view: exact, the scaled sums are multiples of 2^ACC_SHIFT
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (m0 + j0 + j < args.M)
+              args.acc_out[(size_t)(m0 + j0 + j) * args.N + n] =
+                  static_cast<int32_t>(r[j]) >> C::ACC_SHIFT;
+        }
+        if (!has_out) return;
+        if constexpr (C::EPI > 0) emit_codes(r, j0);
+        else emit_y(r, j0);
       };
 
       // staging visible to every epilogue warp (and the warps kept within one tile)
@@ -617,9 +712,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * C::BN);
       // split K: the tile's int32 accumulator (2^ACC_SHIFT-scaled), summed by red.add
-      int32_t* tile_acc = split && !C::OUT_S32
-                              ? args.partial + (size_t)tile * C::BN * C::BM + q * 32 + lane
-                              : nullptr;
+      int32_t* tile_acc =
+          split ? args.partial + (size_t)tile * C::BN * C::BM + q * 32 + lane : nullptr;
       for (int c = h; c < C::NUM_CHUNKS; c += 2) {
         const int j0 = c * C::EPI_CHUNK;
         uint32_t r[16];
@@ -632,26 +726,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         if (m0 + j0 >= args.M) continue;  // whole chunk beyond the last token
         if (!split) {
-          emit(r, j0);
-        } else if constexpr (C::OUT_S32) {
-          // int32 view: the splits add into the zeroed output (exact in any order)
-          if (n < args.N) {
-            int32_t* col = static_cast<int32_t*>(args.out) + n;
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (m0 + j0 + j < args.M)
-                atomicAdd(col + (size_t)(m0 + j0 + j) * args.N,
-                          static_cast<int32_t>(r[j]) >> C::ACC_SHIFT);
-          }
+          finish(r, j0);
         } else {
 #pragma unroll
           for (int j = 0; j < 16; ++j)  // exact in any order; no return value needed
             atomicAdd(tile_acc + (j0 + j) * C::BM, static_cast<int32_t>(r[j]));
         }
       }
-      if (split && !C::OUT_S32 && h < C::NUM_CHUNKS) {
+      if (split && h < C::NUM_CHUNKS) {
         // The last of the tile's splits to finish this warp slice sums the
-        // partials (int32: exact in any order) and writes y.
+        // partials (int32: exact in any order) and finishes them.
         __threadfence();
         __syncwarp();
         int* counter = args.counters + tile * C::EPI_WARPS + e;
@@ -667,7 +751,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j)
               r[j] = static_cast<uint32_t>(__ldcg(tile_acc + (j0 + j) * C::BM));
-            emit(r, j0);
+            finish(r, j0);
           }
         }
       }
@@ -741,7 +825,8 @@ struct SingleArgs {
 template <class C>
 cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
                      const EpilogueArgs& ep, void* out, const SplitScratch* scratch,
-                     cudaStream_t st, bool w_prefetch, const SingleArgs* single = nullptr) {
+                     cudaStream_t st, bool w_prefetch, const SingleArgs* single,
+                     const GemmExtras* ex) {
   CUtensorMap tm_w, tm_x, tm_out;
   bool ok = make_map(&tm_w, qw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, C::BK / 2, C::BM,
                      CU_TENSOR_MAP_SWIZZLE_64B);
@@ -754,11 +839,14 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
   else
     ok = ok && make_map(&tm_x, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, C::BK / 2, C::BN,
                         CU_TENSOR_MAP_SWIZZLE_64B);
-  if (C::OUT_S32)
-    ok = ok && make_map(&tm_out, out, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, N, M, 32, C::EPI_CHUNK,
-                        CU_TENSOR_MAP_SWIZZLE_NONE);
-  else
-    ok = ok && make_map(&tm_out, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 32, C::EPI_CHUNK,
+  int32_t* acc_out = ex ? ex->acc_out : nullptr;
+  if (out == nullptr && acc_out == nullptr) return cudaErrorInvalidValue;
+  if (C::EPI > 0)  // the next linear's int8 codes [M][N], boxes of 32 channels x 16 tokens
+    ok = ok && out && make_map(&tm_out, out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, M, 32,
+                               C::EPI_CHUNK, CU_TENSOR_MAP_SWIZZLE_NONE);
+  else  // y; the int32 debug view alone maps its own buffer here, and never stores to it
+    ok = ok && make_map(&tm_out, out ? out : static_cast<void*>(acc_out),
+                        CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 32, C::EPI_CHUNK,
                         CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return cudaErrorInvalidValue;
 
@@ -773,7 +861,7 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
   // Keep the smaller operand resident in L2: sweep output channels fastest when
   // the packed weights fit comfortably, so each activation tile streams once.
   a.n_fastest = (static_cast<size_t>(N) * K / 2) <= (48u << 20) ? 1 : 0;
-  a.splits = (C::OUT_S32 || scratch != nullptr) ? gemm_splits(M, N, K) : 1;
+  a.splits = scratch != nullptr ? gemm_splits(M, N, K) : 1;
   a.num_units = a.num_tiles * a.splits;
   a.partial = scratch ? scratch->partial : nullptr;
   a.counters = scratch ? scratch->counters : nullptr;
@@ -783,6 +871,15 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
   a.q_alpha = single ? single->table : nullptr;
   a.q_thr = single ? single->thr : nullptr;
   a.ep = ep;
+  a.has_y = out != nullptr ? 1 : 0;
+  a.acc_out = acc_out;
+  a.g_thr = ex ? ex->next_thr : nullptr;
+  a.g_gain = ex ? ex->next_gain : nullptr;
+  a.g_cinv = ex ? ex->next_cinv : nullptr;
+  a.g_s = ex ? ex->next_s : nullptr;
+  a.g_h = ex ? ex->h : nullptr;
+  if (C::EPI > 0 && (a.g_thr == nullptr || a.g_gain == nullptr || a.g_s == nullptr))
+    return cudaErrorInvalidValue;
 
   static std::atomic<bool> attr_set[kAttrDevices] = {};  // per template instance and device
   const cudaError_t e = set_smem_once(gemm_kernel<C>, C::SMEM_BYTES, attr_set);
@@ -791,16 +888,23 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
   return launch_pdl(gemm_kernel<C>, grid, C::THREADS, C::SMEM_BYTES, st, tm_w, tm_x, tm_out, a);
 }
 
-template <int ACT_BITS, bool OUT_S32>
+template <int ACT_BITS, int EPI = 0>
 cudaError_t dispatch_bn(const void* qx, const uint8_t* qw, int M, int N, int K,
                         const EpilogueArgs& ep, void* out, const SplitScratch* sc,
-                        cudaStream_t st, bool wp) {
+                        cudaStream_t st, bool wp, const GemmExtras* ex) {
   switch (bn_for(M)) {
-    case 16: return run_gemm<Cfg<16, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, sc, st, wp);
-    case 32: return run_gemm<Cfg<32, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, sc, st, wp);
-    case 64: return run_gemm<Cfg<64, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, sc, st, wp);
-    case 128: return run_gemm<Cfg<128, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, sc, st, wp);
-    default: return run_gemm<Cfg<256, ACT_BITS, OUT_S32>>(qx, qw, M, N, K, ep, out, sc, st, wp);
+    case 16:
+      return run_gemm<Cfg<16, ACT_BITS, 0, EPI>>(qx, qw, M, N, K, ep, out, sc, st, wp, nullptr, ex);
+    case 32:
+      return run_gemm<Cfg<32, ACT_BITS, 0, EPI>>(qx, qw, M, N, K, ep, out, sc, st, wp, nullptr, ex);
+    case 64:
+      return run_gemm<Cfg<64, ACT_BITS, 0, EPI>>(qx, qw, M, N, K, ep, out, sc, st, wp, nullptr, ex);
+    case 128:
+      return run_gemm<Cfg<128, ACT_BITS, 0, EPI>>(qx, qw, M, N, K, ep, out, sc, st, wp, nullptr,
+                                                   ex);
+    default:
+      return run_gemm<Cfg<256, ACT_BITS, 0, EPI>>(qx, qw, M, N, K, ep, out, sc, st, wp, nullptr,
+                                                   ex);
   }
 }
 
@@ -808,12 +912,12 @@ template <int QBITS>
 cudaError_t dispatch_single(const SingleArgs& sa, const uint8_t* qw, int M, int N, int K,
                             const EpilogueArgs& ep, void* y, cudaStream_t st) {
   switch (bn_for(M)) {
-    case 16: return run_gemm<Cfg<16, 8, false, QBITS>>(nullptr, qw, M, N, K, ep, y, nullptr, st,
-                                                       false, &sa);
-    case 32: return run_gemm<Cfg<32, 8, false, QBITS>>(nullptr, qw, M, N, K, ep, y, nullptr, st,
-                                                       false, &sa);
-    default: return run_gemm<Cfg<64, 8, false, QBITS>>(nullptr, qw, M, N, K, ep, y, nullptr, st,
-                                                       false, &sa);
+    case 16: return run_gemm<Cfg<16, 8, QBITS>>(nullptr, qw, M, N, K, ep, y, nullptr, st, false,
+                                                &sa, nullptr);
+    case 32: return run_gemm<Cfg<32, 8, QBITS>>(nullptr, qw, M, N, K, ep, y, nullptr, st, false,
+                                                &sa, nullptr);
+    default: return run_gemm<Cfg<64, 8, QBITS>>(nullptr, qw, M, N, K, ep, y, nullptr, st, false,
+                                                &sa, nullptr);
   }
 }
 
@@ -851,15 +955,22 @@ size_t gemm_split_scratch_bytes(int M, int N, int K) {
 }
 
 cudaError_t launch_gemm(const void* qx, int act_bits, const uint8_t* qw, int M, int N, int K,
-                        const EpilogueArgs& ep, void* out, bool out_s32,
-                        const SplitScratch* scratch, cudaStream_t st, bool w_prefetch) {
+                        const EpilogueArgs& ep, void* y, const SplitScratch* scratch,
+                        cudaStream_t st, bool w_prefetch, const GemmExtras* extras) {
   if (M == 0) return cudaSuccess;
-  const bool wp = w_prefetch;
-  if (act_bits == 8)
-    return out_s32 ? dispatch_bn<8, true>(qx, qw, M, N, K, ep, out, scratch, st, wp)
-                   : dispatch_bn<8, false>(qx, qw, M, N, K, ep, out, scratch, st, wp);
-  return out_s32 ? dispatch_bn<4, true>(qx, qw, M, N, K, ep, out, scratch, st, wp)
-                 : dispatch_bn<4, false>(qx, qw, M, N, K, ep, out, scratch, st, wp);
+  return act_bits == 8
+             ? dispatch_bn<8>(qx, qw, M, N, K, ep, y, scratch, st, w_prefetch, extras)
+             : dispatch_bn<4>(qx, qw, M, N, K, ep, y, scratch, st, w_prefetch, extras);
+}
+
+cudaError_t launch_gemm_gelu_quant(const void* qx, const uint8_t* qw, int M, int N, int K,
+                                   const EpilogueArgs& ep, int next_bits, int8_t* codes,
+                                   const SplitScratch* scratch, cudaStream_t st, bool w_prefetch,
+                                   const GemmExtras& extras) {
+  if (M == 0) return cudaSuccess;
+  return next_bits == 8
+             ? dispatch_bn<8, 8>(qx, qw, M, N, K, ep, codes, scratch, st, w_prefetch, &extras)
+             : dispatch_bn<8, 4>(qx, qw, M, N, K, ep, codes, scratch, st, w_prefetch, &extras);
 }
 
 }  // namespace wq

@@ -97,10 +97,9 @@ cudaError_t launch_linear_single(const uint16_t* x, const float* cinv, const flo
                                  int K, const EpilogueArgs& ep, void* y, cudaStream_t st);
 
 // Split-K (small token counts): the K blocks of each output tile are spread over
-// `splits` CTAs so that about kSplitTargetCtas CTAs stream the weights.  The
-// bf16 path needs scratch for the int32 partial tiles and one counter per
-// epilogue-warp slice of each tile; the int32 debug path adds its partials
-// atomically into the (zeroed) output instead.
+// `splits` CTAs so that about kSplitTargetCtas CTAs stream the weights, through
+// scratch for the int32 partial tiles and one counter per epilogue-warp slice of
+// each tile.
 constexpr int kSplitTargetCtas = 148;
 int gemm_splits(int M, int N, int K);
 size_t gemm_split_scratch_bytes(int M, int N, int K);  // partials + counters, 0 if no split
@@ -110,16 +109,42 @@ struct SplitScratch {
   int* counters;     // [tiles][8], zero before the launch
 };
 
-// y[M][N] (bf16) = epilogue(qx x qw^T) when out_s32 == false; acc[M][N] (int32)
-// when out_s32 == true (the epilogue arguments are then ignored).  bf16 with
-// scratch == nullptr never splits K; out_s32 splits into atomics on `out`,
-// which the caller must have zeroed when gemm_splits() > 1.
+// Optional parts of a GEMM launch.
+struct GemmExtras {
+  int32_t* acc_out = nullptr;  // int32 [M][N]: a copy of the accumulators (debug view)
+  // launch_gemm_gelu_quant: the next linear's static clipping, thresholds [T] and
+  // stream gains [T][S]; its channel scale [N] (or null); its per-token scales
+  // s_next [M] (written); h = bf16(GELU(y)) [M][N] (written when not null)
+  const float* next_thr = nullptr;
+  const float* next_gain = nullptr;
+  const float* next_cinv = nullptr;
+  float* next_s = nullptr;
+  uint16_t* h = nullptr;
+};
+
+// y[M][N] (bf16) = epilogue(qx x qw^T).  y may be null when extras->acc_out is
+// set: the launch then writes only the int32 accumulators (the epilogue
+// arguments other than S and step are not read).  With scratch == nullptr K is
+// never split; otherwise it is split as gemm_splits() says, through the scratch,
+// which must be zero before the launch.  Every instance writes the same
+// accumulators through the same pipeline whether or not acc_out is set.
 // w_prefetch: the packed weights (and nothing else) may be read before the
 // previous kernel in the stream has finished.  Only valid when that kernel is
 // this library's quantizer, which starts its dependents only after everything
 // launched before it has completed.
 cudaError_t launch_gemm(const void* qx, int act_bits, const uint8_t* qw, int M, int N, int K,
-                        const EpilogueArgs& ep, void* out, bool out_s32,
-                        const SplitScratch* scratch, cudaStream_t st, bool w_prefetch = false);
+                        const EpilogueArgs& ep, void* y, const SplitScratch* scratch,
+                        cudaStream_t st, bool w_prefetch = false,
+                        const GemmExtras* extras = nullptr);
+
+// The FFN up-projection whose epilogue quantizes for the down-projection: the
+// same GEMM on int8 codes qx, y as launch_gemm computes it, then h = bf16(GELU(y))
+// and codes[m][n] = clamp(rint(h * next_cinv[n] / s_next[m]), +-qmax_next) with
+// s_next[m] = (next_thr[step] / next_gain[step][stream]) / qmax_next (qmax_next 127
+// for next_bits 8, 7 for 4), one code per int8 byte [M][N].  y is not stored.
+cudaError_t launch_gemm_gelu_quant(const void* qx, const uint8_t* qw, int M, int N, int K,
+                                   const EpilogueArgs& ep, int next_bits, int8_t* codes,
+                                   const SplitScratch* scratch, cudaStream_t st, bool w_prefetch,
+                                   const GemmExtras& extras);
 
 }  // namespace wq

@@ -23,6 +23,13 @@ __device__ unsigned int g_error_word = 0u;
 // legitimate wait in these kernels lasts microseconds.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
+// The limit in force (kWaitLimitNs unless a test hook lowered it), and the test
+// hook's stall: when >= 0, CTA 0 of every GEMM launch skips the activation copy
+// of that K block of its sequence, so the stage never completes and the waits on
+// it run out.  Both are set only by wq_debug_inject_stall().
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+__device__ int g_stall_kblock = -1;
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -87,8 +94,12 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+__device__ __forceinline__ unsigned long long wait_limit_ns() {
+  return *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+}
+
 // Wait for the phase with the given parity to complete.  Returns false (and
-// raises kErrWaitTimeout) if it did not complete within kWaitLimitNs, or if
+// raises kErrWaitTimeout) if it did not complete within the wait limit, or if
 // another CTA already raised an error.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
@@ -98,10 +109,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(a, parity)) return true;
     if ((i & 255u) == 0u) {
       if (error_raised()) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > wait_limit_ns()) {
         raise_error(kErrWaitTimeout);
         return false;
       }
+    }
+  }
+}
+
+// Wait for copies or MMAs this CTA issued to complete before it exits or frees
+// their memory: bounded by the time limit only (it does not give up early when
+// another CTA raised an error, since the operations are in flight either way).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_test_wait(a, parity)) return true;
+  unsigned long long t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(a, parity)) return true;
+    if ((i & 255u) == 0u && globaltimer_ns() - t0 > wait_limit_ns()) {
+      raise_error(kErrWaitTimeout);
+      return false;
     }
   }
 }
@@ -137,6 +164,17 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* desc, ui
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(desc)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Contiguous bulk copy global -> shared (both 16-byte aligned, bytes a multiple of
+// 16), completion counted on an mbarrier.
+__device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* src, uint32_t bytes,
+                                             uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 

@@ -76,6 +76,26 @@ __device__ __forceinline__ void quantize8_recip(const float (&v)[8], float s, fl
   }
 }
 
+// One code from the reciprocal, as quantize8_recip does for eight: identical to
+// quantize<QMAX>(v, s) for every input (s > 0, r = 1/s finite).  The result's low
+// byte is the code.
+template <int QMAX>
+__device__ __forceinline__ uint32_t quantize1_recip(float v, float s, float r) {
+  const float t = __fmul_rn(v, r);
+  const float u = __fadd_rn(t, kRoundMagic);
+  const float d = __fsub_rn(t, __fsub_rn(u, kRoundMagic));
+  if (fabsf(d) >= 0.5f - 0x1p-12f) return static_cast<uint32_t>(quantize_exact<QMAX>(v, s));
+  return __float_as_uint(fminf(fmaxf(u, kRoundMagic - static_cast<float>(QMAX)),
+                               kRoundMagic + static_cast<float>(QMAX)));
+}
+
+// GELU(v) = v * Phi(v), Phi the standard normal distribution function, written
+// as Phi(v) = erfc(-v / sqrt(2)) / 2 so that it stays accurate for negative v;
+// fp32 with CUDA's erfcf.
+__device__ __forceinline__ float gelu_f32(float v) {
+  return __fmul_rn(__fmul_rn(v, 0.5f), erfcf(__fmul_rn(v, -0.70710678118654752f)));
+}
+
 // Low bytes of four words -> one word.
 __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c,
                                                    uint32_t d) {
@@ -398,11 +418,279 @@ cudaError_t run_act_quant_rows(const uint16_t* x, int M, int K, const float* cin
                     K, cinv, sid, alpha, thr, S, step, qx, s_tok, zero, zero_n16);
 }
 
+// ---------------------------------------------------------------- staged rows
+// Many rows of K = 512*C channels: rows are staged in shared memory by bulk copies
+// (a ring of kRingSlots rounds of R = kRingRoundElems / K rows, copies of later
+// rounds in flight while a round is computed), and every one of the 512 threads
+// owns C fixed channels of every row, so its C channel scales stay in registers
+// for the whole launch and each staged element is read from shared memory once:
+// x' = x * cinv is formed once into registers, the row maxima are combined
+// across the CTA (warp shuffles, then one shared-memory atomic max per warp and
+// row), R threads turn them into the rows' scales, and every thread writes the
+// codes of its channels.  One CTA per SM, persistent over rounds.
+constexpr int kRingThreads = 512;
+constexpr int kRingRoundElems = 32768;  // 64 KB of bf16 per round
+constexpr int kRingSlots = 3;
+#ifndef WQ_RING_MIN_ROWS
+#define WQ_RING_MIN_ROWS 512
+#endif
+constexpr int kRingMinRows = WQ_RING_MIN_ROWS;
+
+template <int C>
+struct Ring {
+  static constexpr int K = kRingThreads * C;
+  static constexpr int R = kRingRoundElems / K;           // rows per round
+  static constexpr int ROUND_BYTES = R * K * 2;
+  static constexpr int OFF_AMAX = kRingSlots * ROUND_BYTES;  // uint32 [2][R]
+  static constexpr int OFF_SCALE = OFF_AMAX + 2 * R * 4;    // float [R] s, then [R] 1/s
+  static constexpr int OFF_BAR = (OFF_SCALE + 2 * R * 4 + 7) / 8 * 8;
+  static constexpr int SMEM = OFF_BAR + kRingSlots * 8;
+  static_assert(R >= 1 && C >= 4 && C % 4 == 0, "C = K / 512 channels per thread");
+};
+
+// N codes from the reciprocal (see quantize8_recip); each result's low byte is the code.
+template <int QMAX, int N>
+__device__ __forceinline__ void quantize_recip_n(const float* v, float s, float r,
+                                                 uint32_t* c) {
+  constexpr float lo = kRoundMagic - static_cast<float>(QMAX);
+  constexpr float hi = kRoundMagic + static_cast<float>(QMAX);
+  bool near_tie = false;
+#pragma unroll
+  for (int e = 0; e < N; ++e) {
+    const float t = __fmul_rn(v[e], r);
+    const float u = __fadd_rn(t, kRoundMagic);
+    const float d = __fsub_rn(t, __fsub_rn(u, kRoundMagic));
+    near_tie = near_tie || fabsf(d) >= 0.5f - 0x1p-12f;
+    c[e] = __float_as_uint(fminf(fmaxf(u, lo), hi));
+  }
+  if (near_tie) {
+#pragma unroll
+    for (int e = 0; e < N; ++e) {
+      const float t = __fmul_rn(v[e], r);
+      const float u = __fadd_rn(t, kRoundMagic);
+      const float d = __fsub_rn(t, __fsub_rn(u, kRoundMagic));
+      if (fabsf(d) >= 0.5f - 0x1p-12f) c[e] = static_cast<uint32_t>(quantize_exact<QMAX>(v[e], s));
+    }
+  }
+}
+
+// Maxima over the warp of R values per lane (R a power of two, at most 32), with
+// R - 1 + 5 - log2(R) shuffles instead of 5 R: each step halves the values a lane
+// keeps and the lanes exchanging them.  Returns, in lane l, the maximum of value
+// index (l >> (5 - log2 R)) over all 32 lanes.
+template <int R>
+__device__ __forceinline__ float warp_max_multi(float (&v)[R], int lane) {
+  int o = 16;
+#pragma unroll
+  for (int n = R; n > 1; n >>= 1, o >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < n / 2; ++j) {
+      const float send = upper ? v[j] : v[j + n / 2];
+      const float keep = upper ? v[j + n / 2] : v[j];
+      v[j] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, o));
+    }
+  }
+#pragma unroll
+  for (; o > 0; o >>= 1) v[0] = fmaxf(v[0], __shfl_xor_sync(0xFFFFFFFFu, v[0], o));
+  return v[0];
+}
+
+template <int R>
+constexpr int log2_of() { return R <= 1 ? 0 : 1 + log2_of<R / 2>(); }
+
+template <int ACT_BITS, int STORE_BITS, int C, bool STATIC>
+__global__ void __launch_bounds__(kRingThreads, 1) act_quant_ring_kernel(
+    const uint16_t* __restrict__ x, int M, const float* __restrict__ cinv,
+    const uint8_t* __restrict__ stream_id, const float* __restrict__ alpha,
+    const float* __restrict__ thr, int S, int step, void* __restrict__ qx,
+    float* __restrict__ s_tok, uint4* __restrict__ zero, size_t zero_n16) {
+  using G = Ring<C>;
+  constexpr int K = G::K, R = G::R;
+  constexpr int QMAX = ACT_BITS == 8 ? 127 : 7;
+  constexpr int CH = C / 4;  // groups of 4 channels a thread owns (8 bytes of bf16 each)
+  extern __shared__ __align__(128) uint8_t ring_smem[];
+  uint32_t* amax_s = reinterpret_cast<uint32_t*>(ring_smem + G::OFF_AMAX);
+  float* scale_s = reinterpret_cast<float*>(ring_smem + G::OFF_SCALE);
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring_smem + G::OFF_BAR);
+  const int t = threadIdx.x;
+  const int warp = t >> 5, lane = t & 31;
+
+  if (t == 0) {
+    for (int i = 0; i < kRingSlots; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
+  if (t < 2 * R) amax_s[t] = 0u;
+  // thread t owns channel groups g = t + 512 * j (channels 4g .. 4g + 3)
+  float ci[C];
+#pragma unroll
+  for (int j = 0; j < CH; ++j) {
+    const int k0 = 4 * (t + kRingThreads * j);
+    const float4 a = cinv ? __ldg(reinterpret_cast<const float4*>(cinv + k0))
+                          : make_float4(1.f, 1.f, 1.f, 1.f);
+    ci[4 * j] = a.x; ci[4 * j + 1] = a.y; ci[4 * j + 2] = a.z; ci[4 * j + 3] = a.w;
+  }
+  __syncthreads();
+  // x, the ids and the split-K scratch may belong to the previous kernel
+  griddep_wait();
+  griddep_launch_dependents();
+  for (size_t i = (size_t)blockIdx.x * kRingThreads + t; i < zero_n16;
+       i += (size_t)gridDim.x * kRingThreads)
+    zero[i] = make_uint4(0u, 0u, 0u, 0u);
+
+  const int rounds = (M + R - 1) / R;
+  auto issue = [&](int local) {  // copy this CTA's round `local` into its slot
+    const int q = blockIdx.x + local * gridDim.x;
+    if (q >= rounds) return;
+    const int rows = min(R, M - q * R);
+    uint64_t* bar = &full[local % kRingSlots];
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows) * K * 2);
+    bulk_load_1d(ring_smem + (local % kRingSlots) * G::ROUND_BYTES, x + (size_t)q * R * K,
+                 static_cast<uint32_t>(rows) * K * 2, bar);
+  };
+  if (t == 0)
+    for (int i = 0; i < kRingSlots; ++i) issue(i);
+
+  int issued = kRingSlots;
+  bool ok = true;
+  int local = 0;
+  for (int q = blockIdx.x; q < rounds; q += gridDim.x, ++local) {
+    const int slot = local % kRingSlots;
+    const int row0 = q * R;
+    const int rows = min(R, M - row0);
+    const bool landed = mbar_wait(&full[slot], (local / kRingSlots) & 1u);
+    // x' of this thread's channels of every row of the round, and the row maxima
+    float xv[R][C];
+    float pmax[R];  // this thread's maximum of |x'| per row
+    const uint8_t* base = ring_smem + slot * G::ROUND_BYTES;
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < CH; ++j) {
+        const uint2 w = (landed && i < rows)
+                            ? *reinterpret_cast<const uint2*>(base + (size_t)i * K * 2 +
+                                                               8 * (t + kRingThreads * j))
+                            : make_uint2(0u, 0u);
+        const float f[4] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y)};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          xv[i][4 * j + e] = __fmul_rn(f[e], ci[4 * j + e]);
+          amax = fmaxf(amax, fabsf(xv[i][4 * j + e]));
+        }
+      }
+      pmax[i] = amax;
+    }
+    if constexpr (!STATIC) {
+      // row (lane >> SH) of the round, reduced over the warp, then over the warps
+      // (non-negative floats order as their bit patterns)
+      constexpr int SH = 5 - log2_of<R>();
+      const float wmax = warp_max_multi<R>(pmax, lane);
+      if ((lane & ((1 << SH) - 1)) == 0 && wmax > 0.0f)
+        atomicMax(&amax_s[(local & 1) * R + (lane >> SH)], __float_as_uint(wmax));
+    }
+    if (t < R) amax_s[((local + 1) & 1) * R + t] = 0u;  // the next round's maxima
+    // every thread has read its channels of the slot, and every row maximum is in
+    if (__syncthreads_or(!landed)) { ok = false; break; }
+    if (t == 0 && issued < kRingSlots + local + 1) {  // refill the slot just read
+      issue(local + kRingSlots);
+      issued = kRingSlots + local + 1;
+    }
+    if (t < rows) {
+      const int row = row0 + t;
+      float sc = 0.0f;
+      const int sid = stream_id[row];
+      if (sid < S) {
+        float clip;
+        if constexpr (STATIC) {
+          const float g = __ldg(alpha + step * S + sid);
+          clip = g > 0.0f ? __fdiv_rn(__ldg(thr + step), g) : 0.0f;
+        } else {
+          clip = __fmul_rn(__ldg(alpha + step * S + sid),
+                           __uint_as_float(amax_s[(local & 1) * R + t]));
+        }
+        sc = __fdiv_rn(clip, static_cast<float>(QMAX));
+      } else {
+        raise_error(kErrBadStreamId);
+      }
+      s_tok[row] = sc;
+      scale_s[t] = sc;
+      scale_s[R + t] = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      if (i >= rows) break;
+      const float sc = scale_s[i], rc = scale_s[R + i];
+      const bool fast = sc > 0.0f && isfinite(rc);
+      const size_t row = static_cast<size_t>(row0 + i);
+#pragma unroll
+      for (int j = 0; j < CH; ++j) {
+        uint32_t cq[4];
+        if (fast) {
+          quantize_recip_n<QMAX, 4>(&xv[i][4 * j], sc, rc, cq);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            cq[e] = static_cast<uint32_t>(quantize<QMAX>(xv[i][4 * j + e], sc));
+        }
+        const int g = t + kRingThreads * j;  // channel group: channels 4g .. 4g + 3
+        if constexpr (STORE_BITS == 8) {
+          reinterpret_cast<uint32_t*>(static_cast<int8_t*>(qx) + row * K)[g] =
+              pack_low_bytes(cq[0], cq[1], cq[2], cq[3]);
+        } else {
+          const uint32_t b = pack_low_bytes(cq[0], cq[1], cq[2], cq[3]) & 0x0F0F0F0Fu;
+          const uint32_t n = b | (b >> 4);  // bytes 0 and 2: (c0 | c1 << 4), (c2 | c3 << 4)
+          reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(qx) + row * (K / 2))[g] =
+              static_cast<uint16_t>(__byte_perm(n, 0u, 0x0020) & 0xFFFFu);
+        }
+      }
+    }
+  }
+  // copies still in flight (after an error, or none): wait for them before exiting
+  if (t == 0) {
+    const int my_rounds = blockIdx.x < rounds ? (rounds - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int last = min(issued, my_rounds);
+    for (int i = ok ? last : local; i < last; ++i)
+      mbar_wait_drain(&full[i % kRingSlots], (i / kRingSlots) & 1u);
+  }
+}
+
+template <int ACT_BITS, int STORE_BITS, int C, bool STATIC>
+cudaError_t run_act_quant_ring(const uint16_t* x, int M, const float* cinv, const uint8_t* sid,
+                               const float* alpha, const float* thr, int S, int step, void* qx,
+                               float* s_tok, uint4* zero, size_t zero_n16, cudaStream_t st) {
+  using G = Ring<C>;
+  static std::atomic<bool> attr_set[kAttrDevices] = {};  // per template instance and device
+  const cudaError_t ea =
+      set_smem_once(act_quant_ring_kernel<ACT_BITS, STORE_BITS, C, STATIC>, G::SMEM, attr_set);
+  if (ea != cudaSuccess) return ea;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int rounds = (M + G::R - 1) / G::R;
+  const int grid = rounds < sms ? rounds : sms;
+  return launch_pdl(act_quant_ring_kernel<ACT_BITS, STORE_BITS, C, STATIC>, grid, kRingThreads,
+                    G::SMEM, st, x, M, cinv, sid, alpha, thr, S, step, qx, s_tok, zero,
+                    zero_n16);
+}
+
 template <int ACT_BITS, int STORE_BITS, bool STATIC>
 cudaError_t dispatch_act_quant(const uint16_t* x, int M, int K, const float* cinv,
                                const uint8_t* sid, const float* alpha, const float* thr, int S,
                                int step, void* qx, float* s_tok, uint4* zero, size_t zero_n16,
                                cudaStream_t st) {
+#define WQ_RING(C_)                                                                         \
+  return run_act_quant_ring<ACT_BITS, STORE_BITS, C_, STATIC>(x, M, cinv, sid, alpha, thr, S, \
+                                                              step, qx, s_tok, zero, zero_n16, st)
+  // Many rows: rows staged in shared memory, channels owned by threads.
+  if (M >= kRingMinRows) {
+    if (K == 2048) WQ_RING(4);
+    if (K == 4096) WQ_RING(8);
+    if (K == 8192) WQ_RING(16);
+    if (K == 16384) WQ_RING(32);
+  }
+#undef WQ_RING
   // Many rows of moderate length: independent warps, one per row (measured faster
   // for M = 4288 and 8512 at K = 2048 and 4096).  Few rows, or long rows, keep a
   // CTA's threads on each row (measured faster for M <= 256, and for K >= 8192).

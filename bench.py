@@ -9,10 +9,13 @@ stream) clip folded in) followed by the int4 x int8 tensor-core GEMM with the
 fused dequantization / bias / output-compensation epilogue.  Weight preparation
 (channel scale, int4 packing) is offline and runs before timing.
 
-Default workload: one hidden-2048 transformer block (QKV 2048->6144, attn-out
-2048->2048, MLP-up 2048->8192, MLP-down 8192->2048), W4A8, M = 4096 video + 64
-proprio + 128 action tokens, seeded synthetic inputs.  Metric: int8 tensor ops
-(2*M*N*K per linear) per second, whole job.
+Default workload: one hidden-4096 transformer block (QKV 4096->12288, attn-out
+4096->4096, MLP-up 4096->16384, MLP-down 16384->4096), W4A8, M = 8192 video + 64
+proprio + 256 action tokens, the step cycling through a 10-row (denoising step x
+stream) clip / compensation table with fresh seeded activations; the same block
+with 4-bit activations (W4A4) is measured after it and reported beside it in the
+line ("w4a4").  Metric: int8 tensor ops (2*M*N*K per linear) per second, whole
+job.
 
 Multi-GPU: every rank runs an independent replica of the step (the path has no
 exchange step); the time is the max over ranks and the value counts all ranks'
@@ -44,13 +47,19 @@ INT8_PER_BF16 = 2.0  # nominal dense ratio (4.5 POPS int8 / 2.25 PFLOP/s bf16)
 L2_BYTES = 126 * 2 ** 20
 
 
+DEFAULT_WORKLOAD = "block4096_w4a8_t10"
+
+
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=500)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["wq", "reference"], default="wq")
-    p.add_argument("--workload", default="block2048_w4a8", choices=sorted(S.WORKLOADS))
+    p.add_argument("--workload", default=None, choices=sorted(S.WORKLOADS),
+                   help=f"default {DEFAULT_WORKLOAD} (--sequence: every block)")
+    p.add_argument("--no-companion", action="store_true",
+                   help="skip the W4A4 run reported beside a W4A8 headline")
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-graph", action="store_true",
@@ -65,7 +74,8 @@ def parse():
     return p.parse_args()
 
 
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_traffic_block2048_w4a8.md")
+def traffic_file(workload):
+    return os.path.join(ROOT, "profiles", f"gemm_traffic_{workload}.md")
 GEMM_SOURCES = [os.path.join(ROOT, "activation_quantized_gemm_wq_b200", "csrc", f)
                 for f in ("wq_gemm.cuh", "wq_ptx.cuh")]
 HOST_SIDE_MARKER = b"// ------------------------------------------------------------------ host side"
@@ -87,11 +97,9 @@ def gemm_device_source_hash(paths=None):
 def gemm_traffic(workload):
     """DRAM bytes per GEMM launch from the committed ncu capture of this workload, or
     None when there is none or the GEMM sources changed since it was taken."""
-    if workload != "block2048_w4a8":
-        return None
     try:
         fields = {}
-        with open(TRAFFIC_FILE) as f:
+        with open(traffic_file(workload)) as f:
             for line in f:
                 if ":" in line and line.startswith("    "):
                     k, v = line.strip().split(":", 1)
@@ -268,28 +276,30 @@ class Layer:
         self.x = [dev(h) for h in self.host_x]
         bits = wl.act_bits
         self.bits = bits
-        self.qx = torch.empty((self.M, self.K) if bits == 8 else (self.M, self.K // 2),
-                              dtype=torch.int8 if bits == 8 else torch.uint8, device="cuda")
-        self.s_tok = torch.empty(self.M, dtype=torch.float32, device="cuda")
+        self.name = lin.name
         self.y = torch.empty((self.M, self.N), dtype=torch.bfloat16, device="cuda")
         self.ws = wq.alloc_workspace(self.M, self.K, self.N, bits)
+        # the fused call's codes (one per int8 byte) and token scales, in its workspace
+        self.ws_codes = self.ws[: self.M * self.K].view(torch.int8).view(self.M, self.K)
+        off = (self.M * self.K + 255) // 256 * 256
+        self.ws_stok = self.ws[off: off + 4 * self.M].view(torch.float32)
 
     def ops(self):
         return 2 * self.M * self.N * self.K
 
 
-def run_gpu(args, rank, world, local):
-    import torch
+# The W4A4 run reported beside the W4A8 headline of the same block shapes.
+COMPANION = {"block4096_w4a8_t10": "block4096_w4a4_t10", "block2048_w4a8": "block2048_w4a4_t10"}
+NOMINAL_INT8_TOPS = 4500.0  # B200 dense int8, NVIDIA's figure without sparsity
 
-    import activation_quantized_gemm_wq_b200 as wq
 
-    torch.cuda.set_device(local)
-    wl = S.WORKLOADS[args.workload]
+def _round256(n):
+    return (n + 255) // 256 * 256
 
-    def dev(a):
-        a = np.ascontiguousarray(a)
-        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
 
+def measure_workload(args, wl, wq, torch, world, local, dev):
+    """Time one workload's step (every linear of the block, fused calls, one CUDA graph
+    per step) and its dominant kernel; returns the fields of the JSON line."""
     _, n_sets = activation_sets(wl)
     layers = [Layer(wl, i, n_sets, wq, torch, dev) for i in range(len(wl.linears))]
     torch.cuda.synchronize()
@@ -306,14 +316,17 @@ def run_gpu(args, rank, world, local):
                            L.ws)
 
     def step_split(it, gemm_events):
-        """The same pass as two calls per linear, with events around each GEMM."""
+        """The same pass, each fused call followed by the GEMM alone on the codes and
+        token scales the call left in its workspace (one code per int8 byte for both
+        widths: the very kernel instance the fused call runs), between events."""
         t = it % T
         r = it % n_sets
         for j, L in enumerate(layers):
-            wq.wq_act_quant(L.x[r], L.cinv, L.sid, L.alpha, t, L.bits, L.qx, L.s_tok)
+            lin_fn[L.bits](L.x[r], L.cinv, L.sid, L.alpha, L.beta, t, L.qw, L.s_w, L.bias, L.y,
+                           L.ws)
             gemm_events[j][0].record(stream)
-            wq.wq_gemm_w4ax(L.qx, L.s_tok, L.bits, L.K, L.sid, L.beta, L.S, L.T, t, L.qw, L.s_w,
-                            L.bias, L.y)
+            wq.wq_gemm_w4ax(L.ws_codes, L.ws_stok, 8, L.K, L.sid, L.beta, L.S, L.T, t, L.qw,
+                            L.s_w, L.bias, L.y)
             gemm_events[j][1].record(stream)
 
     # one CUDA graph per distinct step (denoising step t x activation set r)
@@ -358,18 +371,16 @@ def run_gpu(args, rank, world, local):
     assert status == ("WQ_OK", 0), status
 
     # the dominant kernel's launch duration: the same steps again, launched from the
-    # host as quantizer + GEMM calls with an event pair around every GEMM
+    # host, with an event pair around a GEMM-only launch after every fused call
     ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
            for _ in layers] for _ in range(args.steps)]
-    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    s0.record(stream)
     for it in range(args.steps):
         step_split(args.warmup + it, ev[it])
-    s1.record(stream)
     torch.cuda.synchronize()
-    split_ms = s0.elapsed_time(s1)
-    gemm_ms = sum(a.elapsed_time(b) for per_step in ev for a, b in per_step)
+    per_layer_ms = [sum(ev[it][j][0].elapsed_time(ev[it][j][1]) for it in range(args.steps))
+                    / args.steps for j in range(len(layers))]
+    gemm_ms = sum(per_layer_ms) * args.steps
     assert wq.wq_device_status() == ("WQ_OK", 0)
     if not args.no_graph:
         del graphs
@@ -377,32 +388,16 @@ def run_gpu(args, rank, world, local):
     t_max = max_over_ranks(elapsed_ms, world)
     ops_step = sum(L.ops() for L in layers)
     value = world * ops_step * args.steps / (t_max * 1e-3) / 1e12
-
-    # end to end through the public call with host buffers: pinned x in, y out
     e2e = run_e2e(args, layers, wq, torch, world)
-
-    # torch bf16 matmul of the same shapes, reported beside (not the product)
-    tb = torch_bf16(layers, torch)
 
     bf16_burst, bf16_sust, hbm, src = peaks()
     peak = bf16_burst * INT8_PER_BF16
     gemm_launches = args.steps * len(layers)
-    gemm_avg_ms = gemm_ms / gemm_launches
     achieved = ops_step * args.steps / (gemm_ms * 1e-3) / 1e12
-    out = {
-        "metric": METRIC,
+    ms_step = t_max / args.steps
+    res = {
         "value": round(value, 2),
-        "unit": "TOPS",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": round(t_max / args.steps, 5),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "int8",
-        "data": DATA,
-        "config": workload_config(wl, world),
+        "ms_per_step": round(ms_step, 5),
         "roofline": {
             "bound": "tensor",
             "kernel": "gemm_kernel (tcgen05 kind::i8)",
@@ -414,10 +409,17 @@ def run_gpu(args, rank, world, local):
             "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
             "peak_source": f"{src} bf16 burst {bf16_burst} TFLOP/s x{INT8_PER_BF16} (dense int8 "
                            "/ bf16 nominal ratio); units are int8 tera-ops",
-            "gemm_avg_launch_ms": round(gemm_avg_ms, 5),
-            "gemm_share_of_step": round(gemm_ms / split_ms, 4),
-            "measured": "event pair around every GEMM launch in a second pass of the same "
-                        f"{args.steps} steps (quantizer + GEMM calls from the host)",
+            "frac_of_nominal_int8": round(achieved / NOMINAL_INT8_TOPS, 4),
+            "gemm_avg_launch_ms": round(gemm_ms / gemm_launches, 5),
+            "gemm_share_of_step": round(sum(per_layer_ms) / ms_step, 4),
+            "per_linear": [
+                {"linear": f"{L.name} {L.K}->{L.N}", "gemm_us": round(1e3 * t, 2),
+                 "tops": round(L.ops() / (t * 1e-3) / 1e12, 1),
+                 "frac": round(L.ops() / (t * 1e-3) / 1e12 / peak, 4)}
+                for L, t in zip(layers, per_layer_ms)],
+            "measured": "event pair around a GEMM-only launch (the same kernel instance, on "
+                        "the codes each fused call left in its workspace) after every fused "
+                        f"call, over a second pass of the same {args.steps} steps",
         },
         "timing": ("one CUDA graph replay per step (fused wq_linear calls; the GEMM starts "
                    "under the quantizer by programmatic dependent launch)"
@@ -425,8 +427,90 @@ def run_gpu(args, rank, world, local):
         "clocks": clocks.summary(),
         "e2e": e2e,
         "gpu_launches": 2 * len(layers) * args.steps,
+    }
+    return res, layers
+
+
+def int8_probe(torch):
+    """Dense int8 GEMM throughput of the library path torch ships (torch._int_mm on
+    cuBLASLt, int32 out), 8192^3: a measured reference for the int8 tensor roof."""
+    try:
+        n = 8192
+        a = torch.randint(-128, 128, (n, n), dtype=torch.int8, device="cuda")
+        w = torch.randint(-128, 128, (n, n), dtype=torch.int8, device="cuda")
+        for _ in range(3):
+            torch._int_mm(a, w.t())
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 20
+        e0.record()
+        for _ in range(reps):
+            torch._int_mm(a, w.t())
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        del a, w
+        return {"tops": round(2 * n ** 3 / (ms * 1e-3) / 1e12, 1), "shape": "8192^3",
+                "via": "torch._int_mm (cuBLASLt int8 GEMM, int32 out), mean of 20 after 3"}
+    except Exception as e:  # reported, never fatal
+        return {"tops": None, "error": f"{type(e).__name__}: {str(e)[:160]}"}
+
+
+def run_gpu(args, rank, world, local):
+    import torch
+
+    import activation_quantized_gemm_wq_b200 as wq
+
+    torch.cuda.set_device(local)
+    wl = S.WORKLOADS[args.workload]
+
+    def dev(a):
+        a = np.ascontiguousarray(a)
+        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
+
+    res, layers = measure_workload(args, wl, wq, torch, world, local, dev)
+    # torch bf16 matmul of the same shapes, reported beside (not the product)
+    tb = torch_bf16(layers, torch)
+    del layers
+    torch.cuda.empty_cache()
+    out = {
+        "metric": METRIC,
+        "value": res["value"],
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": res["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": DATA,
+        "config": workload_config(wl, world),
+        "roofline": res["roofline"],
+        "timing": res["timing"],
+        "clocks": res["clocks"],
+        "e2e": res["e2e"],
+        "gpu_launches": res["gpu_launches"],
         "torch_bf16_same_shapes": tb,
     }
+    companion = COMPANION.get(wl.name)
+    if companion and not args.no_companion:
+        wl4 = S.WORKLOADS[companion]
+        r4, layers4 = measure_workload(args, wl4, wq, torch, world, local, dev)
+        del layers4
+        torch.cuda.empty_cache()
+        out["w4a4"] = {"workload": wl4.name, "act_bits": wl4.act_bits, "value": r4["value"],
+                       "unit": "TOPS", "ms_per_step": r4["ms_per_step"],
+                       "roofline": r4["roofline"], "e2e": r4["e2e"], "clocks": r4["clocks"],
+                       "gpu_launches": r4["gpu_launches"],
+                       "note": "same block shapes and token mix, 4-bit activation codes "
+                               "(kept one per byte between the two kernels)"}
+        out["gpu_launches"] += r4["gpu_launches"]
+    out["int8_mm_probe"] = int8_probe(torch)
+    if out["int8_mm_probe"].get("tops"):
+        out["roofline"]["frac_of_int8_mm_probe"] = round(
+            out["roofline"]["achieved"] / out["int8_mm_probe"]["tops"], 4)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(wl, budget_s=12.0)
     return out
@@ -826,9 +910,18 @@ def sweep(args):
             t_lin = _graph_ms(torch, l_fns)
             timing = f"CUDA graph of {calls} calls over {ncopy} input copies"
             del g_fns, l_fns, qws, qxs
-            xb = x.view(torch.bfloat16)
+            # torch bf16 on the same shapes, over activation and weight copies that
+            # together exceed twice the L2 (operands from HBM, as for the wq columns)
             wb = W.view(torch.bfloat16)
-            t_bf16 = _graph_ms(torch, [lambda: torch.nn.functional.linear(xb, wb)] * 10)
+            per_bf16 = 2 * M * K + 2 * N * K
+            nb = max(2, int(np.ceil(2 * l2 / per_bf16)))
+            wbs = [wb] + [wb.clone() for _ in range(nb - 1)]
+            xbs = [xs[r % ncopy].view(torch.bfloat16) if r < ncopy else
+                   xs[r % ncopy].view(torch.bfloat16).clone() for r in range(nb)]
+            t_bf16 = _graph_ms(torch, [lambda r=r: torch.nn.functional.linear(xbs[r % nb],
+                                                                          wbs[r % nb])
+                                       for r in range(max(10, nb))])
+            del wbs, xbs
             ops = 2 * M * N * K
             k1b, k2b = _alg_bytes(M, N, K, bits)
             roof_gemm = max(ops / p_int8, k2b / bw) * 1e3
@@ -871,8 +964,8 @@ def sequence(args):
 
     bf16_burst, _, hbm, src = peaks()
     p_int8 = bf16_burst * INT8_PER_BF16 * 1e12
-    names = [args.workload] if args.workload != "block2048_w4a8" else \
-        ["block2048_w4a4_t10", "block4096_w4a8_t10", "block4096_w4a4_t10"]
+    names = [args.workload] if args.workload else \
+        ["block2048_w4a8", "block2048_w4a4_t10", "block4096_w4a8_t10", "block4096_w4a4_t10"]
     for name in names:
         wl = S.WORKLOADS[name]
         T = wl.T
@@ -923,6 +1016,8 @@ def main():
     if args.sequence:
         sequence(args)
         return
+    if args.workload is None:
+        args.workload = DEFAULT_WORKLOAD
     rank, world, local = dist_init(args.gpus)
     try:
         if args.impl == "reference":

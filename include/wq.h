@@ -187,11 +187,66 @@ wq_status wq_linear_w4ax_single(const wq_bf16* x, int M, int K, int N, const flo
                                 const uint8_t* qw, const float* s_w, const float* bias,
                                 wq_bf16* y, wq_stream_t stream);
 
-/* Debug view of the GEMM's integer core: the same tensor-core mainloop with the
- * epilogue replaced by a raw store of the int32 accumulators acc [M][N] (every
- * element is overwritten).  qx as in wq_gemm_w4ax. */
+/* Debug view of the GEMM's integer core (§4.4): the product GEMM -- the same
+ * kernel instance, pipeline and split of K as the fused linears use for these
+ * sizes -- on codes qx (as in wq_gemm_w4ax), writing the int32 accumulators
+ * acc [M][N] (every element) instead of y.  workspace: device memory of at least
+ * wq_workspace_bytes(M, K, N, act_bits) bytes, 256-byte aligned (only its split-K
+ * part is used, and only for token counts small enough to split K; it may be
+ * NULL when no split is needed); its contents are overwritten. */
 wq_status wq_debug_gemm_s32(const void* qx, int act_bits, const uint8_t* qw, int M, int N,
-                            int K, int32_t* acc, wq_stream_t stream);
+                            int K, int32_t* acc, void* workspace, size_t ws_bytes,
+                            wq_stream_t stream);
+
+/* Debug view of the fused linear: exactly wq_linear_w4a8 (act_bits 8) or
+ * wq_linear_w4a4 (act_bits 4) -- the same two launches -- with the GEMM's int32
+ * accumulators acc [M][N] (sum_k q[m,k] * qw[n,k]) also written.  y, the
+ * workspace's codes and token scales are those of the plain call. */
+wq_status wq_debug_linear_s32(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                              const uint8_t* stream_id, const float* alpha, const float* beta,
+                              int S, int T, int step, int act_bits, const uint8_t* qw,
+                              const float* s_w, const float* bias, wq_bf16* y, int32_t* acc,
+                              void* workspace, size_t ws_bytes, wq_stream_t stream);
+
+/* App. D keeps GELU in BF16 between the FFN's quantized up- and down-projections.
+ * This call is the up-projection with the down-projection's activation
+ * quantization moved into its epilogue, so the bf16 hidden state never goes
+ * through device memory:
+ *   y[m,n]  = the fused linear's output, as wq_linear_w4a8 / w4a4 compute it
+ *             (bf16; act_bits of the up-projection's own activations, 8 or 4)
+ *   h[m,n]  = bf16(GELU(y[m,n])), GELU(v) = v * Phi(v) with Phi the standard
+ *             normal distribution function (fp32, CUDA's erfcf)
+ *   s_next[m] = (thr_next[step] / gain_next[step][stream_id[m]]) / qmax_next
+ *             (static clipping of §4.3 for the down-projection: IEEE divisions,
+ *             0 when the gain is not positive; qmax_next 127 for act_bits_next 8,
+ *             7 for 4)
+ *   codes_next[m,n] = clamp(rint_half_even(h[m,n] * cinv_next[n] / s_next[m]),
+ *             -qmax_next, qmax_next), int8 [M][N], one code per byte for both
+ *             widths; 0 when s_next[m] is 0.
+ * Dynamic clipping needs the maximum over the whole row before any code, which
+ * spans every output tile, so only static clipping can be fused here.
+ * The down-projection then runs wq_gemm_w4ax(codes_next, s_next, 8, ...) (int8
+ * operands for both widths; the int32 sums are the same).
+ *   cinv_next [N] fp32 or NULL (= 1); thr_next [T]; gain_next [T][S];
+ *   s_next [M] fp32 out; h [M][N] bf16 out or NULL (a debug copy; not needed).
+ * Workspace and other arguments as wq_linear_w4a8. */
+wq_status wq_linear_gelu_quant(const wq_bf16* x, int M, int K, int N, const float* cinv,
+                               const uint8_t* stream_id, const float* alpha, const float* beta,
+                               int S, int T, int step, int act_bits, const uint8_t* qw,
+                               const float* s_w, const float* bias, const float* cinv_next,
+                               const float* thr_next, const float* gain_next, int act_bits_next,
+                               int8_t* codes_next, float* s_next, wq_bf16* h, void* workspace,
+                               size_t ws_bytes, wq_stream_t stream);
+
+/* Test hook for the GEMM's bounded waits (off by default; a test of failure
+ * handling, never for production).  enable != 0: in every later GEMM launch on
+ * the current device, CTA 0 leaves out the activation copy of its first K block,
+ * so that pipeline stage never completes, and every wait gives up after limit_us
+ * microseconds (> 0) instead of 2 s.  The launch then ends with the
+ * WQ_DEVICE_ERR_TIMEOUT bit set (wq_device_status), its output undefined, and the
+ * GPU context intact.  enable == 0 restores both defaults.  Synchronizes the
+ * device; call it with no kernel of this library running. */
+wq_status wq_debug_inject_stall(int enable, unsigned limit_us);
 
 /* The fused W4A8 linear for callers that cannot allocate device memory.  The
  * paper has no counterpart to this entry point.
@@ -205,12 +260,17 @@ wq_status wq_debug_gemm_s32(const void* qx, int act_bits, const uint8_t* qw, int
  * GPU that loads the library holds it until the process exits.  No cudaMalloc,
  * cudaFree or other allocating routine is called.
  *
- * Limit: wq_workspace_bytes(M, K, N, 8) must not exceed 16 MiB (about
- * M*K + 4*M bytes; for example M = 4096 tokens at K = 4096).  Larger sizes
- * return WQ_ERR_SCRATCH before anything is launched.
+ * Limit: wq_workspace_bytes(M, K, N, 8) <= 16 MiB (16777216 bytes): the codes
+ * (M*K bytes), the token scales (4*M bytes) and, for token counts small enough
+ * to split K, the split-K scratch, each rounded up to 256 bytes.  For example,
+ * at K = 4096 and N = 4096, M = 4092 tokens fits exactly and M = 4093 does not.
+ * Larger sizes return WQ_ERR_SCRATCH before anything is launched.
  * The first call on a device looks up the scratch array's device address with
- * that device current (cudaGetSymbolAddress) and caches it; make that first
- * call before any stream capture on the device.
+ * that device current (cudaGetSymbolAddress) and caches it for the process;
+ * make that first call before any stream capture on the device.  A device reset
+ * (cudaDeviceReset) or any other teardown of the device's primary context
+ * invalidates the cached address: do not call this entry point on that device
+ * after one.
  * Every call shares the one array and reuses it as it stands: each call
  * rewrites all of the scratch it reads before reading it, so nothing needs
  * clearing, but calls whose work overlaps on the GPU (concurrent streams, or
@@ -225,7 +285,9 @@ wq_status wq_linear_w4a8_noalloc(const wq_bf16* x, int M, int K, int N, const fl
 /* Reads and clears the device error word of the current device (synchronizes
  * the device).  *flags receives the WQ_DEVICE_ERR_* bits seen since the last
  * call (may be NULL).  Returns WQ_OK, WQ_ERR_TIMEOUT, WQ_ERR_DEVICE or
- * WQ_ERR_CUDA. */
+ * WQ_ERR_CUDA.  While a WQ_DEVICE_ERR_TIMEOUT bit is set, later GEMM launches
+ * stop at their first wait that does not complete at once (their outputs are
+ * then undefined), so clear it before relying on further results. */
 wq_status wq_device_status(unsigned* flags);
 
 #ifdef __cplusplus

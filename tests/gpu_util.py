@@ -73,10 +73,61 @@ def gpu_linear(x, cinv, sid, alpha, beta, step, bits, qw, s_w, bias):
 
 
 def gpu_gemm_s32(qx, bits, qw, K):
+    """The product GEMM's int32 accumulators on codes qx (K split as the fused linear
+    splits it for these sizes, through a workspace)."""
     M, N = qx.shape[0], qw.shape[0]
     acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
-    wq.wq_debug_gemm_s32(dev(qx), bits, dev(qw), K, acc)
+    ws = wq.alloc_workspace(M, K, N, bits)
+    wq.wq_debug_gemm_s32(dev(qx), bits, dev(qw), K, acc, ws)
     return host(acc)
+
+
+def unpack_codes(packed):
+    """Packed int4 codes [M][K/2] (low nibble = even k, two's complement) -> int8 [M][K]."""
+    p = np.asarray(packed, np.uint8)
+    lo = (p & 0xF).astype(np.int16)
+    hi = (p >> 4).astype(np.int16)
+    lo -= (lo >= 8) * 16
+    hi -= (hi >= 8) * 16
+    out = np.empty((p.shape[0], p.shape[1] * 2), np.int8)
+    out[:, 0::2] = lo
+    out[:, 1::2] = hi
+    return out
+
+
+def _round256(n):
+    return (n + 255) // 256 * 256
+
+
+def gpu_linear_debug(x, cinv, sid, alpha, beta, step, bits, qw, s_w, bias, rows=None):
+    """wq_debug_linear_s32 (the fused linear with its accumulators also written).
+    Returns host copies of (y bf16 bits, acc int32, workspace codes int8 [.][K],
+    workspace token scales), restricted to `rows` when given."""
+    M, K = x.shape
+    N = qw.shape[0]
+    t = lambda a: None if a is None else (a if isinstance(a, torch.Tensor) else dev(a))
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    ws = wq.alloc_workspace(M, K, N, bits)
+    wq.wq_debug_linear_s32(t(x), t(cinv), t(sid), t(alpha), t(beta), step, bits, t(qw), t(s_w),
+                           t(bias), y, acc, ws)
+    codes = ws[: M * K].view(torch.int8).view(M, K)
+    off = _round256(M * K)
+    s_tok = ws[off: off + 4 * M].view(torch.float32)
+    if rows is not None:
+        idx = torch.as_tensor(np.asarray(rows), device="cuda", dtype=torch.long)
+        y, acc, codes, s_tok = y[idx], acc[idx], codes[idx], s_tok[idx]
+    return host(y.view(torch.int16), np.uint16), host(acc), host(codes), host(s_tok)
+
+
+def gpu_gemm_w4ax(qx, s_tok, bits, K, sid, beta, step, qw, s_w, bias):
+    """wq_gemm_w4ax on codes qx (int8 [M][K] or packed int4 [M][K/2])."""
+    M, N = qx.shape[0], qw.shape[0]
+    T, S_, _ = beta.shape
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    wq.wq_gemm_w4ax(dev(qx), dev(s_tok), bits, K, dev(sid), dev(beta), S_, T, step, dev(qw),
+                    dev(s_w), None if bias is None else dev(bias), y)
+    return host(y.view(torch.int16), np.uint16)
 
 
 def gpu_act_quant_static(x, cinv, sid, thr, gain, step, bits):

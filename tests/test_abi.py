@@ -79,7 +79,14 @@ def test_other_entry_points_reject_on_host(lib):
     assert lib.wq_act_quant(FAKE, 8, 200, None, FAKE, FAKE, 3, 1, 0, 8, FAKE, FAKE, None) == 2
     assert lib.wq_pack_int4(FAKE, None, 16, 96, FAKE, FAKE, None) == 2
     assert lib.wq_pack_int4(None, None, 16, 128, FAKE, FAKE, None) == 1
-    assert lib.wq_debug_gemm_s32(FAKE, 8, FAKE, 16, 24, 128, FAKE, None) == 2
+    assert lib.wq_debug_gemm_s32(FAKE, 8, FAKE, 16, 24, 128, FAKE, None, 0, None) == 2
+    assert lib.wq_debug_gemm_s32(FAKE, 5, FAKE, 16, 32, 128, FAKE, None, 0, None) == 4
+    assert lib.wq_debug_gemm_s32(FAKE, 8, FAKE, 16, 32, 128, None, None, 0, None) == 1
+    # 16 tokens x 128 channels x K = 4096: K is split, so the scratch is required
+    assert lib.wq_debug_gemm_s32(FAKE, 8, FAKE, 16, 128, 4096, FAKE, None, 0, None) == 1
+    assert lib.wq_debug_gemm_s32(FAKE, 8, FAKE, 16, 128, 4096, FAKE, FAKE + 16, 1 << 20,
+                                 None) == 3
+    assert lib.wq_debug_gemm_s32(FAKE, 8, FAKE, 16, 128, 4096, FAKE, FAKE, 64, None) == 4
     assert lib.wq_gemm_w4ax(FAKE, FAKE, 4, 16, 128, 32, FAKE, None, 3, 2, 2, FAKE, FAKE, None,
                             FAKE, None) == 4
     assert lib.wq_channel_scale(None, 4, FAKE, 4, 128, FAKE, FAKE, None) == 1
@@ -163,3 +170,52 @@ def test_every_pointer_is_checked_for_alignment(lib):
     for i in (0, 2, 5, 6):
         bad = list(cs); bad[i] = MIS
         assert lib.wq_channel_scale(*bad) == 3, i
+
+
+def _gelu(lib, **kw):
+    # (x, M, K, N, cinv, sid, alpha, beta, S, T, step, bits, qw, s_w, bias, cinv_next,
+    #  thr_next, gain_next, bits_next, codes, s_next, h, ws, ws_bytes, st)
+    a = dict(x=FAKE, M=64, K=256, N=256, cinv=FAKE, sid=FAKE, alpha=FAKE, beta=FAKE, S=3, T=1,
+             step=0, bits=8, qw=FAKE, s_w=FAKE, bias=FAKE, cinv_next=FAKE, thr=FAKE, gain=FAKE,
+             bits_next=8, codes=FAKE, s_next=FAKE, h=None, ws=FAKE, ws_bytes=1 << 30, st=None)
+    a.update(kw)
+    return lib.wq_linear_gelu_quant(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(bits_next=6), 4), (dict(bits=5), 4), (dict(thr=None), 1), (dict(gain=None), 1),
+    (dict(s_next=None), 1), (dict(codes=None), 1), (dict(codes=MIS), 3), (dict(h=MIS), 3),
+    (dict(cinv_next=MIS), 3), (dict(s_next=MIS), 3), (dict(N=250), 2), (dict(ws_bytes=10), 4),
+    (dict(step=1), 4), (dict(M=0, x=None, sid=None, codes=None, s_next=None), 0),
+])
+def test_gelu_quant_rejects_bad_arguments_on_host(lib, kw, code):
+    assert _gelu(lib, **kw) == code
+
+
+def test_debug_linear_rejects_on_host(lib):
+    # (x, M, K, N, cinv, sid, alpha, beta, S, T, step, bits, qw, s_w, bias, y, acc, ws, ws_bytes, st)
+    args = [FAKE, 64, 256, 256, FAKE, FAKE, FAKE, FAKE, 3, 1, 0, 8, FAKE, FAKE, FAKE, FAKE, FAKE,
+            FAKE, 1 << 30, None]
+    bad = list(args); bad[16] = None
+    assert lib.wq_debug_linear_s32(*bad) == 1        # no accumulator buffer
+    bad = list(args); bad[16] = MIS
+    assert lib.wq_debug_linear_s32(*bad) == 3
+    bad = list(args); bad[11] = 2
+    assert lib.wq_debug_linear_s32(*bad) == 4
+
+
+def test_stall_hook_needs_a_limit(lib):
+    assert lib.wq_debug_inject_stall(1, 0) == 4
+
+
+def test_noalloc_scratch_limit_is_exact(lib):
+    """wq_workspace_bytes(M, K, N, 8) <= 16 MiB is the rule: at K = N = 4096 the
+    largest M is 4092 (16 MiB exactly); M = 4093 is rejected before any launch."""
+    limit = 16 << 20
+    assert wq.wq_workspace_bytes(4092, 4096, 4096, 8) == limit
+    assert wq.wq_workspace_bytes(4093, 4096, 4096, 8) > limit
+    args = lambda m: (FAKE, m, 4096, 4096, None, FAKE, FAKE, None, 3, 1, 0, FAKE, FAKE, None,
+                      FAKE, None)
+    assert wq.STATUS[lib.wq_linear_w4a8_noalloc(*args(4093))] == "WQ_ERR_SCRATCH"
+    # 4092 passes the size check; without a GPU the next step (finding the device) fails
+    assert wq.STATUS[lib.wq_linear_w4a8_noalloc(*args(4092))] != "WQ_ERR_SCRATCH"

@@ -113,7 +113,15 @@ def test_every_other_wrapper_marshals_in_header_order(fake):
                              a["qw"], a["s_w"], a["bias"], a["y"], stream=0)
     wq.wq_linear_w4a8_noalloc(a["x"], a["cinv"], a["sid"], a["alpha"], a["beta"], STEP, a["qw"],
                               a["s_w"], a["bias"], a["y"], stream=0)
-    wq.wq_debug_gemm_s32(a["qx"], 8, a["qw"], K, a["acc"], stream=0)
+    wq.wq_debug_gemm_s32(a["qx"], 8, a["qw"], K, a["acc"], a["ws"], stream=0)
+    wq.wq_debug_linear_s32(a["x"], a["cinv"], a["sid"], a["alpha"], a["beta"], STEP, 4, a["qw"],
+                           a["s_w"], a["bias"], a["y"], a["acc"], a["ws"], stream=0)
+    codes, s_next, h = DevT((M, N), torch.int8), DevT((M,), F32), DevT((M, N), BF16)
+    cinv_n, gain_n = DevT((N,), F32), DevT((T, S), F32)
+    wq.wq_linear_gelu_quant(a["x"], a["cinv"], a["sid"], a["alpha"], a["beta"], STEP, 8, a["qw"],
+                            a["s_w"], a["bias"], cinv_n, a["thr"], gain_n, 4, codes, s_next, h,
+                            a["ws"], stream=0)
+    wq.wq_debug_inject_stall(True, 50000)
     got = dict((n, args) for n, args in fake.calls[:2])
     assert got["wq_channel_scale"] == (p(xc), 7, p(W), N, K, p(c), p(a["cinv"]), 0)
     assert got["wq_pack_int4"] == (p(W), p(c), N, K, p(a["qw"]), p(a["s_w"]), 0)
@@ -121,7 +129,8 @@ def test_every_other_wrapper_marshals_in_header_order(fake):
     assert [n for n, _ in fake.calls[2:]] == [
         "wq_act_quant", "wq_act_quant", "wq_act_quant_static", "wq_gemm_w4ax", "wq_linear_w4a4",
         "wq_linear_w4ax_static", "wq_linear_w4ax_single", "wq_linear_w4a8_noalloc",
-        "wq_debug_gemm_s32"]
+        "wq_debug_gemm_s32", "wq_debug_linear_s32", "wq_linear_gelu_quant",
+        "wq_debug_inject_stall"]
     assert rest[0] == (p(a["x"]), M, K, p(a["cinv"]), p(a["sid"]), p(a["alpha"]), S, T, STEP, 8,
                        p(a["qx"]), p(a["s_tok"]), 0)
     assert rest[1] == (p(a4["x"]), M, K, None, p(a4["sid"]), p(a4["alpha"]), S, T, STEP, 4,
@@ -142,7 +151,45 @@ def test_every_other_wrapper_marshals_in_header_order(fake):
     assert rest[7] == (p(a["x"]), M, K, N, p(a["cinv"]), p(a["sid"]), p(a["alpha"]),
                        p(a["beta"]), S, T, STEP, p(a["qw"]), p(a["s_w"]), p(a["bias"]),
                        p(a["y"]), 0)
-    assert rest[8] == (p(a["qx"]), 8, p(a["qw"]), M, N, K, p(a["acc"]), 0)
+    assert rest[8] == (p(a["qx"]), 8, p(a["qw"]), M, N, K, p(a["acc"]), p(a["ws"]),
+                       wq_ws_bytes(8), 0)
+    assert rest[9] == (p(a["x"]), M, K, N, p(a["cinv"]), p(a["sid"]), p(a["alpha"]),
+                       p(a["beta"]), S, T, STEP, 4, p(a["qw"]), p(a["s_w"]), p(a["bias"]),
+                       p(a["y"]), p(a["acc"]), p(a["ws"]), wq_ws_bytes(8), 0)
+    assert rest[10] == (p(a["x"]), M, K, N, p(a["cinv"]), p(a["sid"]), p(a["alpha"]),
+                        p(a["beta"]), S, T, STEP, 8, p(a["qw"]), p(a["s_w"]), p(a["bias"]),
+                        p(cinv_n), p(a["thr"]), p(gain_n), 4, p(codes), p(s_next), p(h),
+                        p(a["ws"]), wq_ws_bytes(8), 0)
+    assert rest[11] == (1, 50000)
+
+
+@pytest.mark.parametrize("which,bad", [
+    ("codes", DevT((M, N - 16), torch.int8)),     # codes smaller than M x N
+    ("codes", DevT((M, N), torch.int32)),         # one int8 byte per code
+    ("s_next", DevT((M - 1,), F32)),
+    ("h", DevT((M, N), F32)),                     # h is bf16
+    ("cinv_n", DevT((N - 16,), F32)),             # the next linear's channel scale covers N
+    ("gain_n", DevT((T, S - 1), F32)),
+])
+def test_gelu_quant_rejects_a_bad_tensor_before_the_call(fake, which, bad):
+    a = tensors()
+    t = dict(codes=DevT((M, N), torch.int8), s_next=DevT((M,), F32), h=DevT((M, N), BF16),
+             cinv_n=DevT((N,), F32), gain_n=DevT((T, S), F32))
+    t[which] = bad
+    with pytest.raises((ValueError, TypeError)):
+        wq.wq_linear_gelu_quant(a["x"], a["cinv"], a["sid"], a["alpha"], a["beta"], STEP, 8,
+                                a["qw"], a["s_w"], a["bias"], t["cinv_n"], a["thr"], t["gain_n"],
+                                8, t["codes"], t["s_next"], t["h"], a["ws"], stream=0)
+    assert fake.calls == []
+
+
+def test_debug_linear_checks_the_accumulator_buffer(fake):
+    a = tensors()
+    for bad in (DevT((M, N - 16), torch.int32), DevT((M, N), F32)):
+        with pytest.raises((ValueError, TypeError)):
+            wq.wq_debug_linear_s32(a["x"], a["cinv"], a["sid"], a["alpha"], a["beta"], STEP, 8,
+                                   a["qw"], a["s_w"], a["bias"], a["y"], bad, a["ws"], stream=0)
+    assert fake.calls == []
 
 
 def _linear(a):
@@ -185,7 +232,7 @@ def test_codes_buffer_is_sized_by_the_code_width(fake):
         wq.wq_gemm_w4ax(a["qx"], a["s_tok"], 8, K, a["sid"], None, S, T, STEP, a["qw"],
                         a["s_w"], None, a["y"], 0)
     with pytest.raises(ValueError):           # acc [M][N+16] needs N+16 weight rows
-        wq.wq_debug_gemm_s32(a["qx"], 4, a["qw"], K, DevT((M, N + 16), torch.int32), 0)
+        wq.wq_debug_gemm_s32(a["qx"], 4, a["qw"], K, DevT((M, N + 16), torch.int32), stream=0)
     assert len(fake.calls) == 1
 
 

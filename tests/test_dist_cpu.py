@@ -60,10 +60,10 @@ def test_gemm_traffic_tracks_the_kernel_source(tmp_path, monkeypatch):
     import hashlib
     src = tmp_path / "k.cuh"
     src.write_bytes(b"kernel v1")
-    prof = tmp_path / "traffic.md"
+    prof = tmp_path / "gemm_traffic_block2048_w4a8.md"
     digest = hashlib.sha256(b"kernel v1").hexdigest()
     prof.write_text(f"# t\n\n    traffic_bytes_per_launch: 1234\n    source_sha256: {digest}\n")
-    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(prof))
+    monkeypatch.setattr(bench, "traffic_file", lambda w: str(tmp_path / f"gemm_traffic_{w}.md"))
     monkeypatch.setattr(bench, "GEMM_SOURCES", [str(src)])
     assert bench.gemm_traffic("block2048_w4a8") == 1234
     assert bench.gemm_traffic("block4096_w4a8_t10") is None   # no capture for that workload
@@ -77,9 +77,9 @@ def test_gemm_traffic_ignores_host_side_edits(tmp_path, monkeypatch):
     src = tmp_path / "g.cuh"
     src.write_text(f"__global__ void k() {{}}\n{marker}\nint host_a();\n")
     digest = bench.gemm_device_source_hash([str(src)])
-    prof = tmp_path / "traffic.md"
+    prof = tmp_path / "gemm_traffic_block2048_w4a8.md"
     prof.write_text(f"    traffic_bytes_per_launch: 77\n    source_sha256: {digest}\n")
-    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(prof))
+    monkeypatch.setattr(bench, "traffic_file", lambda w: str(tmp_path / f"gemm_traffic_{w}.md"))
     monkeypatch.setattr(bench, "GEMM_SOURCES", [str(src)])
     assert bench.gemm_traffic("block2048_w4a8") == 77
     src.write_text(f"__global__ void k() {{}}\n{marker}\nint host_b();\n")   # host side only

@@ -15,8 +15,8 @@ import activation_quantized_gemm_wq_b200 as wq
 from activation_quantized_gemm_wq_b200 import synth as S
 
 import oracle_pins as P
-from gpu_util import (dev, gpu_act_quant, gpu_gemm_s32, gpu_linear, gpu_prep, host,
-                      within_tolerance)
+from gpu_util import (dev, gpu_act_quant, gpu_gemm_s32, gpu_gemm_w4ax, gpu_linear,
+                      gpu_linear_debug, gpu_prep, host, unpack_codes, within_tolerance)
 
 pytestmark = pytest.mark.gpu
 
@@ -50,9 +50,12 @@ def test_channel_scale_and_pack_bit_exact(oracle, wl, layer):
 
 # ------------------------------------------------------------------ activation codes
 
-# M >= 1024 with K <= 4096 takes the one-warp-per-row kernel, the rest the CTA-per-rows one
+# M >= 512 with K in {2048, 4096, 8192, 16384} takes the staged-rows kernel (the last
+# round of rows ragged here), other M >= 1024 with K <= 4096 the one-warp-per-row
+# kernel, the rest the CTA-per-rows one
 AQ_SHAPES = [(64, 256), (37, 384), (300, 2048), (16, 8192), (9, 16384), (3, 32768), (1, 128),
-             (1100, 256), (1030, 4096), (2048, 2048), (1050, 8192), (1025, 32768)]
+             (1100, 256), (1030, 4096), (2048, 2048), (1050, 8192), (1025, 32768),
+             (513, 2048), (777, 16384), (600, 8192), (1111, 1024)]
 
 
 @pytest.mark.parametrize("bits", [8, 4])
@@ -101,8 +104,10 @@ def test_act_quant_near_ties(oracle, bits, qmax):
 
 # ------------------------------------------------------------------ int32 core
 
+# the last four split K over several CTAs (few output tiles), as the fused linear does
 GEMM_SHAPES = [(1, 16, 128), (16, 144, 256), (17, 128, 512), (64, 256, 256), (100, 272, 384),
-               (128, 128, 128), (129, 400, 256), (300, 384, 512), (513, 128, 1024)]
+               (128, 128, 128), (129, 400, 256), (300, 384, 512), (513, 128, 1024),
+               (16, 128, 4096), (40, 512, 2048), (100, 1024, 1024), (256, 2048, 2048)]
 
 
 @pytest.mark.parametrize("bits", [8, 4])
@@ -132,23 +137,28 @@ def test_gemm_s32_extreme_values(oracle):
 # ------------------------------------------------------------------ the fused linear
 
 def _check_linear(oracle, x, sid, L, bits, step, rows=None, use_gpu_prep=True):
+    """One fused linear through wq_debug_linear_s32 (the product's two launches, with
+    the accumulators also written) against the oracle on `rows` (all by default):
+    the workspace's codes and token scales bit for bit (4-bit codes are kept one per
+    byte there), the int32 accumulators bit for bit, y within the tolerance."""
     c_ref, cinv_ref = oracle.channel_scale(L.x_cal, L.W)
     qw_ref, sw_ref = oracle.pack_int4(L.W, c_ref)
     if use_gpu_prep:
         _, cinv_d, qw_d, sw_d = gpu_prep(L.W, L.x_cal)
     else:
         cinv_d, qw_d, sw_d = cinv_ref, qw_ref, sw_ref
-    y = gpu_linear(x, cinv_d, sid, L.alpha, L.beta, step, bits, qw_d, sw_d, L.bias)
     if rows is None:
         rows = np.arange(x.shape[0])
+    y, acc, codes, s_tok = gpu_linear_debug(x, cinv_d, sid, L.alpha, L.beta, step, bits, qw_d,
+                                            sw_d, L.bias, rows=rows)
     y_ref, q_ref, s_ref, acc_ref = oracle.linear(x[rows], cinv_ref, sid[rows], L.alpha, L.beta,
                                                  step, bits, qw_ref, sw_ref, L.bias)
-    ok, worst = within_tolerance(y[rows], y_ref)
+    assert np.array_equal(_f32bits(s_tok), _f32bits(s_ref)), "token scales"
+    q_ref8 = q_ref if bits == 8 else unpack_codes(q_ref)
+    assert np.array_equal(codes, q_ref8), "activation codes"
+    assert np.array_equal(acc, acc_ref), "int32 accumulators"
+    ok, worst = within_tolerance(y, y_ref)
     assert ok, f"bf16 outputs outside tolerance (worst error/allowance {worst:.3f})"
-    # the integer path underneath, bit for bit
-    q, s = gpu_act_quant(x[rows], cinv_ref, sid[rows], L.alpha, step, bits)
-    assert np.array_equal(_f32bits(s), _f32bits(s_ref))
-    assert np.array_equal(q.view(np.uint8), q_ref.view(np.uint8))
     return worst
 
 
@@ -167,13 +177,21 @@ def test_linear_ragged_all_elements(oracle, M, K, N, bits):
     wl = S.custom(f"lin{M}x{K}x{N}", K, N, tuple(r for r in rows if r[1] > 0), act_bits=bits, T=3)
     L = S.layer_inputs(wl, 0)
     x = S.activations(wl, 0, step=2)
-    _check_linear(oracle, x, S.stream_ids(wl), L, bits, 2)
+    sid = S.stream_ids(wl)
+    _check_linear(oracle, x, sid, L, bits, 2)
+    # the debug view is the product path: the plain call gives the same y bit for bit
+    _, cinv, qw, s_w = gpu_prep(L.W, L.x_cal)
+    y_plain = gpu_linear(x, cinv, sid, L.alpha, L.beta, 2, bits, qw, s_w, L.bias)
+    y_dbg = gpu_linear_debug(x, cinv, sid, L.alpha, L.beta, 2, bits, qw, s_w, L.bias)[0]
+    assert np.array_equal(y_plain, y_dbg)
 
 
-def test_linear_many_streams_and_optional_inputs(oracle):
-    """S = 7 (> 4: per-element table reads), shuffled ids, no bias, no beta, no cinv."""
-    g = np.random.default_rng(5)
-    M, K, N, T, Sn = 200, 384, 272, 5, 7
+@pytest.mark.parametrize("Sn", [4, 6, 7])
+def test_linear_many_streams_and_optional_inputs(oracle, Sn):
+    """S = 4 (the largest per-lane table), 6 and 7 (> 4: per-element table reads),
+    shuffled ids, no bias, no beta, no cinv."""
+    g = np.random.default_rng(5 + Sn)
+    M, K, N, T = 200, 384, 272, 5
     wl = S.custom("many", K, N, ((0, M),), act_bits=8, T=T)
     L = S.layer_inputs(wl, 0)
     x = S.activations(wl, 0)
@@ -204,6 +222,9 @@ def test_linear_empty_batch():
 
 
 # ------------------------------------------------------------------ full-size shapes, sampled
+# Every layer of both blocks at full size (K up to 16384, M = 4288 and 8512), through
+# the same two launches the benchmark times: codes, token scales and int32
+# accumulators of the sampled token rows bit for bit, y within the tolerance.
 
 def _sample_rows(wl, n_random, seed=0):
     """Every stream's first and last rows, the batch's last row, and random rows."""
@@ -228,7 +249,7 @@ def test_block2048_full_size_sampled_rows(oracle, wl, step, layer):
 
 
 @pytest.mark.parametrize("wl", [S.BLOCK4096_A8, S.BLOCK4096_A4], ids=["w4a8", "w4a4"])
-@pytest.mark.parametrize("layer", [0, 3])
+@pytest.mark.parametrize("layer", [0, 1, 2, 3])
 def test_block4096_full_size_sampled_rows(oracle, wl, layer):
     L = S.layer_inputs(wl, layer)
     step = 5
@@ -246,3 +267,44 @@ def test_small_m_weight_streaming(oracle, M, bits):
         x = S.activations(wl, layer, 0)
         rows = None if M <= 64 else np.arange(0, M, 7)
         _check_linear(oracle, x, S.stream_ids(wl), L, bits, 0, rows=rows)
+
+
+# ------------------------------------------------------------------ GEMM-only entry point
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("M,K,N", [(1, 256, 16), (300, 512, 384), (520, 256, 2048),
+                                   (33, 1024, 144), (4288, 2048, 2048)])
+def test_gemm_w4ax_against_oracle(oracle, M, K, N, bits):
+    """wq_gemm_w4ax on the oracle's codes and token scales: int8 codes, or packed
+    int4 codes (the packed-activation mainloop, which unpacks them per tile)."""
+    rows_ = ((0, M - M // 4 - M // 8), (1, M // 8), (2, M // 4))
+    wl = S.custom(f"gemm{M}x{K}x{N}", K, N, tuple(r for r in rows_ if r[1] > 0), act_bits=bits,
+                  T=3)
+    L = S.layer_inputs(wl, 0)
+    x = S.activations(wl, 0, step=1)
+    sid = S.stream_ids(wl)
+    c, cinv = oracle.channel_scale(L.x_cal, L.W)
+    qw, s_w = oracle.pack_int4(L.W, c)
+    qx, s_tok = oracle.act_quant(x, cinv, sid, L.alpha, 1, bits)
+    y = gpu_gemm_w4ax(qx, s_tok, bits, K, sid, L.beta, 1, qw, s_w, L.bias)
+    rows = np.arange(M) if M <= 600 else _sample_rows(wl, 24)
+    acc = oracle.gemm_s32(qx[rows], bits, qw, K)
+    y_ref = oracle.epilogue(acc, s_tok[rows], s_w, L.bias, L.beta, sid[rows], 1)
+    ok, worst = within_tolerance(y[rows], y_ref)
+    assert ok, worst
+
+
+
+@pytest.mark.parametrize("M", [16, 256])
+@pytest.mark.parametrize("parent,layer", [(p, i) for p in (S.BLOCK2048_A8, S.BLOCK4096_A8)
+                                          for i in range(4)],
+                         ids=[f"{p}_{n}" for p in ("h2048", "h4096")
+                              for n in ("qkv", "attn_out", "mlp_up", "mlp_down")])
+def test_small_m_every_weight_shape(oracle, parent, layer, M):
+    """Every small-M weight shape at 16 and 256 action tokens: the split of K over
+    CTAs (int32 partial tiles summed through the workspace) gives the exact sums."""
+    wl = S.small_m(parent, M, "action", 8)
+    L = S.layer_inputs(wl, layer)
+    x = S.activations(wl, layer, 0)
+    _check_linear(oracle, x, S.stream_ids(wl), L, 8, 0,
+                  rows=None if M <= 16 else np.arange(0, M, 5))

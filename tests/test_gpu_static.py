@@ -39,7 +39,7 @@ def _tables(g, T, Sn, x, cinv, qmax):
 
 @pytest.mark.parametrize("bits,qmax", [(8, 127), (4, 7)])
 @pytest.mark.parametrize("M,K", [(64, 256), (300, 2048), (16, 8192), (3, 32768), (37, 384),
-                                 (1200, 2048)])
+                                 (1200, 2048), (1030, 4096), (515, 8192), (601, 16384)])
 def test_act_quant_static_bit_exact(oracle, M, K, bits, qmax):
     g = np.random.default_rng(M * 13 + K)
     wl = S.custom(f"st{M}x{K}", K, 16, ((0, M),), act_bits=bits, T=3)
@@ -55,7 +55,8 @@ def test_act_quant_static_bit_exact(oracle, M, K, bits, qmax):
 
 
 @pytest.mark.parametrize("bits,qmax", [(8, 127), (4, 7)])
-@pytest.mark.parametrize("M,K,N", [(300, 512, 384), (16, 2048, 1024), (1, 256, 16)])
+@pytest.mark.parametrize("M,K,N", [(300, 512, 384), (16, 2048, 1024), (1, 256, 16),
+                                   (700, 4096, 256)])
 def test_linear_static_matches_oracle(oracle, M, K, N, bits, qmax):
     g = np.random.default_rng(M + K + N)
     rows = ((0, M - M // 4), (2, M // 4))

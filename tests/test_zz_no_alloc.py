@@ -5,9 +5,11 @@ the library's fixed 16 MiB scratch instead of a caller workspace.
 
 Checked through the C ABI against wq_linear_w4a8 (which uses a caller
 workspace) on two calls in a row with different inputs, so stale scratch
-contents from the first call cannot leak into the second.  This file is
-collected last, and it needs nothing from the other test files, so it passes
-alone in a fresh process as well as after them."""
+contents from the first call cannot leak into the second.  Both run the same two
+kernels on the same inputs, so their outputs must be equal bit for bit; the
+first call is also compared with the CPU oracle, within the tolerance the other
+tests use.  This file is collected last, and it needs nothing from the other test
+files, so it passes alone in a fresh process as well as after them."""
 import numpy as np
 import pytest
 import torch
@@ -31,6 +33,20 @@ def _within_tolerance(y, ref):
     """max |y - y_ref| <= 2^-7 |y_ref| + 1e-3 rms(y_ref), element-wise."""
     rms = np.sqrt(np.mean(ref ** 2))
     return bool(np.all(np.abs(y - ref) <= 2.0 ** -7 * np.abs(ref) + 1e-3 * rms))
+
+
+def _oracle_y(wl, x_host, step):
+    """The oracle's y (as float64) for the first linear of `wl` on activations x_host."""
+    from oracle import Oracle
+    orc = Oracle()
+    L = S.layer_inputs(wl, 0)
+    c, cinv = orc.channel_scale(L.x_cal, L.W)
+    qw, s_w = orc.pack_int4(L.W, c)
+    rows = np.arange(x_host.shape[0]) if x_host.shape[0] <= 512 else \
+        np.arange(0, x_host.shape[0], 61)
+    y = orc.linear(x_host[rows], cinv, S.stream_ids(wl)[rows], L.alpha, L.beta, step, 8, qw,
+                   s_w, L.bias)[0]
+    return rows, (y.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def _prepared(wl):
@@ -61,13 +77,18 @@ def test_noalloc_matches_workspace_linear_twice(wl):
     ws = wq.alloc_workspace(M, K, N, 8)
     step = wl.T - 1
     for call in range(2):  # two calls in a row, different activations each time
-        x = _dev(S.activations(wl, 0, step=call % wl.T, seed=call))
+        x_host = S.activations(wl, 0, step=call % wl.T, seed=call)
+        x = _dev(x_host)
         y_ref = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
         y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
         wq.wq_linear_w4a8(x, cinv, sid, alpha, beta, step, qw, s_w, bias, y_ref, ws)
         wq.wq_linear_w4a8_noalloc(x, cinv, sid, alpha, beta, step, qw, s_w, bias, y)
         torch.cuda.synchronize()
-        assert _within_tolerance(_f64(y), _f64(y_ref)), f"call {call} differs"
+        # the same kernels on the same inputs: equal bit for bit
+        assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16)), f"call {call} differs"
+        if call == 0:  # and right, as the oracle computes it
+            rows, y_orc = _oracle_y(wl, x_host, step)
+            assert _within_tolerance(_f64(y)[rows], y_orc), "differs from the oracle"
     assert wq.wq_device_status() == ("WQ_OK", 0)
 
 
