@@ -60,6 +60,9 @@ def parse():
                    help=f"default {DEFAULT_WORKLOAD} (--sequence: every block)")
     p.add_argument("--no-companion", action="store_true",
                    help="skip the W4A4 run reported beside a W4A8 headline")
+    p.add_argument("--layers", default="",
+                   help="comma-separated linear indices to run (default: every linear of the "
+                        "block); a smaller case for profiling one kernel")
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-graph", action="store_true",
@@ -237,12 +240,14 @@ def activation_sets(wl):
     return in_bytes, n_sets
 
 
-def workload_config(wl, world):
+def workload_config(wl, world, layers=""):
     """The `config` object of the JSON line, the same for the GPU and reference arms."""
     in_bytes, n_sets = activation_sets(wl)
+    chosen = [int(i) for i in layers.split(",")] if layers else range(len(wl.linears))
     return {
-        "workload": wl.name,
-        "linears": [f"{l.name} {l.K}->{l.N}" for l in wl.linears],
+        "workload": wl.name if not layers else f"{wl.name} (linears {layers} only)",
+        "linears": [f"{wl.linears[i].name} {wl.linears[i].K}->{wl.linears[i].N}"
+                    for i in chosen],
         "M": wl.M,
         "token_rows": {"video": dict(wl.rows).get(0, 0), "proprio": dict(wl.rows).get(1, 0),
                        "action": dict(wl.rows).get(2, 0)},
@@ -301,7 +306,8 @@ def measure_workload(args, wl, wq, torch, world, local, dev):
     """Time one workload's step (every linear of the block, fused calls, one CUDA graph
     per step) and its dominant kernel; returns the fields of the JSON line."""
     _, n_sets = activation_sets(wl)
-    layers = [Layer(wl, i, n_sets, wq, torch, dev) for i in range(len(wl.linears))]
+    chosen = [int(i) for i in args.layers.split(",")] if args.layers else range(len(wl.linears))
+    layers = [Layer(wl, i, n_sets, wq, torch, dev) for i in chosen]
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     T = wl.T
@@ -486,7 +492,7 @@ def run_gpu(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "int8",
         "data": DATA,
-        "config": workload_config(wl, world),
+        "config": workload_config(wl, world, args.layers),
         "roofline": res["roofline"],
         "timing": res["timing"],
         "clocks": res["clocks"],
