@@ -381,6 +381,7 @@ wq_status wq_linear_gelu_quant(const wq_bf16* x, int M, int K, int N, const floa
       (cinv_next && !aligned16(cinv_next)) || (h && !aligned16(h)))
     return WQ_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  WQ_TRY(from_cuda(wq::ensure_gelu_table(st)));
   const Workspace w = carve(workspace, M, K, N);
   WQ_TRY(quantize_into(w, x, M, K, cinv, stream_id, alpha, S, step, act_bits, nullptr, st));
   const wq::EpilogueArgs ep{w.s_tok, stream_id, s_w, bias, beta, S, step};

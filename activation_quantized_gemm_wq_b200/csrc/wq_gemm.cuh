@@ -36,7 +36,36 @@
 #include "wq_quant.cuh"
 
 namespace wq {
+
+// bf16(GELU(y)) for every bf16 y with 2^-10 <= |y| < 16 (exponent field 117..130),
+// indexed [sign][exponent - 117][mantissa]: the GELU-and-quantize epilogue looks
+// values up here instead of evaluating erfcf for each element.  Built on the GPU
+// with the same fp32 arithmetic the epilogue uses for the values outside that range
+// (gelu_table_kernel), so a lookup returns exactly what the evaluation would.
+constexpr int kGeluTabExp0 = 117, kGeluTabExps = 14;
+__device__ uint16_t g_gelu_tab[2 * kGeluTabExps * 128];
+
 namespace {
+
+__global__ void gelu_table_kernel() {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= 2 * kGeluTabExps * 128) return;
+  const uint32_t sign = static_cast<uint32_t>(i / (kGeluTabExps * 128));
+  const uint32_t e = static_cast<uint32_t>((i / 128) % kGeluTabExps + kGeluTabExp0);
+  const uint32_t bits = (sign << 15) | (e << 7) | static_cast<uint32_t>(i % 128);
+  const float y = __uint_as_float(bits << 16);
+  g_gelu_tab[i] = __bfloat16_as_ushort(__float2bfloat16_rn(gelu_f32(y)));
+}
+
+// h = bf16(GELU(y)) for a bf16 y, by table where it covers y.
+__device__ __forceinline__ uint16_t gelu_bf16_bits(uint16_t ybits) {
+  const uint32_t e = (ybits >> 7) & 0xFFu;
+  if (e - kGeluTabExp0 < static_cast<uint32_t>(kGeluTabExps))
+    return __ldg(&g_gelu_tab[(ybits >> 15) * (kGeluTabExps * 128) + (e - kGeluTabExp0) * 128 +
+                             (ybits & 0x7Fu)]);
+  return __bfloat16_as_ushort(
+      __float2bfloat16_rn(gelu_f32(__uint_as_float(static_cast<uint32_t>(ybits) << 16))));
+}
 
 struct TileArgs {
   void* out;  // y [M][N] bf16, or acc [M][N] int32
@@ -88,9 +117,18 @@ __device__ __forceinline__ void split_range(int num_k, int splits, int sp, int& 
 // tile the MMA reads.  No codes go through HBM.
 // EPI > 0: the up-projection of an FFN whose epilogue emits the down-projection's
 // activation codes (qmax 127 for EPI 8, 7 for EPI 4) instead of y.
-template <int BN_, int ACT_BITS_, int QBITS_ = 0, int EPI_ = 0>
+// PAIR: two CTAs (a cluster) share one tile of 256 output channels x BN tokens
+// through the pair MMA (tcgen05 cta_group::2): each CTA unpacks its own 128
+// weight rows and loads half of the token rows (BN/2), rank 0 issues the MMAs, and
+// each CTA's TMEM receives the accumulators of its own 128 channels for all BN
+// tokens, which its epilogue writes.  Per SM this halves the activation tile's
+// copy and the tensor core's reads of it from shared memory.
+template <int BN_, int ACT_BITS_, int QBITS_ = 0, int EPI_ = 0, bool PAIR_ = false>
 struct Cfg {
   static constexpr int BN = BN_;
+  static constexpr bool PAIR = PAIR_;
+  static constexpr int BNX = PAIR ? BN / 2 : BN;  // token rows of the activation tile here
+  static constexpr int TILE_N = PAIR ? 256 : 128;  // output channels per work unit
   static constexpr int ACT_BITS = ACT_BITS_;
   static constexpr int QBITS = QBITS_;
   static constexpr int QMAX = QBITS == 4 ? 7 : 127;
@@ -100,6 +138,8 @@ struct Cfg {
                 "the single-kernel linear quantizes into the int8 mainloop, one token tile");
   static_assert(EPI == 0 || ((EPI == 8 || EPI == 4) && QBITS == 0 && ACT_BITS == 8),
                 "the GELU-and-quantize epilogue follows the int8-activation mainloop");
+  static_assert(!PAIR || (QBITS == 0 && BN == 256 && ACT_BITS == 8),
+                "CTA pairs serve the 256-token tiles of int8 activation codes");
   static constexpr int BM = 128;  // output channels per tile (MMA M)
   static constexpr int BK = 128;  // K elements per pipeline stage
   static constexpr int UNPACK_WARPS = ACT_BITS == 4 ? 8 : WQ_UNPACK_WARPS_A8;
@@ -120,8 +160,8 @@ struct Cfg {
 
   static constexpr int WP_BYTES = BM * BK / 2;                               // packed W
   static constexpr int WU_BYTES = BM * BK;                                   // int8 W
-  static constexpr int XS_BYTES = ACT_BITS == 8 ? BN * BK : BN * BK / 2;     // staged x
-  static constexpr int XU_BYTES = ACT_BITS == 8 ? 0 : BN * BK;               // int8 x (A4)
+  static constexpr int XS_BYTES = ACT_BITS == 8 ? BNX * BK : BNX * BK / 2;   // staged x
+  static constexpr int XU_BYTES = ACT_BITS == 8 ? 0 : BNX * BK;             // int8 x (A4)
   static constexpr int XB_BYTES = QBITS ? BN * BK * 2 : 0;                  // staged bf16 x
   static constexpr int STAGE_BYTES = WP_BYTES + (QBITS ? XB_BYTES : XS_BYTES);  // TMA bytes
   static constexpr int STAGE_SMEM = WP_BYTES + XS_BYTES + XB_BYTES;
@@ -266,16 +306,21 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int num_k = args.K / C::BK;
+  // work units: one per CTA, or one per CTA pair (rank 0 issues the pair's MMAs)
+  const uint32_t rank = C::PAIR ? cluster_ctarank() : 0u;
+  const int unit0 = C::PAIR ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+  const int ustep = C::PAIR ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&done[s], 1);
     }
-    for (int u = 0; u < C::NU; ++u) mbar_init(&ufull[u], C::UNPACK_WARPS);
+    // a pair's unpack and epilogue warps of both CTAs arrive on rank 0's barriers
+    for (int u = 0; u < C::NU; ++u) mbar_init(&ufull[u], C::UNPACK_WARPS * (C::PAIR ? 2 : 1));
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], C::EPI_WARPS);
+      mbar_init(&tempty[b], C::EPI_WARPS * (C::PAIR ? 2 : 1));
       mbar_init(&tokbar[b], C::EPI_WARPS);
     }
     mbar_init(qready, C::EPI_WARPS);
@@ -289,11 +334,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     tma_prefetch_desc(&tm_out);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (C::PAIR) {
+      tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (C::PAIR) cluster_sync();  // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   // Every CTA of this grid is resident (at most one per SM): the next kernel may
@@ -309,14 +360,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // the caller says so: start streaming them before waiting for it.
       uint32_t pre = 0;
       if (args.w_prefetch) {
-        for (int unit = blockIdx.x; unit < args.num_units && pre < C::NS; unit += gridDim.x) {
+        for (int unit = unit0; unit < args.num_units && pre < C::NS; unit += ustep) {
           int n_tile, m_tile, kb0, kb1;
           decode_tile(args, unit / args.splits, n_tile, m_tile);
           split_range(num_k, args.splits, unit % args.splits, kb0, kb1);
           for (int kb = kb0; kb < kb1 && pre < C::NS; ++kb, ++pre) {
             mbar_arrive_expect_tx(&full[pre], C::STAGE_BYTES);
             tma_load_2d(smem + C::OFF_WP + pre * C::WP_BYTES, &tm_w, &full[pre],
-                        kb * (C::BK / 2), n_tile * C::BM);
+                        kb * (C::BK / 2), n_tile * C::TILE_N + rank * C::BM);
           }
         }
       }
@@ -325,7 +376,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const int stall = blockIdx.x == 0 ? *reinterpret_cast<volatile int*>(&g_stall_kblock) : -1;
       uint32_t g = 0;
       bool ok = true;
-      for (int unit = blockIdx.x; ok && unit < args.num_units; unit += gridDim.x) {
+      for (int unit = unit0; ok && unit < args.num_units; unit += ustep) {
         int n_tile, m_tile, kb0, kb1;
         decode_tile(args, unit / args.splits, n_tile, m_tile);
         split_range(num_k, args.splits, unit % args.splits, kb0, kb1);
@@ -339,7 +390,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             }
             mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
             tma_load_2d(smem + C::OFF_WP + s * C::WP_BYTES, &tm_w, &full[s], kb * (C::BK / 2),
-                        n_tile * C::BM);
+                        n_tile * C::TILE_N + rank * C::BM);
           }
           if (static_cast<int>(g) == stall) {
             // leave the stage one copy short: its phase never completes
@@ -350,7 +401,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         kb * C::BK + 64, m_tile * C::BN);
           } else {
             tma_load_2d(smem + C::OFF_XS + s * C::XS_BYTES, &tm_x, &full[s],
-                        kb * (C::ACT_BITS == 8 ? C::BK : C::BK / 2), m_tile * C::BN);
+                        kb * (C::ACT_BITS == 8 ? C::BK : C::BK / 2),
+                        m_tile * C::BN + rank * C::BNX);
           }
         }
       }
@@ -369,13 +421,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // Per K block: one wait (its unpacked buffer; the unpack warps arrive there
     // only after the stage's TMA landed, which orders the activation tile too),
     // four MMAs, one commit (frees the stage and the unpacked buffer).
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(C::BN);
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_i8(C::BN, C::PAIR ? 256u : 128u);
       uint32_t g = 0;
       int b = 0;
       uint32_t ph_b = 0;
       bool ok = true;
-      for (int unit = blockIdx.x; ok && unit < args.num_units; unit += gridDim.x) {
+      for (int unit = unit0; ok && unit < args.num_units; unit += ustep) {
         int kb0, kb1;
         split_range(num_k, args.splits, unit % args.splits, kb0, kb1);
         if (!mbar_wait(&tempty[b], ph_b ^ 1u)) { ok = false; break; }
@@ -390,18 +442,25 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                : smem_u32(smem + C::OFF_XU + u * C::XU_BYTES);
           const uint32_t a_addr = smem_u32(smem + C::OFF_WU + u * C::WU_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < C::BK / 32; ++kk)
-            mma_i8_ss(d_tmem, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32),
-                      idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
-          mma_commit(&done[s]);
+          for (int kk = 0; kk < C::BK / 32; ++kk) {
+            const uint64_t ad = smem_desc_sw128(a_addr + kk * 32);
+            const uint64_t bd = smem_desc_sw128(b_addr + kk * 32);
+            const uint32_t acc = (kb != kb0 || kk != 0) ? 1u : 0u;
+            if constexpr (C::PAIR) mma_i8_ss_pair(d_tmem, ad, bd, idesc, acc);
+            else mma_i8_ss(d_tmem, ad, bd, idesc, acc);
+          }
+          if constexpr (C::PAIR) mma_commit_pair(&done[s], 3);  // both CTAs' stage s
+          else mma_commit(&done[s]);
         }
         if (!ok) break;
-        mma_commit(&tfull[b]);
+        if constexpr (C::PAIR) mma_commit_pair(&tfull[b], 3);
+        else mma_commit(&tfull[b]);
         if (++b == 2) { b = 0; ph_b ^= 1u; }
       }
       // Every MMA issued has completed before the TMEM is freed (after an error the
       // epilogue may not have waited for the last ones).
-      mma_commit(mma_drained);
+      if constexpr (C::PAIR) mma_commit_pair(mma_drained, 1);
+      else mma_commit(mma_drained);
       mbar_wait_drain(mma_drained, 0);
     }
     __syncwarp();
@@ -414,7 +473,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint32_t g = 0;
     bool ok = true;
     if constexpr (C::QBITS > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(qready, 0));
-    for (int unit = blockIdx.x; ok && unit < args.num_units; unit += gridDim.x) {
+    for (int unit = unit0; ok && unit < args.num_units; unit += ustep) {
       int kb0, kb1;
       split_range(num_k, args.splits, unit % args.splits, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb, ++g) {
@@ -434,8 +493,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         unpack_tile<C::BM, NT, C::ACT_BITS == 8>(smem + C::OFF_WP + s * C::WP_BYTES,
                                                  smem + C::OFF_WU + u * C::WU_BYTES, tid);
         if constexpr (C::ACT_BITS == 4) {
-          unpack_tile<C::BN, NT, false>(smem + C::OFF_XS + s * C::XS_BYTES,
-                                        smem + C::OFF_XU + u * C::XU_BYTES, tid);
+          unpack_tile<C::BNX, NT, false>(smem + C::OFF_XS + s * C::XS_BYTES,
+                                         smem + C::OFF_XU + u * C::XU_BYTES, tid);
         }
         if constexpr (C::QBITS > 0) {
           // chunk i: token row i / 16, channels 8*(i % 16) .. +7 of this K block
@@ -474,7 +533,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ufull[u]);
+        if (lane == 0) {
+          if constexpr (C::PAIR) mbar_arrive_cluster(mapa_shared(&ufull[u], 0));
+          else mbar_arrive(&ufull[u]);
+        }
       }
     }
   } else if (C::epi_index(warp) >= 0) {
@@ -551,11 +613,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // y (or the next linear's codes) is written unless this is the int32 debug view
     const bool has_out = args.has_y != 0;
     float* nxt_s = reinterpret_cast<float*>(smem + C::OFF_TOK + C::OFF_TOK_NEXT);  // EPI
-    for (int unit = blockIdx.x; unit < args.num_units; unit += gridDim.x, ++it) {
+    for (int unit = unit0; unit < args.num_units; unit += ustep, ++it) {
       const int tile = unit / args.splits;
       int n_tile, m_tile;
       decode_tile(args, tile, n_tile, m_tile);
-      const int n_base = n_tile * C::BM + q * 32;
+      const int n_base = n_tile * C::TILE_N + static_cast<int>(rank) * C::BM + q * 32;
       const int n = n_base + lane;
       const int m0 = m_tile * C::BN;
       float* sts = tok_s + (it & 1) * C::BN;
@@ -668,12 +730,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int j = 0; j < 16; ++j) {
           const float v =
               fmaf(sts[j0 + j] * sw, __int2float_rn(static_cast<int>(r[j])), offset(sds[j0 + j]));
-          const float yv = __bfloat162float(__float2bfloat16_rn(v));
-          const __nv_bfloat16 hb = __float2bfloat16_rn(gelu_f32(yv));
+          const uint16_t hbits = gelu_bf16_bits(__bfloat16_as_ushort(__float2bfloat16_rn(v)));
           const int m = m0 + j0 + j;
           if (args.g_h != nullptr && n < args.N && m < args.M)
-            args.g_h[(size_t)m * args.N + n] = __bfloat16_as_ushort(hb);
-          const float xv = __fmul_rn(__bfloat162float(hb), g_ci);
+            args.g_h[(size_t)m * args.N + n] = hbits;
+          const float xv = __fmul_rn(__uint_as_float(static_cast<uint32_t>(hbits) << 16), g_ci);
           const float sn = g_s[j0 + j], rn = g_s[C::BN + j0 + j];
           const uint32_t code = (sn > 0.0f && isfinite(rn))
                                     ? quantize1_recip<C::QMAX_NEXT>(xv, sn, rn)
@@ -707,7 +768,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tc_fence_after();
       if (h >= C::NUM_CHUNKS) {  // no chunk for this warp (token tiles of 16)
         tc_fence_before();
-        if (lane == 0) mbar_arrive(&tempty[b]);
+        if (lane == 0) {
+          if constexpr (C::PAIR) mbar_arrive_cluster(mapa_shared(&tempty[b], 0));
+          else mbar_arrive(&tempty[b]);
+        }
       }
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * C::BN);
@@ -722,7 +786,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (c + 2 >= C::NUM_CHUNKS) {  // last chunk of this warp: hand the accumulator back
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[b]);
+          if (lane == 0) {
+            if constexpr (C::PAIR) mbar_arrive_cluster(mapa_shared(&tempty[b], 0));
+            else mbar_arrive(&tempty[b]);
+          }
         }
         if (m0 + j0 >= args.M) continue;  // whole chunk beyond the last token
         if (!split) {
@@ -763,10 +830,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  // a pair: neither CTA leaves (or frees the TMEM) while the other may still
+  // arrive on its barriers or have the pair MMA read its shared memory
+  if constexpr (C::PAIR) cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (C::PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
@@ -833,11 +904,11 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
   if (C::QBITS > 0)  // bf16 activations, boxes of 64 channels x BN tokens
     ok = ok && single && make_map(&tm_x, single->x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, 64,
                                   C::BN, CU_TENSOR_MAP_SWIZZLE_NONE);
-  else if (C::ACT_BITS == 8)
-    ok = ok && make_map(&tm_x, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, C::BK, C::BN,
+  else if (C::ACT_BITS == 8)  // each CTA of a pair loads half of the token tile
+    ok = ok && make_map(&tm_x, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, C::BK, C::BNX,
                         CU_TENSOR_MAP_SWIZZLE_128B);
   else
-    ok = ok && make_map(&tm_x, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, C::BK / 2, C::BN,
+    ok = ok && make_map(&tm_x, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, C::BK / 2, C::BNX,
                         CU_TENSOR_MAP_SWIZZLE_64B);
   int32_t* acc_out = ex ? ex->acc_out : nullptr;
   if (out == nullptr && acc_out == nullptr) return cudaErrorInvalidValue;
@@ -856,12 +927,12 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
   a.N = N;
   a.K = K;
   a.tiles_m = (M + C::BN - 1) / C::BN;
-  a.tiles_n = (N + C::BM - 1) / C::BM;
+  a.tiles_n = (N + C::TILE_N - 1) / C::TILE_N;
   a.num_tiles = a.tiles_m * a.tiles_n;
   // Keep the smaller operand resident in L2: sweep output channels fastest when
   // the packed weights fit comfortably, so each activation tile streams once.
   a.n_fastest = (static_cast<size_t>(N) * K / 2) <= (48u << 20) ? 1 : 0;
-  a.splits = scratch != nullptr ? gemm_splits(M, N, K) : 1;
+  a.splits = (scratch != nullptr && !C::PAIR) ? gemm_splits(M, N, K) : 1;
   a.num_units = a.num_tiles * a.splits;
   a.partial = scratch ? scratch->partial : nullptr;
   a.counters = scratch ? scratch->counters : nullptr;
@@ -884,14 +955,45 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
   static std::atomic<bool> attr_set[kAttrDevices] = {};  // per template instance and device
   const cudaError_t e = set_smem_once(gemm_kernel<C>, C::SMEM_BYTES, attr_set);
   if (e != cudaSuccess) return e;
+  if constexpr (C::PAIR) {  // clusters of two CTAs, one unit per pair at a time
+    static std::atomic<int> max_pairs[kAttrDevices] = {};  // resident pairs, per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int fit = (dev >= 0 && dev < kAttrDevices) ? max_pairs[dev].load() : 0;
+    if (fit == 0) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(2 * (sm_count() / 2));
+      q.blockDim = dim3(C::THREADS);
+      q.dynamicSmemBytes = C::SMEM_BYTES;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 2;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      q.attrs = at;
+      q.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&fit, gemm_kernel<C>, &q) != cudaSuccess || fit < 1)
+        fit = sm_count() / 2;
+      if (dev >= 0 && dev < kAttrDevices) max_pairs[dev].store(fit);
+    }
+    const int pairs = a.num_units < fit ? a.num_units : fit;
+    return launch_pdl(gemm_kernel<C>, 2 * pairs, C::THREADS, C::SMEM_BYTES, st, 2, tm_w, tm_x,
+                      tm_out, a);
+  }
   const int grid = a.num_units < sm_count() ? a.num_units : sm_count();
-  return launch_pdl(gemm_kernel<C>, grid, C::THREADS, C::SMEM_BYTES, st, tm_w, tm_x, tm_out, a);
+  return launch_pdl(gemm_kernel<C>, grid, C::THREADS, C::SMEM_BYTES, st, 1, tm_w, tm_x, tm_out, a);
 }
 
+// 256-token tiles go to CTA pairs unless K is split (few tokens, few tiles).
 template <int ACT_BITS, int EPI = 0>
 cudaError_t dispatch_bn(const void* qx, const uint8_t* qw, int M, int N, int K,
                         const EpilogueArgs& ep, void* out, const SplitScratch* sc,
                         cudaStream_t st, bool wp, const GemmExtras* ex) {
+  if constexpr (ACT_BITS == 8) {
+    if (bn_for(M) == 256 && (sc == nullptr || gemm_splits(M, N, K) == 1))
+      return run_gemm<Cfg<256, 8, 0, EPI, true>>(qx, qw, M, N, K, ep, out, nullptr, st, wp,
+                                                 nullptr, ex);
+  }
   switch (bn_for(M)) {
     case 16:
       return run_gemm<Cfg<16, ACT_BITS, 0, EPI>>(qx, qw, M, N, K, ep, out, sc, st, wp, nullptr, ex);
@@ -961,6 +1063,26 @@ cudaError_t launch_gemm(const void* qx, int act_bits, const uint8_t* qw, int M, 
   return act_bits == 8
              ? dispatch_bn<8>(qx, qw, M, N, K, ep, y, scratch, st, w_prefetch, extras)
              : dispatch_bn<4>(qx, qw, M, N, K, ep, y, scratch, st, w_prefetch, extras);
+}
+
+// The GELU table, once per device: launched on the caller's stream, and marked
+// built only after a launch outside stream capture has completed (a launch inside a
+// capture becomes part of the graph and rebuilds the table on every replay).
+cudaError_t ensure_gelu_table(cudaStream_t st) {
+  static std::atomic<bool> built[kAttrDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaGetLastError();
+  const bool cached = dev >= 0 && dev < kAttrDevices;
+  if (cached && built[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return cudaGetLastError();
+  constexpr int n = 2 * kGeluTabExps * 128;
+  gelu_table_kernel<<<(n + 127) / 128, 128, 0, st>>>();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || cs != cudaStreamCaptureStatusNone) return e;
+  e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess && cached) built[dev].store(true, std::memory_order_release);
+  return e;
 }
 
 cudaError_t launch_gemm_gelu_quant(const void* qx, const uint8_t* qw, int M, int N, int K,

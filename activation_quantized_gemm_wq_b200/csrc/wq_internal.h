@@ -13,19 +13,24 @@ namespace wq {
 // Launch with programmatic stream serialization: the kernel may start while the
 // previous kernel in the stream is still running, and must call griddep_wait()
 // before it touches anything that kernel (or an earlier one) writes.
+// cluster > 1: clusters of that many CTAs along x (the grid a multiple of it).
 template <class... KArgs, class... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem,
-                       cudaStream_t st, Args... args) {
+                       cudaStream_t st, int cluster, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(block);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(cluster > 1 ? cluster : 1);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cluster > 1 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
@@ -136,6 +141,10 @@ cudaError_t launch_gemm(const void* qx, int act_bits, const uint8_t* qw, int M, 
                         const EpilogueArgs& ep, void* y, const SplitScratch* scratch,
                         cudaStream_t st, bool w_prefetch = false,
                         const GemmExtras* extras = nullptr);
+
+// Builds, once per device, the GELU table launch_gemm_gelu_quant reads; call before
+// anything of that call is launched (it may synchronize the stream once).
+cudaError_t ensure_gelu_table(cudaStream_t st);
 
 // The FFN up-projection whose epilogue quantizes for the down-projection: the
 // same GEMM on int8 codes qx, y as launch_gemm computes it, then h = bf16(GELU(y))

@@ -159,39 +159,10 @@ __device__ __forceinline__ uint32_t mapa_shared(const void* p, uint32_t rank) {
   return r;
 }
 
-// Arrive on an mbarrier of either CTA of the cluster (address from mapa_shared).
+// Arrive on an mbarrier of either CTA of the cluster (address from mapa_shared),
+// with the default (CTA-scope release) semantics.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// mbar_wait for a barrier that threads of the other CTA arrive on (acquire at
-// cluster scope); bounded in the same way.
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
-  const uint32_t a = smem_u32(bar);
-  unsigned long long t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait_cluster(a, parity)) return true;
-    if ((i & 255u) == 0u) {
-      if (error_raised()) return false;
-      if (globaltimer_ns() - t0 > wait_limit_ns()) {
-        raise_error(kErrWaitTimeout);
-        return false;
-      }
-    }
-  }
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // TMEM of a CTA pair: issued by the same warp of both CTAs, with the same holder

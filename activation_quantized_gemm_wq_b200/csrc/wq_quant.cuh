@@ -299,7 +299,7 @@ cudaError_t run_act_quant(const uint16_t* x, int M, int K, const float* cinv,
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int groups = (M + RPC - 1) / RPC;
   const int grid = groups < per_sm * sms ? groups : per_sm * sms;
-  return launch_pdl(act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT, STATIC>, grid, 256, smem, st, x, M, K, cinv, sid,
+  return launch_pdl(act_quant_kernel<ACT_BITS, STORE_BITS, TPR, CPT, STATIC>, grid, 256, smem, st, 1, x, M, K, cinv, sid,
                     alpha, thr, S, step, qx, s_tok, zero, zero_n16);
 }
 
@@ -414,7 +414,7 @@ cudaError_t run_act_quant_rows(const uint16_t* x, int M, int K, const float* cin
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int want = (M + 7) / 8;  // one warp per row
   const int grid = want < per_sm * sms ? want : per_sm * sms;
-  return launch_pdl(act_quant_row_kernel<ACT_BITS, STORE_BITS, STATIC>, grid, 256, 0, st, x, M,
+  return launch_pdl(act_quant_row_kernel<ACT_BITS, STORE_BITS, STATIC>, grid, 256, 0, st, 1, x, M,
                     K, cinv, sid, alpha, thr, S, step, qx, s_tok, zero, zero_n16);
 }
 
@@ -428,18 +428,20 @@ cudaError_t run_act_quant_rows(const uint16_t* x, int M, int K, const float* cin
 // across the CTA (warp shuffles, then one shared-memory atomic max per warp and
 // row), R threads turn them into the rows' scales, and every thread writes the
 // codes of its channels.  One CTA per SM, persistent over rounds.
-constexpr int kRingThreads = 512;
-constexpr int kRingRoundElems = 32768;  // 64 KB of bf16 per round
+constexpr int kRingElemsPerThread = 64;  // of every round
+
 constexpr int kRingSlots = 3;
 #ifndef WQ_RING_MIN_ROWS
 #define WQ_RING_MIN_ROWS 512
 #endif
 constexpr int kRingMinRows = WQ_RING_MIN_ROWS;
 
-template <int C>
+// NT threads per CTA (512: one CTA per SM; 256: two, so that one computes while
+// the other waits at a barrier), C channels per thread.
+template <int C, int NT>
 struct Ring {
-  static constexpr int K = kRingThreads * C;
-  static constexpr int R = kRingRoundElems / K;           // rows per round
+  static constexpr int K = NT * C;
+  static constexpr int R = kRingElemsPerThread / C;       // rows per round
   static constexpr int ROUND_BYTES = R * K * 2;
   static constexpr int OFF_AMAX = kRingSlots * ROUND_BYTES;  // uint32 [2][R]
   static constexpr int OFF_SCALE = OFF_AMAX + 2 * R * 4;    // float [R] s, then [R] 1/s
@@ -499,43 +501,98 @@ __device__ __forceinline__ float warp_max_multi(float (&v)[R], int lane) {
 template <int R>
 constexpr int log2_of() { return R <= 1 ? 0 : 1 + log2_of<R / 2>(); }
 
-template <int ACT_BITS, int STORE_BITS, int C, bool STATIC>
-__global__ void __launch_bounds__(kRingThreads, 1) act_quant_ring_kernel(
+// Codes of one group of GW = 4 or 8 values (x' as GW/2 pairs), scale s > 0 with
+// r = 1/s finite, as bytes (GW/4 words): the general path, one value at a time
+// (float clamp, exact quotient at near ties).  Kept out of line: the packed path
+// below serves almost every group.
+template <int QMAX, int GW>
+__device__ __noinline__ uint2 codes_general(float4 a, float4 b, float s, float r) {
+  const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t c[8];
+  quantize_recip_n<QMAX, GW>(v, s, r, c);
+  return make_uint2(pack_low_bytes(c[0], c[1], c[2], c[3]),
+                    GW == 8 ? pack_low_bytes(c[4], c[5], c[6], c[7]) : 0u);
+}
+
+// The same codes two values at a time: t = x' * r, u = t + 1.5*2^23 (u's low 16 bits
+// are rint(t) as a two's-complement int16 while |t| < 2^15), clamped as 16-bit
+// pairs.  `narrow` says |t| < 2^15 holds for the row (its maximum |x'| <= 16384 s).
+// Falls back to codes_general when a value lies near a half-integer or the row is
+// not narrow; the result equals quantize<QMAX>(v, s) for every value.
+template <int QMAX, int GW>
+__device__ __forceinline__ uint2 codes_packed(const float2 (&v)[GW / 2], float s, float r,
+                                              bool narrow) {
+  const float2 r2 = make_float2(r, r);
+  const float2 m2 = make_float2(kRoundMagic, kRoundMagic);
+  const float2 nm2 = make_float2(-kRoundMagic, -kRoundMagic);
+  const float2 neg1 = make_float2(-1.0f, -1.0f);
+  bool near_tie = false;
+  uint32_t h[GW / 2];
+#pragma unroll
+  for (int p = 0; p < GW / 2; ++p) {
+    const float2 t = __fmul2_rn(v[p], r2);
+    const float2 u = __fadd2_rn(t, m2);
+    const float2 d = __ffma2_rn(__fadd2_rn(u, nm2), neg1, t);  // t - rint(t), exact
+    near_tie = near_tie || fabsf(d.x) >= 0.5f - 0x1p-12f || fabsf(d.y) >= 0.5f - 0x1p-12f;
+    h[p] = __byte_perm(__float_as_uint(u.x), __float_as_uint(u.y), 0x5410);
+  }
+  if (near_tie || !narrow) {
+    const float4 a = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
+    const float4 b = GW == 8 ? make_float4(v[GW / 2 - 2].x, v[GW / 2 - 2].y, v[GW / 2 - 1].x,
+                                           v[GW / 2 - 1].y)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    return codes_general<QMAX, GW>(a, b, s, r);
+  }
+  constexpr uint32_t lo = static_cast<uint32_t>(static_cast<uint16_t>(-QMAX)) * 0x00010001u;
+  constexpr uint32_t hi = static_cast<uint32_t>(QMAX) * 0x00010001u;
+#pragma unroll
+  for (int p = 0; p < GW / 2; ++p) h[p] = __vmins2(__vmaxs2(h[p], lo), hi);
+  return make_uint2(__byte_perm(h[0], h[1], 0x6420),
+                    GW == 8 ? __byte_perm(h[GW / 2 - 2], h[GW / 2 - 1], 0x6420) : 0u);
+}
+
+template <int ACT_BITS, int STORE_BITS, int C, int NT, bool STATIC>
+__global__ void __launch_bounds__(NT, 512 / NT) act_quant_ring_kernel(
     const uint16_t* __restrict__ x, int M, const float* __restrict__ cinv,
     const uint8_t* __restrict__ stream_id, const float* __restrict__ alpha,
     const float* __restrict__ thr, int S, int step, void* __restrict__ qx,
     float* __restrict__ s_tok, uint4* __restrict__ zero, size_t zero_n16) {
-  using G = Ring<C>;
+  using G = Ring<C, NT>;
   constexpr int K = G::K, R = G::R;
   constexpr int QMAX = ACT_BITS == 8 ? 127 : 7;
-  constexpr int CH = C / 4;  // groups of 4 channels a thread owns (8 bytes of bf16 each)
+  // thread t owns channel groups g = t + NT * j of GW channels each
+  constexpr int GW = C % 8 == 0 ? 8 : 4;
+  constexpr int NG = C / GW;
+  constexpr int P = C / 2;  // value pairs per row and thread
   extern __shared__ __align__(128) uint8_t ring_smem[];
   uint32_t* amax_s = reinterpret_cast<uint32_t*>(ring_smem + G::OFF_AMAX);
   float* scale_s = reinterpret_cast<float*>(ring_smem + G::OFF_SCALE);
   uint64_t* full = reinterpret_cast<uint64_t*>(ring_smem + G::OFF_BAR);
   const int t = threadIdx.x;
-  const int warp = t >> 5, lane = t & 31;
+  const int lane = t & 31;
 
   if (t == 0) {
     for (int i = 0; i < kRingSlots; ++i) mbar_init(&full[i], 1);
     fence_mbar_init();
   }
   if (t < 2 * R) amax_s[t] = 0u;
-  // thread t owns channel groups g = t + 512 * j (channels 4g .. 4g + 3)
-  float ci[C];
+  float2 ci[P];
 #pragma unroll
-  for (int j = 0; j < CH; ++j) {
-    const int k0 = 4 * (t + kRingThreads * j);
-    const float4 a = cinv ? __ldg(reinterpret_cast<const float4*>(cinv + k0))
-                          : make_float4(1.f, 1.f, 1.f, 1.f);
-    ci[4 * j] = a.x; ci[4 * j + 1] = a.y; ci[4 * j + 2] = a.z; ci[4 * j + 3] = a.w;
+  for (int j = 0; j < NG; ++j) {
+#pragma unroll
+    for (int q4 = 0; q4 < GW / 4; ++q4) {
+      const int k0 = GW * (t + NT * j) + 4 * q4;
+      const float4 a = cinv ? __ldg(reinterpret_cast<const float4*>(cinv + k0))
+                            : make_float4(1.f, 1.f, 1.f, 1.f);
+      ci[j * (GW / 2) + 2 * q4] = make_float2(a.x, a.y);
+      ci[j * (GW / 2) + 2 * q4 + 1] = make_float2(a.z, a.w);
+    }
   }
   __syncthreads();
   // x, the ids and the split-K scratch may belong to the previous kernel
   griddep_wait();
   griddep_launch_dependents();
-  for (size_t i = (size_t)blockIdx.x * kRingThreads + t; i < zero_n16;
-       i += (size_t)gridDim.x * kRingThreads)
+  for (size_t i = (size_t)blockIdx.x * NT + t; i < zero_n16; i += (size_t)gridDim.x * NT)
     zero[i] = make_uint4(0u, 0u, 0u, 0u);
 
   const int rounds = (M + R - 1) / R;
@@ -560,28 +617,39 @@ __global__ void __launch_bounds__(kRingThreads, 1) act_quant_ring_kernel(
     const int rows = min(R, M - row0);
     const bool landed = mbar_wait(&full[slot], (local / kRingSlots) & 1u);
     // x' of this thread's channels of every row of the round, and the row maxima
-    float xv[R][C];
+    float2 xv[R][P];
     float pmax[R];  // this thread's maximum of |x'| per row
     const uint8_t* base = ring_smem + slot * G::ROUND_BYTES;
 #pragma unroll
     for (int i = 0; i < R; ++i) {
       float amax = 0.0f;
 #pragma unroll
-      for (int j = 0; j < CH; ++j) {
-        const uint2 w = (landed && i < rows)
-                            ? *reinterpret_cast<const uint2*>(base + (size_t)i * K * 2 +
-                                                               8 * (t + kRingThreads * j))
-                            : make_uint2(0u, 0u);
-        const float f[4] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y)};
+      for (int j = 0; j < NG; ++j) {
+        uint32_t w[GW / 2];
+        const uint8_t* src = base + (size_t)i * K * 2 + 2 * GW * (t + NT * j);
+        if (landed && i < rows) {
+          if constexpr (GW == 8) {
+            const uint4 q4 = *reinterpret_cast<const uint4*>(src);
+            w[0] = q4.x; w[1] = q4.y; w[2 % (GW / 2)] = q4.z; w[3 % (GW / 2)] = q4.w;
+          } else {
+            const uint2 q2 = *reinterpret_cast<const uint2*>(src);
+            w[0] = q2.x; w[1] = q2.y;
+          }
+        } else {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          xv[i][4 * j + e] = __fmul_rn(f[e], ci[4 * j + e]);
-          amax = fmaxf(amax, fabsf(xv[i][4 * j + e]));
+          for (int e = 0; e < GW / 2; ++e) w[e] = 0u;
+        }
+#pragma unroll
+        for (int e = 0; e < GW / 2; ++e) {
+          const float2 f = make_float2(bf16lo(w[e]), bf16hi(w[e]));
+          const float2 v = __fmul2_rn(f, ci[j * (GW / 2) + e]);
+          xv[i][j * (GW / 2) + e] = v;
+          amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
         }
       }
       pmax[i] = amax;
     }
-    if constexpr (!STATIC) {
+    {
       // row (lane >> SH) of the round, reduced over the warp, then over the warps
       // (non-negative floats order as their bit patterns)
       constexpr int SH = 5 - log2_of<R>();
@@ -598,6 +666,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) act_quant_ring_kernel(
     }
     if (t < rows) {
       const int row = row0 + t;
+      const float amax = __uint_as_float(amax_s[(local & 1) * R + t]);
       float sc = 0.0f;
       const int sid = stream_id[row];
       if (sid < S) {
@@ -606,43 +675,66 @@ __global__ void __launch_bounds__(kRingThreads, 1) act_quant_ring_kernel(
           const float g = __ldg(alpha + step * S + sid);
           clip = g > 0.0f ? __fdiv_rn(__ldg(thr + step), g) : 0.0f;
         } else {
-          clip = __fmul_rn(__ldg(alpha + step * S + sid),
-                           __uint_as_float(amax_s[(local & 1) * R + t]));
+          clip = __fmul_rn(__ldg(alpha + step * S + sid), amax);
         }
         sc = __fdiv_rn(clip, static_cast<float>(QMAX));
       } else {
         raise_error(kErrBadStreamId);
       }
       s_tok[row] = sc;
+      const float rc = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+      // negative reciprocal: this row takes the general path (a zero or tiny scale)
+      const bool fast = sc > 0.0f && isfinite(rc);
       scale_s[t] = sc;
-      scale_s[R + t] = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+      scale_s[R + t] = fast ? (amax <= 16384.0f * sc ? rc : -rc) : 0.0f;
     }
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < R; ++i) {
       if (i >= rows) break;
-      const float sc = scale_s[i], rc = scale_s[R + i];
-      const bool fast = sc > 0.0f && isfinite(rc);
+      const float sc = scale_s[i], rs = scale_s[R + i];
+      const float rc = fabsf(rs);
+      const bool fast = rs != 0.0f;
+      const bool narrow = rs > 0.0f;
       const size_t row = static_cast<size_t>(row0 + i);
 #pragma unroll
-      for (int j = 0; j < CH; ++j) {
-        uint32_t cq[4];
+      for (int j = 0; j < NG; ++j) {
+        uint2 cw;
         if (fast) {
-          quantize_recip_n<QMAX, 4>(&xv[i][4 * j], sc, rc, cq);
-        } else {
+          float2 vv[GW / 2];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            cq[e] = static_cast<uint32_t>(quantize<QMAX>(xv[i][4 * j + e], sc));
-        }
-        const int g = t + kRingThreads * j;  // channel group: channels 4g .. 4g + 3
-        if constexpr (STORE_BITS == 8) {
-          reinterpret_cast<uint32_t*>(static_cast<int8_t*>(qx) + row * K)[g] =
-              pack_low_bytes(cq[0], cq[1], cq[2], cq[3]);
+          for (int e = 0; e < GW / 2; ++e) vv[e] = xv[i][j * (GW / 2) + e];
+          cw = codes_packed<QMAX, GW>(vv, sc, rc, narrow);
         } else {
-          const uint32_t b = pack_low_bytes(cq[0], cq[1], cq[2], cq[3]) & 0x0F0F0F0Fu;
-          const uint32_t n = b | (b >> 4);  // bytes 0 and 2: (c0 | c1 << 4), (c2 | c3 << 4)
-          reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(qx) + row * (K / 2))[g] =
-              static_cast<uint16_t>(__byte_perm(n, 0u, 0x0020) & 0xFFFFu);
+          uint32_t cq[GW];
+#pragma unroll
+          for (int e = 0; e < GW / 2; ++e) {
+            cq[2 * e] = static_cast<uint32_t>(quantize<QMAX>(xv[i][j * (GW / 2) + e].x, sc));
+            cq[2 * e + 1] = static_cast<uint32_t>(quantize<QMAX>(xv[i][j * (GW / 2) + e].y, sc));
+          }
+          cw = make_uint2(pack_low_bytes(cq[0], cq[1], cq[2], cq[3]),
+                          GW == 8 ? pack_low_bytes(cq[4 % GW], cq[5 % GW], cq[6 % GW], cq[7 % GW])
+                                  : 0u);
+        }
+        const int g = t + NT * j;  // channel group: channels GW*g .. GW*g + GW-1
+        if constexpr (STORE_BITS == 8) {
+          if constexpr (GW == 8)
+            reinterpret_cast<uint2*>(static_cast<int8_t*>(qx) + row * K)[g] = cw;
+          else
+            reinterpret_cast<uint32_t*>(static_cast<int8_t*>(qx) + row * K)[g] = cw.x;
+        } else {
+          // nibbles: bytes 0 and 2 of n hold (c0 | c1 << 4) and (c2 | c3 << 4)
+          uint32_t n0 = cw.x & 0x0F0F0F0Fu;
+          n0 |= n0 >> 4;
+          if constexpr (GW == 8) {
+            uint32_t n1 = cw.y & 0x0F0F0F0Fu;
+            n1 |= n1 >> 4;
+            reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(qx) + row * (K / 2))[g] =
+                __byte_perm(n0, n1, 0x6420);
+          } else {
+            reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(qx) + row * (K / 2))[g] =
+                static_cast<uint16_t>(__byte_perm(n0, 0u, 0x0020) & 0xFFFFu);
+          }
         }
       }
     }
@@ -656,23 +748,23 @@ __global__ void __launch_bounds__(kRingThreads, 1) act_quant_ring_kernel(
   }
 }
 
-template <int ACT_BITS, int STORE_BITS, int C, bool STATIC>
+template <int ACT_BITS, int STORE_BITS, int C, int NT, bool STATIC>
 cudaError_t run_act_quant_ring(const uint16_t* x, int M, const float* cinv, const uint8_t* sid,
                                const float* alpha, const float* thr, int S, int step, void* qx,
                                float* s_tok, uint4* zero, size_t zero_n16, cudaStream_t st) {
-  using G = Ring<C>;
+  using G = Ring<C, NT>;
   static std::atomic<bool> attr_set[kAttrDevices] = {};  // per template instance and device
-  const cudaError_t ea =
-      set_smem_once(act_quant_ring_kernel<ACT_BITS, STORE_BITS, C, STATIC>, G::SMEM, attr_set);
+  const cudaError_t ea = set_smem_once(act_quant_ring_kernel<ACT_BITS, STORE_BITS, C, NT, STATIC>,
+                                       G::SMEM, attr_set);
   if (ea != cudaSuccess) return ea;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int rounds = (M + G::R - 1) / G::R;
-  const int grid = rounds < sms ? rounds : sms;
-  return launch_pdl(act_quant_ring_kernel<ACT_BITS, STORE_BITS, C, STATIC>, grid, kRingThreads,
-                    G::SMEM, st, x, M, cinv, sid, alpha, thr, S, step, qx, s_tok, zero,
-                    zero_n16);
+  const int slots = sms * (512 / NT);  // resident CTAs
+  const int grid = rounds < slots ? rounds : slots;
+  return launch_pdl(act_quant_ring_kernel<ACT_BITS, STORE_BITS, C, NT, STATIC>, grid, NT, G::SMEM,
+                    st, 1, x, M, cinv, sid, alpha, thr, S, step, qx, s_tok, zero, zero_n16);
 }
 
 template <int ACT_BITS, int STORE_BITS, bool STATIC>
@@ -680,16 +772,14 @@ cudaError_t dispatch_act_quant(const uint16_t* x, int M, int K, const float* cin
                                const uint8_t* sid, const float* alpha, const float* thr, int S,
                                int step, void* qx, float* s_tok, uint4* zero, size_t zero_n16,
                                cudaStream_t st) {
-#define WQ_RING(C_)                                                                         \
-  return run_act_quant_ring<ACT_BITS, STORE_BITS, C_, STATIC>(x, M, cinv, sid, alpha, thr, S, \
-                                                              step, qx, s_tok, zero, zero_n16, st)
-  // Many rows: rows staged in shared memory, channels owned by threads.
-  if (M >= kRingMinRows) {
-    if (K == 2048) WQ_RING(4);
-    if (K == 4096) WQ_RING(8);
-    if (K == 8192) WQ_RING(16);
-    if (K == 16384) WQ_RING(32);
-  }
+#define WQ_RING(C_, NT_)                                                                      \
+  return run_act_quant_ring<ACT_BITS, STORE_BITS, C_, NT_, STATIC>(x, M, cinv, sid, alpha, thr, \
+                                                                   S, step, qx, s_tok, zero,    \
+                                                                   zero_n16, st)
+  // Many rows of K = 4096: rows staged in shared memory, channels owned by threads,
+  // two CTAs of 256 threads per SM (measured 16 % faster than one warp per row at
+  // M = 8512; at K = 2048, 8192 and 16384 the kernels below were as fast or faster).
+  if (M >= kRingMinRows && K == 4096) WQ_RING(16, 256);
 #undef WQ_RING
   // Many rows of moderate length: independent warps, one per row (measured faster
   // for M = 4288 and 8512 at K = 2048 and 4096).  Few rows, or long rows, keep a

@@ -71,6 +71,9 @@ def parse():
     p.add_argument("--sweep", action="store_true",
                    help="per-shape table over every configured workload (not the JSON line)")
     p.add_argument("--sweep-filter", default="", help="only sweep entries whose label has this")
+    p.add_argument("--ffn", action="store_true",
+                   help="each block's FFN pair with GELU fused into the quantization for the "
+                        "down-projection, against the unfused pair (JSON lines)")
     p.add_argument("--sequence", action="store_true",
                    help="whole denoising sequences (every step of a block's four linears in "
                         "one CUDA graph), one JSON line per workload (not the bench line)")
@@ -955,6 +958,62 @@ def sweep(args):
               f"{r['bound']} | {r['gemm_frac']} | {r['linear_frac']} | {r['bf16_us']} |")
 
 
+def ffn(args):
+    """The FFN pair of each block (up-projection, GELU, down-projection), W4A8, full
+    token batch: the up-projection quantizing for the down-projection in its epilogue
+    (wq_linear_gelu_quant, then wq_gemm_w4ax on its codes), against the same steps
+    unfused: wq_linear_w4a8 for the up-projection, GELU on its bf16 output as a
+    separate kernel (torch's exact-erf GELU, a library kernel standing in for any
+    elementwise pass), then the static-clipping linear reading the GELU output.  One
+    CUDA graph per variant over two activation sets; mean of 20 replays."""
+    import torch
+
+    import activation_quantized_gemm_wq_b200 as wq
+
+    def dev(a):
+        a = np.ascontiguousarray(a)
+        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
+
+    bf16_burst, _, hbm, src = peaks()
+    p_int8 = bf16_burst * INT8_PER_BF16 * 1e12
+    for wl in (S.BLOCK2048_A8, S.BLOCK4096_A8):
+        up, down = [Layer(wl, i, 2, wq, torch, dev) for i in (2, 3)]
+        M, Kh = wl.M, up.N
+        T = up.T
+        codes = torch.empty((M, Kh), dtype=torch.int8, device="cuda")
+        s_next = torch.empty(M, dtype=torch.float32, device="cuda")
+        thr = torch.full((T,), 0.5, dtype=torch.float32, device="cuda")
+        gain = down.alpha  # stream gains around 1 (values matter only for parity)
+        ws_static = wq.alloc_workspace(M, Kh, down.N, 8)
+        h = torch.empty((M, Kh), dtype=torch.bfloat16, device="cuda")
+
+        def fused(r):
+            wq.wq_linear_gelu_quant(up.x[r], up.cinv, up.sid, up.alpha, up.beta, 0, 8, up.qw,
+                                    up.s_w, up.bias, down.cinv, thr, gain, 8, codes, s_next, None,
+                                    up.ws)
+            wq.wq_gemm_w4ax(codes, s_next, 8, Kh, down.sid, down.beta, down.S, down.T, 0, down.qw,
+                            down.s_w, down.bias, down.y)
+
+        def unfused(r):
+            wq.wq_linear_w4a8(up.x[r], up.cinv, up.sid, up.alpha, up.beta, 0, up.qw, up.s_w,
+                              up.bias, up.y, up.ws)
+            torch.ops.aten.gelu.out(up.y, approximate="none", out=h)
+            wq.wq_linear_w4ax_static(h, down.cinv, down.sid, thr, gain, down.beta, 0, 8,
+                                     down.qw, down.s_w, down.bias, down.y, ws_static)
+
+        ops = up.ops() + down.ops()
+        for name, fn in (("gelu_quant_fused", fused), ("two_linears_unfused", unfused)):
+            ms = _graph_ms(torch, [lambda r=r: fn(r % 2) for r in range(4)], replays=20)
+            print(json.dumps({"ffn": wl.name, "variant": name, "M": M,
+                              "shapes": f"{up.K}->{up.N}->{down.N}", "ms_per_ffn": round(ms, 4),
+                              "tops": round(ops / (ms * 1e-3) / 1e12, 1),
+                              "frac_of_int8_roof": round(ops / p_int8 / (ms * 1e-3), 3),
+                              "peak_source": src}), flush=True)
+        assert wq.wq_device_status() == ("WQ_OK", 0)
+        del up, down, codes, ws_static, h
+        torch.cuda.empty_cache()
+
+
 def sequence(args):
     """A block's whole denoising sequence (T steps x its four fused linears, every step
     with its own activations and table row) captured once in a CUDA graph; the quantizer
@@ -1021,6 +1080,9 @@ def main():
         return
     if args.sequence:
         sequence(args)
+        return
+    if args.ffn:
+        ffn(args)
         return
     if args.workload is None:
         args.workload = DEFAULT_WORKLOAD

@@ -229,7 +229,12 @@ wq_status wq_debug_linear_s32(const wq_bf16* x, int M, int K, int N, const float
  * operands for both widths; the int32 sums are the same).
  *   cinv_next [N] fp32 or NULL (= 1); thr_next [T]; gain_next [T][S];
  *   s_next [M] fp32 out; h [M][N] bf16 out or NULL (a debug copy; not needed).
- * Workspace and other arguments as wq_linear_w4a8. */
+ * Workspace and other arguments as wq_linear_w4a8.
+ * The first call on a device also builds a 7 KB table of bf16(GELU(y)) for the
+ * bf16 values 2^-10 <= |y| < 16 (one small kernel on `stream`, then a wait for
+ * it); make that first call outside stream capture.  (Inside a capture the table
+ * kernel is captured too and reruns with every replay, which is correct but
+ * slower.) */
 wq_status wq_linear_gelu_quant(const wq_bf16* x, int M, int K, int N, const float* cinv,
                                const uint8_t* stream_id, const float* alpha, const float* beta,
                                int S, int T, int step, int act_bits, const uint8_t* qw,

@@ -50,12 +50,12 @@ def test_channel_scale_and_pack_bit_exact(oracle, wl, layer):
 
 # ------------------------------------------------------------------ activation codes
 
-# M >= 512 with K in {2048, 4096, 8192, 16384} takes the staged-rows kernel (the last
-# round of rows ragged here), other M >= 1024 with K <= 4096 the one-warp-per-row
-# kernel, the rest the CTA-per-rows one
+# M >= 512 with K = 4096 takes the staged-rows kernel (the last round of rows ragged
+# here), other M >= 1024 with K <= 4096 the one-warp-per-row kernel, the rest the
+# CTA-per-rows one
 AQ_SHAPES = [(64, 256), (37, 384), (300, 2048), (16, 8192), (9, 16384), (3, 32768), (1, 128),
              (1100, 256), (1030, 4096), (2048, 2048), (1050, 8192), (1025, 32768),
-             (513, 2048), (777, 16384), (600, 8192), (1111, 1024)]
+             (513, 4096), (777, 16384), (600, 8192), (1111, 1024), (1031, 2048)]
 
 
 @pytest.mark.parametrize("bits", [8, 4])
