@@ -57,14 +57,18 @@ __global__ void gelu_table_kernel() {
   g_gelu_tab[i] = __bfloat16_as_ushort(__float2bfloat16_rn(gelu_f32(y)));
 }
 
-// h = bf16(GELU(y)) for a bf16 y, by table where it covers y.
-__device__ __forceinline__ uint16_t gelu_bf16_bits(uint16_t ybits) {
+// Index of bf16 pattern y in the GELU table, or -1 outside it.
+__device__ __forceinline__ int gelu_tab_index(uint32_t ybits) {
   const uint32_t e = (ybits >> 7) & 0xFFu;
-  if (e - kGeluTabExp0 < static_cast<uint32_t>(kGeluTabExps))
-    return __ldg(&g_gelu_tab[(ybits >> 15) * (kGeluTabExps * 128) + (e - kGeluTabExp0) * 128 +
-                             (ybits & 0x7Fu)]);
-  return __bfloat16_as_ushort(
-      __float2bfloat16_rn(gelu_f32(__uint_as_float(static_cast<uint32_t>(ybits) << 16))));
+  return e - kGeluTabExp0 < static_cast<uint32_t>(kGeluTabExps)
+             ? static_cast<int>((ybits >> 15) * (kGeluTabExps * 128) + (e - kGeluTabExp0) * 128 +
+                                (ybits & 0x7Fu))
+             : -1;
+}
+
+// h = bf16(GELU(y)) evaluated (the values the table does not cover).
+__device__ __noinline__ uint32_t gelu_bf16_eval(uint32_t ybits) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(gelu_f32(__uint_as_float(ybits << 16))));
 }
 
 struct TileArgs {
@@ -180,9 +184,11 @@ struct Cfg {
   static constexpr int EPI_BUF_BYTES = EPI_CHUNK * 32 * EPI_ELEM;
   // staged s_tok and stream ids, x2; then (QBITS) each token's scale and its
   // reciprocal; then (EPI) the next linear's token scales and reciprocals, x2
-  static constexpr int TOK_BYTES =
-      2 * BN * 4 + 2 * BN + (QBITS ? 2 * BN * 4 : 0) + (EPI ? 2 * 2 * BN * 4 : 0);
+  static constexpr int GELU_TAB_BYTES = 2 * 14 * 128 * 2;  // EPI: the GELU table, copied here
+  static constexpr int TOK_BYTES = 2 * BN * 4 + 2 * BN + (QBITS ? 2 * BN * 4 : 0) +
+                                   (EPI ? 2 * 2 * BN * 4 + GELU_TAB_BYTES : 0);
   static constexpr int OFF_TOK_NEXT = 2 * BN * 4 + 2 * BN + (QBITS ? 2 * BN * 4 : 0);
+  static constexpr int OFF_GELU_TAB = OFF_TOK_NEXT + 2 * 2 * BN * 4;  // EPI
   static constexpr int SMEM_LIMIT = 232448;  // 227 KB opt-in per CTA
   static constexpr int RESERVED = 1024 /*alignment slack*/ + 512 /*barriers*/;
   static constexpr int FIXED = RESERVED + NU * (WU_BYTES + XU_BYTES) + TOK_BYTES;
@@ -609,6 +615,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // every row's scale staged (after a timeout the waits below give up too)
       __all_sync(0xFFFFFFFFu, mbar_wait(qready, 0));
     }
+    if constexpr (C::EPI > 0) {  // the GELU table into shared memory (read only below)
+      uint32_t* tab_s = reinterpret_cast<uint32_t*>(smem + C::OFF_TOK + C::OFF_GELU_TAB);
+      const uint32_t* tab_g = reinterpret_cast<const uint32_t*>(g_gelu_tab);
+      for (int i = et; i < C::GELU_TAB_BYTES / 4; i += C::EPI_THREADS) tab_s[i] = tab_g[i];
+    }
     const bool split = args.splits > 1;
     // y (or the next linear's codes) is written unless this is the int32 debug view
     const bool has_out = args.has_y != 0;
@@ -724,23 +735,59 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // EPI > 0: y as above, then h = bf16(GELU(y)) and the next linear's code of
       // h * cinv_next[n] with its static scale, staged as int8 [16 tokens][32
       // channels] and written with a TMA store; h itself only to the debug buffer.
+      // The 16 elements go through each step together (independent chains, no
+      // branch inside a step), so their latencies overlap; the rare cases (a value
+      // outside the GELU table, a code near a half-integer, a zero or tiny scale)
+      // take a second pass.
       auto emit_codes = [&](const uint32_t (&r)[16], int j0) {
         uint8_t* sb = stage_buf();
+        const uint16_t* tab = reinterpret_cast<const uint16_t*>(smem + C::OFF_TOK + C::OFF_GELU_TAB);
+        uint32_t hb[16];
+        bool rare = false;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const float v =
               fmaf(sts[j0 + j] * sw, __int2float_rn(static_cast<int>(r[j])), offset(sds[j0 + j]));
-          const uint16_t hbits = gelu_bf16_bits(__bfloat16_as_ushort(__float2bfloat16_rn(v)));
-          const int m = m0 + j0 + j;
-          if (args.g_h != nullptr && n < args.N && m < args.M)
-            args.g_h[(size_t)m * args.N + n] = hbits;
-          const float xv = __fmul_rn(__uint_as_float(static_cast<uint32_t>(hbits) << 16), g_ci);
-          const float sn = g_s[j0 + j], rn = g_s[C::BN + j0 + j];
-          const uint32_t code = (sn > 0.0f && isfinite(rn))
-                                    ? quantize1_recip<C::QMAX_NEXT>(xv, sn, rn)
-                                    : static_cast<uint32_t>(quantize<C::QMAX_NEXT>(xv, sn));
-          sb[j * 32 + lane] = static_cast<uint8_t>(code);
+          const uint32_t yb = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+          const int ti = gelu_tab_index(yb);
+          hb[j] = ti >= 0 ? tab[ti] : (yb | 0x80000000u);  // high bit: evaluate below
+          rare = rare || ti < 0;
         }
+        if (rare) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (hb[j] & 0x80000000u) hb[j] = gelu_bf16_eval(hb[j] & 0xFFFFu);
+        }
+        if (args.g_h != nullptr && n < args.N) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (m0 + j0 + j < args.M) args.g_h[(size_t)(m0 + j0 + j) * args.N + n] = hb[j];
+        }
+        constexpr float kq = static_cast<float>(C::QMAX_NEXT);
+        uint32_t code[16];
+        bool slow = false;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float xv = __fmul_rn(__uint_as_float(hb[j] << 16), g_ci);
+          const float sn = g_s[j0 + j], rn = g_s[C::BN + j0 + j];
+          const float t = __fmul_rn(xv, rn);
+          const float u = __fadd_rn(t, kRoundMagic);
+          const float d = __fsub_rn(t, __fsub_rn(u, kRoundMagic));
+          slow = slow || fabsf(d) >= 0.5f - 0x1p-12f || !(sn > 0.0f) || !isfinite(rn);
+          code[j] = __float_as_uint(fminf(fmaxf(u, kRoundMagic - kq), kRoundMagic + kq));
+        }
+        if (slow) {  // exact codes for every element of the chunk (as quantize1_recip)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float xv = __fmul_rn(__uint_as_float(hb[j] << 16), g_ci);
+            const float sn = g_s[j0 + j], rn = g_s[C::BN + j0 + j];
+            code[j] = (sn > 0.0f && isfinite(rn))
+                          ? quantize1_recip<C::QMAX_NEXT>(xv, sn, rn)
+                          : static_cast<uint32_t>(quantize<C::QMAX_NEXT>(xv, sn));
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) sb[j * 32 + lane] = static_cast<uint8_t>(code[j]);
         store_buf(sb, j0);
       };
 
