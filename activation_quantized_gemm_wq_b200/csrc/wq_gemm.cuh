@@ -40,9 +40,10 @@ namespace wq {
 // bf16(GELU(y)) for every bf16 y with 2^-10 <= |y| < 16 (exponent field 117..130),
 // indexed [sign][exponent - 117][mantissa]: the GELU-and-quantize epilogue looks
 // values up here instead of evaluating erfcf for each element.  Built on the GPU
-// with the same fp32 arithmetic the epilogue uses for the values outside that range
-// (gelu_table_kernel), so a lookup returns exactly what the evaluation would.
-constexpr int kGeluTabExp0 = 117, kGeluTabExps = 14;
+// with the fp32 arithmetic the epilogue evaluates where neither the table nor a
+// closed form applies (gelu_table_kernel), so a lookup returns exactly what the
+// evaluation would; below and above the table h has closed forms (emit_codes).
+constexpr int kGeluTabExp0 = 117, kGeluTabExps = 14, kGeluTabEnd = kGeluTabExp0 + kGeluTabExps;
 __device__ uint16_t g_gelu_tab[2 * kGeluTabExps * 128];
 
 namespace {
@@ -57,18 +58,23 @@ __global__ void gelu_table_kernel() {
   g_gelu_tab[i] = __bfloat16_as_ushort(__float2bfloat16_rn(gelu_f32(y)));
 }
 
-// Index of bf16 pattern y in the GELU table, or -1 outside it.
-__device__ __forceinline__ int gelu_tab_index(uint32_t ybits) {
-  const uint32_t e = (ybits >> 7) & 0xFFu;
-  return e - kGeluTabExp0 < static_cast<uint32_t>(kGeluTabExps)
-             ? static_cast<int>((ybits >> 15) * (kGeluTabExps * 128) + (e - kGeluTabExp0) * 128 +
-                                (ybits & 0x7Fu))
-             : -1;
-}
-
 // h = bf16(GELU(y)) evaluated (the values the table does not cover).
 __device__ __noinline__ uint32_t gelu_bf16_eval(uint32_t ybits) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(gelu_f32(__uint_as_float(ybits << 16))));
+}
+
+// The next linear's code of xv with scale sn, exactly (as the quantizer takes it):
+// from the reciprocal rn where that is a finite positive scale's, else from the
+// quotient.  Out of line: only elements near a half-integer, or with a bad
+// scale, come here.
+template <int QMAX>
+__device__ __noinline__ uint32_t code_exact_next(float xv, float sn, float rn) {
+  return (sn > 0.0f && isfinite(rn)) ? quantize1_recip<QMAX>(xv, sn, rn)
+                                     : static_cast<uint32_t>(quantize<QMAX>(xv, sn));
+}
+
+__device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 v) {
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
 
 struct TileArgs {
@@ -655,7 +661,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
               sn = __fdiv_rn(clip, static_cast<float>(C::QMAX_NEXT));
             }
             g_s[i] = sn;
-            g_s[C::BN + i] = sn > 0.0f ? __frcp_rn(sn) : 0.0f;
+            const float rn = sn > 0.0f ? __frcp_rn(sn) : 0.0f;
+            g_s[C::BN + i] = sn > 0.0f && isfinite(rn) ? rn : __int_as_float(0x7FC00000);
             if (n_tile == 0 && unit % args.splits == 0 && m < args.M) args.g_s[m] = sn;
           }
         }
@@ -735,25 +742,67 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // EPI > 0: y as above, then h = bf16(GELU(y)) and the next linear's code of
       // h * cinv_next[n] with its static scale, staged as int8 [16 tokens][32
       // channels] and written with a TMA store; h itself only to the debug buffer.
-      // The 16 elements go through each step together (independent chains, no
-      // branch inside a step), so their latencies overlap; the rare cases (a value
-      // outside the GELU table, a code near a half-integer, a zero or tiny scale)
-      // take a second pass.
+      // The 16 elements go through each step together, two at a time in packed
+      // fp32x2 arithmetic (the same IEEE roundings per element) and without a
+      // branch inside a step; the rare cases (a value outside the GELU table, a code
+      // near a half-integer, a zero, tiny or infinite scale, whose reciprocal is
+      // staged as NaN) take a second pass that calls out of line.
       auto emit_codes = [&](const uint32_t (&r)[16], int j0) {
         uint8_t* sb = stage_buf();
         const uint16_t* tab = reinterpret_cast<const uint16_t*>(smem + C::OFF_TOK + C::OFF_GELU_TAB);
-        uint32_t hb[16];
-        bool rare = false;
+        float off[16];
+        const int sd_l = sds[j0 + (lane & 15)];
+        const int sd0 = sds[j0];
+        if (__all_sync(0xFFFFFFFFu, sd_l == sd0)) {  // one stream in the chunk (the usual case)
+          const float o = offset(sd0);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float v =
-              fmaf(sts[j0 + j] * sw, __int2float_rn(static_cast<int>(r[j])), offset(sds[j0 + j]));
-          const uint32_t yb = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-          const int ti = gelu_tab_index(yb);
-          hb[j] = ti >= 0 ? tab[ti] : (yb | 0x80000000u);  // high bit: evaluate below
-          rare = rare || ti < 0;
+          for (int j = 0; j < 16; ++j) off[j] = o;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) off[j] = offset(sds[j0 + j]);
         }
-        if (rare) {
+        const float4* st4 = reinterpret_cast<const float4*>(sts + j0);
+        const float2 sw2 = make_float2(sw, sw);
+        uint32_t hb[16];
+        uint32_t rare = 0;
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+          const float4 t = st4[j4];
+#pragma unroll
+          for (int p = 0; p < 2; ++p) {
+            const int j = 4 * j4 + 2 * p;
+            const float2 s2 = __fmul2_rn(p ? make_float2(t.z, t.w) : make_float2(t.x, t.y), sw2);
+            const float2 a2 = make_float2(__int2float_rn(static_cast<int>(r[j])),
+                                          __int2float_rn(static_cast<int>(r[j + 1])));
+            const float2 v2 = __ffma2_rn(s2, a2, make_float2(off[j], off[j + 1]));
+            const uint32_t y2 = bf162_bits(__floats2bfloat162_rn(v2.x, v2.y));
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const uint32_t yb = k ? y2 >> 16 : y2 & 0xFFFFu;
+              // table row: exponent field kGeluTabExp0.., either sign
+              const uint32_t mag = yb & 0x7FFFu;
+              const uint32_t u = mag - (kGeluTabExp0 << 7);
+              const bool in = u < static_cast<uint32_t>(kGeluTabExps * 128);
+              const uint32_t ti = in ? u + (yb >> 15) * (kGeluTabExps * 128) : 0u;
+              const uint32_t hv = tab[ti];
+              // Outside the table, the correctly rounded GELU in closed form:
+              //  * normal |y| < 2^-10: GELU(y) = y/2 (1 + erf(y/sqrt2)) with
+              //    |erf(y/sqrt2)| < 0.0008, under half of bf16's relative spacing (2^-9),
+              //    so h = y/2 exactly: the exponent field minus one;
+              //  * finite |y| >= 16: 1 - Phi(16) < 2^-60, so h = y for y > 0, and h = -0
+              //    for y < 0 (|GELU(y)| < 2^-180, far below bf16's smallest subnormal).
+              // Zeros, subnormals, infinities and NaN are evaluated.
+              const bool tiny = mag - 0x100u < (kGeluTabExp0 << 7) - 0x100u;
+              const bool wide = mag - (kGeluTabEnd << 7) < 0x7F80u - (kGeluTabEnd << 7);
+              const uint32_t hx = tiny ? yb - 0x80u : yb & (0xFFFFu ^ ((yb >> 15) * 0x7FFFu));
+              hb[j + k] = in               ? hv
+                          : (tiny || wide) ? hx
+                                           : (yb | 0x80000000u);  // high bit: evaluate below
+              rare |= hb[j + k];
+            }
+          }
+        }
+        if (rare & 0x80000000u) {
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             if (hb[j] & 0x80000000u) hb[j] = gelu_bf16_eval(hb[j] & 0xFFFFu);
@@ -764,26 +813,42 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             if (m0 + j0 + j < args.M) args.g_h[(size_t)(m0 + j0 + j) * args.N + n] = hb[j];
         }
         constexpr float kq = static_cast<float>(C::QMAX_NEXT);
+        const float4* rn4 = reinterpret_cast<const float4*>(g_s + C::BN + j0);
+        const float2 ci2 = make_float2(g_ci, g_ci);
+        const float2 m2 = make_float2(kRoundMagic, kRoundMagic);
+        const float2 nm2 = make_float2(-kRoundMagic, -kRoundMagic);
+        const float2 neg1 = make_float2(-1.0f, -1.0f);
         uint32_t code[16];
-        bool slow = false;
+        bool ok = true;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float xv = __fmul_rn(__uint_as_float(hb[j] << 16), g_ci);
-          const float sn = g_s[j0 + j], rn = g_s[C::BN + j0 + j];
-          const float t = __fmul_rn(xv, rn);
-          const float u = __fadd_rn(t, kRoundMagic);
-          const float d = __fsub_rn(t, __fsub_rn(u, kRoundMagic));
-          slow = slow || fabsf(d) >= 0.5f - 0x1p-12f || !(sn > 0.0f) || !isfinite(rn);
-          code[j] = __float_as_uint(fminf(fmaxf(u, kRoundMagic - kq), kRoundMagic + kq));
+        for (int j4 = 0; j4 < 4; ++j4) {
+          const float4 rv = rn4[j4];
+#pragma unroll
+          for (int p = 0; p < 2; ++p) {
+            const int j = 4 * j4 + 2 * p;
+            const float2 x2 = __fmul2_rn(
+                make_float2(__uint_as_float(hb[j] << 16), __uint_as_float(hb[j + 1] << 16)), ci2);
+            const float2 t = __fmul2_rn(x2, p ? make_float2(rv.z, rv.w) : make_float2(rv.x, rv.y));
+            const float2 u = __fadd2_rn(t, m2);                        // magic + rint(t)
+            const float2 d = __ffma2_rn(__fadd2_rn(u, nm2), neg1, t);  // t - rint(t), exact
+            // the fast code is exact unless t lies near a half-integer inside the
+            // range (|t| >= QMAX + 1 clamps either way); a NaN t (NaN h, a bad scale
+            // staged as a NaN reciprocal) fails the test too
+            ok = ok && (fabsf(d.x) < 0.5f - 0x1p-12f || fabsf(t.x) >= kq + 1.0f) &&
+                 (fabsf(d.y) < 0.5f - 0x1p-12f || fabsf(t.y) >= kq + 1.0f);
+            code[j] = __float_as_uint(fminf(fmaxf(u.x, kRoundMagic - kq), kRoundMagic + kq));
+            code[j + 1] = __float_as_uint(fminf(fmaxf(u.y, kRoundMagic - kq), kRoundMagic + kq));
+          }
         }
-        if (slow) {  // exact codes for every element of the chunk (as quantize1_recip)
+        if (!ok) {  // exact codes where the fast one may differ
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const float xv = __fmul_rn(__uint_as_float(hb[j] << 16), g_ci);
-            const float sn = g_s[j0 + j], rn = g_s[C::BN + j0 + j];
-            code[j] = (sn > 0.0f && isfinite(rn))
-                          ? quantize1_recip<C::QMAX_NEXT>(xv, sn, rn)
-                          : static_cast<uint32_t>(quantize<C::QMAX_NEXT>(xv, sn));
+            const float rn = g_s[C::BN + j0 + j];
+            const float t = __fmul_rn(xv, rn);
+            const float d = __fsub_rn(t, __fsub_rn(__fadd_rn(t, kRoundMagic), kRoundMagic));
+            if (!(fabsf(d) < 0.5f - 0x1p-12f || fabsf(t) >= kq + 1.0f))
+              code[j] = code_exact_next<C::QMAX_NEXT>(xv, g_s[j0 + j], rn);
           }
         }
 #pragma unroll
