@@ -85,7 +85,7 @@ struct TileArgs {
   int splits;     // K ranges per tile (1: no split)
   int num_units;  // num_tiles * splits work units, unit = tile * splits + split
   int32_t* partial;  // bf16 split: [tiles][BN][128] int32 sums of the splits (zeroed)
-  int* counters;     // bf16 split: [tiles][8] arrivals per epilogue-warp slice
+  int* counters;     // split K: [tiles][kMaxEpiWarps] arrivals per epilogue-warp slice
   int w_prefetch;    // weights of the first NS K blocks loaded before griddep_wait()
   // single-kernel linear (Cfg QBITS > 0): the bf16 activations, the channel
   // scale [K] (or null) and the clip ratios [T][S] the kernel quantizes with
@@ -153,17 +153,21 @@ struct Cfg {
   static constexpr int BM = 128;  // output channels per tile (MMA M)
   static constexpr int BK = 128;  // K elements per pipeline stage
   static constexpr int UNPACK_WARPS = ACT_BITS == 4 ? 8 : WQ_UNPACK_WARPS_A8;
-  static constexpr int EPI_WARPS = 8;  // two per TMEM lane quadrant
+  // epilogue warps per TMEM lane quadrant: three for the GELU-and-quantize
+  // epilogue, whose longer per-element path would otherwise outlast the mainloop
+  static constexpr int EPI_PER_Q = EPI ? 3 : 2;
+  static constexpr int EPI_WARPS = 4 * EPI_PER_Q;
+  static_assert(EPI_WARPS <= kMaxEpiWarps, "split-K counters hold kMaxEpiWarps per tile");
   static constexpr int EPI_THREADS = EPI_WARPS * 32;
   // Warp roles: warp 0 issues TMA, warp 1 issues MMAs, then the unpack warps,
-  // then the epilogue warps (two per TMEM lane quadrant, warp % 4).
+  // then the epilogue warps (EPI_PER_Q per TMEM lane quadrant, warp % 4).
   static constexpr int NUM_WARPS = 2 + UNPACK_WARPS + EPI_WARPS;
   static constexpr int THREADS = NUM_WARPS * 32;
   // index among the unpack warps, or -1
   __device__ static int unpack_index(int w) {
     return (w >= 2 && w < 2 + UNPACK_WARPS) ? w - 2 : -1;
   }
-  // index among the epilogue warps (quadrant w % 4, half e / 4), or -1
+  // index among the epilogue warps (quadrant w % 4, chunk phase e / 4), or -1
   __device__ static int epi_index(int w) {
     return (w >= 2 + UNPACK_WARPS && w < NUM_WARPS) ? w - 2 - UNPACK_WARPS : -1;
   }
@@ -890,12 +894,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // split K: the tile's int32 accumulator (2^ACC_SHIFT-scaled), summed by red.add
       int32_t* tile_acc =
           split ? args.partial + (size_t)tile * C::BN * C::BM + q * 32 + lane : nullptr;
-      for (int c = h; c < C::NUM_CHUNKS; c += 2) {
+      for (int c = h; c < C::NUM_CHUNKS; c += C::EPI_PER_Q) {
         const int j0 = c * C::EPI_CHUNK;
         uint32_t r[16];
         tmem_ld_32x32b_x16(tbase + j0, r);
         tmem_wait_ld();
-        if (c + 2 >= C::NUM_CHUNKS) {  // last chunk of this warp: hand the accumulator back
+        if (c + C::EPI_PER_Q >= C::NUM_CHUNKS) {  // last chunk of this warp: hand the accumulator back
           tc_fence_before();
           __syncwarp();
           if (lane == 0) {
@@ -923,7 +927,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
         if (prev == args.splits - 1) {
           __threadfence();
-          for (int c = h; c < C::NUM_CHUNKS; c += 2) {
+          for (int c = h; c < C::NUM_CHUNKS; c += C::EPI_PER_Q) {
             const int j0 = c * C::EPI_CHUNK;
             if (m0 + j0 >= args.M) continue;
             uint32_t r[16];
@@ -1164,7 +1168,7 @@ size_t gemm_split_scratch_bytes(int M, int N, int K) {
   const int BN = bn_for(M);
   const size_t tiles = static_cast<size_t>((M + BN - 1) / BN) * ((N + 127) / 128);
   const size_t partial = tiles * BN * 128 * sizeof(int32_t);
-  const size_t counters = tiles * 8 * sizeof(int);
+  const size_t counters = tiles * kMaxEpiWarps * sizeof(int);
   return (partial + 255) / 256 * 256 + (counters + 255) / 256 * 256;
 }
 

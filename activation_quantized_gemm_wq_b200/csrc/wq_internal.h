@@ -106,12 +106,14 @@ cudaError_t launch_linear_single(const uint16_t* x, const float* cinv, const flo
 // scratch for the int32 partial tiles and one counter per epilogue-warp slice of
 // each tile.
 constexpr int kSplitTargetCtas = 148;
+// epilogue warps of a GEMM CTA at most (the split-K counters hold one per warp and tile)
+constexpr int kMaxEpiWarps = 12;
 int gemm_splits(int M, int N, int K);
 size_t gemm_split_scratch_bytes(int M, int N, int K);  // partials + counters, 0 if no split
 
 struct SplitScratch {
   int32_t* partial;  // [tiles][BN][128] int32 sums of the splits, zero before the launch
-  int* counters;     // [tiles][8], zero before the launch
+  int* counters;     // [tiles][kMaxEpiWarps], zero before the launch
 };
 
 // Optional parts of a GEMM launch.
