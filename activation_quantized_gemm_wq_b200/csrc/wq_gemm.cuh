@@ -133,7 +133,11 @@ __device__ __forceinline__ void split_range(int num_k, int splits, int sp, int& 
 // each CTA's TMEM receives the accumulators of its own 128 channels for all BN
 // tokens, which its epilogue writes.  Per SM this halves the activation tile's
 // copy and the tensor core's reads of it from shared memory.
-template <int BN_, int ACT_BITS_, int QBITS_ = 0, int EPI_ = 0, bool PAIR_ = false>
+// KS: 128-deep K sub-blocks per pipeline stage.  The TMA engine moves a box row by
+// row, and a 64-byte row of packed weights (128 K) streams at about 40 GB/s per
+// SM, a 128-byte row at about 70: narrow token tiles, whose time is the weights'
+// stream, take 256-deep stages (KS = 2) so that each weight row is 128 bytes.
+template <int BN_, int ACT_BITS_, int QBITS_ = 0, int EPI_ = 0, bool PAIR_ = false, int KS_ = 1>
 struct Cfg {
   static constexpr int BN = BN_;
   static constexpr bool PAIR = PAIR_;
@@ -150,8 +154,11 @@ struct Cfg {
                 "the GELU-and-quantize epilogue follows the int8-activation mainloop");
   static_assert(!PAIR || (QBITS == 0 && BN == 256 && ACT_BITS == 8),
                 "CTA pairs serve the 256-token tiles of int8 activation codes");
-  static constexpr int BM = 128;  // output channels per tile (MMA M)
-  static constexpr int BK = 128;  // K elements per pipeline stage
+  static constexpr int KS = KS_;
+  static_assert(KS == 1 || (KS == 2 && !PAIR && QBITS == 0 && BN <= 64),
+                "256-deep stages serve the narrow token tiles of the two-kernel path");
+  static constexpr int BM = 128;       // output channels per tile (MMA M)
+  static constexpr int BK = 128 * KS;  // K elements per pipeline stage
   static constexpr int UNPACK_WARPS = ACT_BITS == 4 ? 8 : WQ_UNPACK_WARPS_A8;
   // epilogue warps per TMEM lane quadrant: three for the GELU-and-quantize
   // epilogue, whose longer per-element path would otherwise outlast the mainloop
@@ -159,32 +166,46 @@ struct Cfg {
   static constexpr int EPI_WARPS = 4 * EPI_PER_Q;
   static_assert(EPI_WARPS <= kMaxEpiWarps, "split-K counters hold kMaxEpiWarps per tile");
   static constexpr int EPI_THREADS = EPI_WARPS * 32;
-  // Warp roles: warp 0 issues TMA, warp 1 issues MMAs, then the unpack warps,
-  // then the epilogue warps (EPI_PER_Q per TMEM lane quadrant, warp % 4).
-  static constexpr int NUM_WARPS = 2 + UNPACK_WARPS + EPI_WARPS;
+  // MMA-issuing warps.  One thread issues a K block's four MMAs and its commit in
+  // about 235 cycles, and its wait (with acquire) for the unpacked operands costs
+  // about 200 more while its earlier MMAs are in flight: 440 cycles per K block,
+  // above the tensor work of a tile narrower than 256 tokens (4 x N/2 cycles).
+  // Narrow tiles therefore spread their K blocks over several issuing warps, each
+  // accumulating into its own TMEM columns; the epilogue adds the partial sums.
+  // (The GELU-and-quantize epilogue's twelve warps leave registers for two.)
+  static constexpr int MMA_WARPS =
+      PAIR ? 1 : BN <= 64 ? (EPI || KS == 2 ? 2 : 4) : BN == 128 ? 2 : 1;
+  // Warp roles: warp 0 issues TMA, warps 1..MMA_WARPS issue MMAs, then the unpack
+  // warps, then the epilogue warps (EPI_PER_Q per TMEM lane quadrant, warp % 4).
+  static constexpr int NUM_WARPS = 1 + MMA_WARPS + UNPACK_WARPS + EPI_WARPS;
   static constexpr int THREADS = NUM_WARPS * 32;
+  // index among the MMA-issuing warps, or -1
+  __device__ static int mma_index(int w) { return (w >= 1 && w <= MMA_WARPS) ? w - 1 : -1; }
   // index among the unpack warps, or -1
   __device__ static int unpack_index(int w) {
-    return (w >= 2 && w < 2 + UNPACK_WARPS) ? w - 2 : -1;
+    return (w > MMA_WARPS && w <= MMA_WARPS + UNPACK_WARPS) ? w - 1 - MMA_WARPS : -1;
   }
   // index among the epilogue warps (quadrant w % 4, chunk phase e / 4), or -1
   __device__ static int epi_index(int w) {
-    return (w >= 2 + UNPACK_WARPS && w < NUM_WARPS) ? w - 2 - UNPACK_WARPS : -1;
+    return (w > MMA_WARPS + UNPACK_WARPS && w < NUM_WARPS) ? w - 1 - MMA_WARPS - UNPACK_WARPS
+                                                           : -1;
   }
 
   static constexpr int WP_BYTES = BM * BK / 2;                               // packed W
   static constexpr int WU_BYTES = BM * BK;                                   // int8 W
   static constexpr int XS_BYTES = ACT_BITS == 8 ? BNX * BK : BNX * BK / 2;   // staged x
   static constexpr int XU_BYTES = ACT_BITS == 8 ? 0 : BNX * BK;             // int8 x (A4)
+  // one 128-deep sub-block of an int8 operand tile: [rows][128 B], 128-byte swizzle
+  static constexpr int SUB_W = BM * 128;
+  static constexpr int SUB_X = BNX * 128;
   static constexpr int XB_BYTES = QBITS ? BN * BK * 2 : 0;                  // staged bf16 x
   static constexpr int STAGE_BYTES = WP_BYTES + (QBITS ? XB_BYTES : XS_BYTES);  // TMA bytes
   static constexpr int STAGE_SMEM = WP_BYTES + XS_BYTES + XB_BYTES;
   // Pipeline: NS TMA stages (packed weights + activation tile), NU unpacked
   // buffers, and one "MMA done with K block g" barrier per stage (a ring of NS).
-  // The single MMA-issuing thread does one wait and one commit per K block: it
-  // can queue barely one instruction ahead of the tensor pipe, so its per-block
-  // overhead, not the pipeline depth alone, decides whether the pipe stays fed.
-  static constexpr int NU = ACT_BITS == 8 ? 3 : 2;
+  // Each MMA-issuing thread does one wait and one commit per K block of its own.
+  static constexpr int NU_BASE = ACT_BITS == 8 && KS == 1 ? 3 : 2;
+  static constexpr int NU = MMA_WARPS > NU_BASE ? MMA_WARPS : NU_BASE;
   static constexpr int EPI_ELEM = 2;  // bf16 y (the codes of EPI > 0 use half of it)
   // The tensor cores accumulate 16x (int8 activations) or 256x (both operands
   // unpacked from int4) the code products; see unpack32.
@@ -208,7 +229,9 @@ struct Cfg {
   static constexpr int EPI_NBUF = NS_WITH_2 >= 4 ? 2 : 1;
   static constexpr int EPI_BYTES = EPI_WARPS * EPI_NBUF * EPI_BUF_BYTES;
   static constexpr int NS_FIT = (SMEM_LIMIT - FIXED - EPI_BYTES) / STAGE_SMEM;
-  static constexpr int NS = NS_FIT > WQ_MAX_STAGES ? WQ_MAX_STAGES : NS_FIT;
+  // narrow tiles stream weights with little else to do: let more copies fly
+  static constexpr int NS_CAP = BN <= 64 ? 2 * WQ_MAX_STAGES : WQ_MAX_STAGES;
+  static constexpr int NS = NS_FIT > NS_CAP ? NS_CAP : NS_FIT;
   static_assert(NS >= NU && NS >= 2, "the done ring needs NS >= NU");
   static_assert(BN % EPI_CHUNK == 0 && NUM_CHUNKS >= 1, "token tile is a multiple of 16");
 
@@ -227,8 +250,14 @@ struct Cfg {
                     OFF_XU % 1024 == 0 && OFF_EPI % 1024 == 0 && OFF_BAR % 8 == 0,
                 "swizzled tiles need 1024-byte alignment");
 
-  static constexpr uint32_t TMEM_COLS =
-      2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
+  // two tile buffers x MMA_WARPS partial accumulators of BN columns
+  static constexpr int ACC_COLS = 2 * MMA_WARPS * BN;
+  static_assert(ACC_COLS <= 512, "TMEM holds 512 columns");
+  static constexpr uint32_t TMEM_COLS = ACC_COLS <= 32    ? 32
+                                        : ACC_COLS <= 64  ? 64
+                                        : ACC_COLS <= 128 ? 128
+                                        : ACC_COLS <= 256 ? 256
+                                                          : 512;
 };
 
 __device__ __forceinline__ void decode_tile(const TileArgs& a, int tile, int& n_tile,
@@ -270,32 +299,36 @@ __device__ __forceinline__ void unpack32(const uint4 p, uint4& lo16, uint4& hi16
   hi16 = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// Packed tile [ROWS][64 B] with the 64-byte swizzle -> int8 tile [ROWS][128 B]
-// with the 128-byte swizzle.  Task i covers row i/4, packed 16-byte chunk i%4;
-// each thread issues all of its loads before converting (latency hiding).
-template <int ROWS, int NT, bool NATURAL>
+// Packed tile [ROWS][64 KS bytes] (KS = 1: 64-byte rows, 64-byte swizzle; KS = 2:
+// 128-byte rows, 128-byte swizzle) -> KS int8 sub-tiles [ROWS][128 B] with the
+// 128-byte swizzle, ROWS * 128 bytes apart.  Task i covers row i / (4 KS), packed
+// 16-byte chunk p = i % (4 KS), which holds k = 32p .. 32p + 31: sub-tile p / 4.
+// Each thread issues all of its loads before converting (latency hiding).
+template <int ROWS, int NT, bool NATURAL, int KS = 1>
 __device__ __forceinline__ void unpack_tile(const uint8_t* src, uint8_t* dst, int tid) {
-  constexpr int TASKS = ROWS * 4;
+  constexpr int CPR = 4 * KS;  // packed chunks per row
+  constexpr int TASKS = ROWS * CPR;
   constexpr int PER = (TASKS + NT - 1) / NT;
   uint4 v[PER];
 #pragma unroll
   for (int k = 0; k < PER; ++k) {
     const int i = tid + k * NT;
     if (TASKS % NT == 0 || i < TASKS) {
-      const int r = i >> 2, p = i & 3;
-      v[k] = *reinterpret_cast<const uint4*>(src + r * 64 + ((p ^ ((r >> 1) & 3)) << 4));
+      const int r = i / CPR, p = i % CPR;
+      const int sw = KS == 1 ? (p ^ ((r >> 1) & 3)) : (p ^ (r & 7));
+      v[k] = *reinterpret_cast<const uint4*>(src + r * (16 * CPR) + (sw << 4));
     }
   }
 #pragma unroll
   for (int k = 0; k < PER; ++k) {
     const int i = tid + k * NT;
     if (TASKS % NT == 0 || i < TASKS) {
-      const int r = i >> 2, p = i & 3;
+      const int r = i / CPR, p = i % CPR, pp = p & 3;
       uint4 lo, hi;
       unpack32<NATURAL>(v[k], lo, hi);
-      uint8_t* row = dst + r * 128;
-      *reinterpret_cast<uint4*>(row + (((2 * p) ^ (r & 7)) << 4)) = lo;
-      *reinterpret_cast<uint4*>(row + (((2 * p + 1) ^ (r & 7)) << 4)) = hi;
+      uint8_t* row = dst + (p >> 2) * (ROWS * 128) + r * 128;
+      *reinterpret_cast<uint4*>(row + (((2 * pp) ^ (r & 7)) << 4)) = lo;
+      *reinterpret_cast<uint4*>(row + (((2 * pp + 1) ^ (r & 7)) << 4)) = hi;
     }
   }
 }
@@ -335,12 +368,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // a pair's unpack and epilogue warps of both CTAs arrive on rank 0's barriers
     for (int u = 0; u < C::NU; ++u) mbar_init(&ufull[u], C::UNPACK_WARPS * (C::PAIR ? 2 : 1));
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull[b], 1);
+      mbar_init(&tfull[b], C::MMA_WARPS);
       mbar_init(&tempty[b], C::EPI_WARPS * (C::PAIR ? 2 : 1));
       mbar_init(&tokbar[b], C::EPI_WARPS);
     }
     mbar_init(qready, C::EPI_WARPS);
-    mbar_init(mma_drained, 1);
+    mbar_init(mma_drained, C::MMA_WARPS);
     fence_mbar_init();
     fence_proxy_async_smem();
   }
@@ -415,9 +448,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         m_tile * C::BN);
             tma_load_2d(smem + C::OFF_XB + s * C::XB_BYTES + C::BN * 128, &tm_x, &full[s],
                         kb * C::BK + 64, m_tile * C::BN);
-          } else {
-            tma_load_2d(smem + C::OFF_XS + s * C::XS_BYTES, &tm_x, &full[s],
-                        kb * (C::ACT_BITS == 8 ? C::BK : C::BK / 2),
+          } else if constexpr (C::ACT_BITS == 8) {  // KS boxes of 128 channels
+#pragma unroll
+            for (int i = 0; i < C::KS; ++i)
+              tma_load_2d(smem + C::OFF_XS + s * C::XS_BYTES + i * C::SUB_X, &tm_x, &full[s],
+                          kb * C::BK + i * 128, m_tile * C::BN + rank * C::BNX);
+          } else {  // packed int4: one box of BK / 2 bytes per token row
+            tma_load_2d(smem + C::OFF_XS + s * C::XS_BYTES, &tm_x, &full[s], kb * (C::BK / 2),
                         m_tile * C::BN + rank * C::BNX);
           }
         }
@@ -432,11 +469,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // Per K block: one wait (its unpacked buffer; the unpack warps arrive there
-    // only after the stage's TMA landed, which orders the activation tile too),
-    // four MMAs, one commit (frees the stage and the unpacked buffer).
+  } else if (C::mma_index(warp) >= 0) {
+    // ------------------------------------------------------------ MMA issuers
+    // Issuer i takes the K blocks kb0 + i, kb0 + i + MMA_WARPS, ... of each tile
+    // into its own accumulator.  Per K block: one wait (its unpacked buffer; the
+    // unpack warps arrive there only after the stage's TMA landed, which orders
+    // the activation tile too), four MMAs, one commit (frees the stage and the
+    // unpacked buffer).  Every issuer commits the tile's tfull once.
+    const int mi = C::mma_index(warp);
     if (lane == 0 && rank == 0) {
       constexpr uint32_t idesc = idesc_i8(C::BN, C::PAIR ? 256u : 128u);
       uint32_t g = 0;
@@ -448,8 +488,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         split_range(num_k, args.splits, unit % args.splits, kb0, kb1);
         if (!mbar_wait(&tempty[b], ph_b ^ 1u)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * C::BN);
+        const uint32_t d_tmem =
+            tmem_base + static_cast<uint32_t>((b * C::MMA_WARPS + mi) * C::BN);
         for (int kb = kb0; kb < kb1; ++kb, ++g) {
+          if ((kb - kb0) % C::MMA_WARPS != mi) continue;
           const uint32_t s = g % C::NS, u = g % C::NU;
           if (!mbar_wait(&ufull[u], (g / C::NU) & 1u)) { ok = false; break; }
           tc_fence_after();
@@ -458,10 +500,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                : smem_u32(smem + C::OFF_XU + u * C::XU_BYTES);
           const uint32_t a_addr = smem_u32(smem + C::OFF_WU + u * C::WU_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < C::BK / 32; ++kk) {
-            const uint64_t ad = smem_desc_sw128(a_addr + kk * 32);
-            const uint64_t bd = smem_desc_sw128(b_addr + kk * 32);
-            const uint32_t acc = (kb != kb0 || kk != 0) ? 1u : 0u;
+          for (int kk = 0; kk < C::BK / 32; ++kk) {  // sub-block kk / 4, 32 deep each
+            const uint64_t ad = smem_desc_sw128(a_addr + (kk >> 2) * C::SUB_W + (kk & 3) * 32);
+            const uint64_t bd = smem_desc_sw128(b_addr + (kk >> 2) * C::SUB_X + (kk & 3) * 32);
+            const uint32_t acc = (kb - kb0 >= C::MMA_WARPS || kk != 0) ? 1u : 0u;
             if constexpr (C::PAIR) mma_i8_ss_pair(d_tmem, ad, bd, idesc, acc);
             else mma_i8_ss(d_tmem, ad, bd, idesc, acc);
           }
@@ -506,11 +548,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         // int8 activations arrive in k order, so the weights must too; int4
         // activations are unpacked exactly like the weights, so both may keep
         // the cheaper permuted order.
-        unpack_tile<C::BM, NT, C::ACT_BITS == 8>(smem + C::OFF_WP + s * C::WP_BYTES,
-                                                 smem + C::OFF_WU + u * C::WU_BYTES, tid);
+        unpack_tile<C::BM, NT, C::ACT_BITS == 8, C::KS>(smem + C::OFF_WP + s * C::WP_BYTES,
+                                                        smem + C::OFF_WU + u * C::WU_BYTES, tid);
         if constexpr (C::ACT_BITS == 4) {
-          unpack_tile<C::BNX, NT, false>(smem + C::OFF_XS + s * C::XS_BYTES,
-                                         smem + C::OFF_XU + u * C::XU_BYTES, tid);
+          unpack_tile<C::BNX, NT, false, C::KS>(smem + C::OFF_XS + s * C::XS_BYTES,
+                                                smem + C::OFF_XU + u * C::XU_BYTES, tid);
         }
         if constexpr (C::QBITS > 0) {
           // chunk i: token row i / 16, channels 8*(i % 16) .. +7 of this K block
@@ -889,8 +931,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           else mbar_arrive(&tempty[b]);
         }
       }
-      const uint32_t tbase =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * C::BN);
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(b * C::MMA_WARPS * C::BN);
+      // issuers that accumulated into this tile (one per K block, up to MMA_WARPS)
+      int nparts = 1;
+      if constexpr (C::MMA_WARPS > 1) {
+        int kb0, kb1;
+        split_range(num_k, args.splits, unit % args.splits, kb0, kb1);
+        nparts = kb1 - kb0 < C::MMA_WARPS ? kb1 - kb0 : C::MMA_WARPS;
+      }
       // split K: the tile's int32 accumulator (2^ACC_SHIFT-scaled), summed by red.add
       int32_t* tile_acc =
           split ? args.partial + (size_t)tile * C::BN * C::BM + q * 32 + lane : nullptr;
@@ -898,6 +947,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const int j0 = c * C::EPI_CHUNK;
         uint32_t r[16];
         tmem_ld_32x32b_x16(tbase + j0, r);
+#pragma unroll
+        for (int p = 1; p < C::MMA_WARPS; ++p) {  // the other issuers' partial sums
+          if (p < nparts) {
+            uint32_t t[16];
+            tmem_ld_32x32b_x16(tbase + p * C::BN + j0, t);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) r[j] += t[j];  // int32 sums: exact in any order
+          }
+        }
         tmem_wait_ld();
         if (c + C::EPI_PER_Q >= C::NUM_CHUNKS) {  // last chunk of this warp: hand the accumulator back
           tc_fence_before();
@@ -1015,17 +1074,20 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
                      cudaStream_t st, bool w_prefetch, const SingleArgs* single,
                      const GemmExtras* ex) {
   CUtensorMap tm_w, tm_x, tm_out;
+  // packed rows of BK / 2 bytes: 64 (64-byte swizzle) or 128 (128-byte swizzle)
+  constexpr CUtensorMapSwizzle kPackedSwizzle =
+      C::KS == 1 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   bool ok = make_map(&tm_w, qw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, C::BK / 2, C::BM,
-                     CU_TENSOR_MAP_SWIZZLE_64B);
+                     kPackedSwizzle);
   if (C::QBITS > 0)  // bf16 activations, boxes of 64 channels x BN tokens
     ok = ok && single && make_map(&tm_x, single->x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, 64,
                                   C::BN, CU_TENSOR_MAP_SWIZZLE_NONE);
   else if (C::ACT_BITS == 8)  // each CTA of a pair loads half of the token tile
-    ok = ok && make_map(&tm_x, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, C::BK, C::BNX,
+    ok = ok && make_map(&tm_x, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128, C::BNX,
                         CU_TENSOR_MAP_SWIZZLE_128B);
   else
     ok = ok && make_map(&tm_x, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, C::BK / 2, C::BNX,
-                        CU_TENSOR_MAP_SWIZZLE_64B);
+                        kPackedSwizzle);
   int32_t* acc_out = ex ? ex->acc_out : nullptr;
   if (out == nullptr && acc_out == nullptr) return cudaErrorInvalidValue;
   if (C::EPI > 0)  // the next linear's int8 codes [M][N], boxes of 32 channels x 16 tokens
@@ -1110,13 +1172,24 @@ cudaError_t dispatch_bn(const void* qx, const uint8_t* qw, int M, int N, int K,
       return run_gemm<Cfg<256, 8, 0, EPI, true>>(qx, qw, M, N, K, ep, out, nullptr, st, wp,
                                                  nullptr, ex);
   }
+  // narrow token tiles stream 256-deep stages when K allows
+  const bool ks2 = K % 256 == 0;
   switch (bn_for(M)) {
     case 16:
-      return run_gemm<Cfg<16, ACT_BITS, 0, EPI>>(qx, qw, M, N, K, ep, out, sc, st, wp, nullptr, ex);
+      return ks2 ? run_gemm<Cfg<16, ACT_BITS, 0, EPI, false, 2>>(qx, qw, M, N, K, ep, out, sc, st,
+                                                                  wp, nullptr, ex)
+                 : run_gemm<Cfg<16, ACT_BITS, 0, EPI>>(qx, qw, M, N, K, ep, out, sc, st, wp,
+                                                       nullptr, ex);
     case 32:
-      return run_gemm<Cfg<32, ACT_BITS, 0, EPI>>(qx, qw, M, N, K, ep, out, sc, st, wp, nullptr, ex);
+      return ks2 ? run_gemm<Cfg<32, ACT_BITS, 0, EPI, false, 2>>(qx, qw, M, N, K, ep, out, sc, st,
+                                                                  wp, nullptr, ex)
+                 : run_gemm<Cfg<32, ACT_BITS, 0, EPI>>(qx, qw, M, N, K, ep, out, sc, st, wp,
+                                                       nullptr, ex);
     case 64:
-      return run_gemm<Cfg<64, ACT_BITS, 0, EPI>>(qx, qw, M, N, K, ep, out, sc, st, wp, nullptr, ex);
+      return ks2 ? run_gemm<Cfg<64, ACT_BITS, 0, EPI, false, 2>>(qx, qw, M, N, K, ep, out, sc, st,
+                                                                  wp, nullptr, ex)
+                 : run_gemm<Cfg<64, ACT_BITS, 0, EPI>>(qx, qw, M, N, K, ep, out, sc, st, wp,
+                                                       nullptr, ex);
     case 128:
       return run_gemm<Cfg<128, ACT_BITS, 0, EPI>>(qx, qw, M, N, K, ep, out, sc, st, wp, nullptr,
                                                    ex);

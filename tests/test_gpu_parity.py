@@ -107,7 +107,9 @@ def test_act_quant_near_ties(oracle, bits, qmax):
 # the last four split K over several CTAs (few output tiles), as the fused linear does
 GEMM_SHAPES = [(1, 16, 128), (16, 144, 256), (17, 128, 512), (64, 256, 256), (100, 272, 384),
                (128, 128, 128), (129, 400, 256), (300, 384, 512), (513, 128, 1024),
-               (16, 128, 4096), (40, 512, 2048), (100, 1024, 1024), (256, 2048, 2048)]
+               (16, 128, 4096), (40, 512, 2048), (100, 1024, 1024), (256, 2048, 2048),
+               # K % 256 == 128 at narrow token tiles: 128-deep stages over 2-4 issuers
+               (33, 256, 384), (48, 192, 1152)]
 
 
 @pytest.mark.parametrize("bits", [8, 4])
