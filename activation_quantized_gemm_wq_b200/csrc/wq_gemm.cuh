@@ -73,6 +73,14 @@ __device__ __noinline__ uint32_t code_exact_next(float xv, float sn, float rn) {
                                      : static_cast<uint32_t>(quantize<QMAX>(xv, sn));
 }
 
+// v clamped to [-q, q], NaN kept (PTX min/max with .NaN propagate it).
+__device__ __forceinline__ float clamp_nan(float v, float q) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(v), "f"(-q));
+  asm("min.NaN.f32 %0, %0, %1;" : "+f"(r) : "f"(q));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 v) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
@@ -875,15 +883,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const float2 x2 = __fmul2_rn(
                 make_float2(__uint_as_float(hb[j] << 16), __uint_as_float(hb[j + 1] << 16)), ci2);
             const float2 t = __fmul2_rn(x2, p ? make_float2(rv.z, rv.w) : make_float2(rv.x, rv.y));
-            const float2 u = __fadd2_rn(t, m2);                        // magic + rint(t)
-            const float2 d = __ffma2_rn(__fadd2_rn(u, nm2), neg1, t);  // t - rint(t), exact
-            // the fast code is exact unless t lies near a half-integer inside the
-            // range (|t| >= QMAX + 1 clamps either way); a NaN t (NaN h, a bad scale
-            // staged as a NaN reciprocal) fails the test too
-            ok = ok && (fabsf(d.x) < 0.5f - 0x1p-12f || fabsf(t.x) >= kq + 1.0f) &&
-                 (fabsf(d.y) < 0.5f - 0x1p-12f || fabsf(t.y) >= kq + 1.0f);
-            code[j] = __float_as_uint(fminf(fmaxf(u.x, kRoundMagic - kq), kRoundMagic + kq));
-            code[j + 1] = __float_as_uint(fminf(fmaxf(u.y, kRoundMagic - kq), kRoundMagic + kq));
+            // clamp first: beyond +-QMAX the exact quotient (within |t| 2^-22 of t)
+            // rounds to the same end, so only t inside the range is rounded; the clamp
+            // keeps a NaN t (NaN h, a bad scale staged as a NaN reciprocal)
+            const float2 tc = make_float2(clamp_nan(t.x, kq), clamp_nan(t.y, kq));
+            const float2 u = __fadd2_rn(tc, m2);                         // magic + rint(tc)
+            const float2 d = __ffma2_rn(__fadd2_rn(u, nm2), neg1, tc);   // tc - rint(tc)
+            // exact unless tc lies near a half-integer; NaN fails the test too
+            ok = ok && fabsf(d.x) < 0.5f - 0x1p-12f && fabsf(d.y) < 0.5f - 0x1p-12f;
+            code[j] = __float_as_uint(u.x);
+            code[j + 1] = __float_as_uint(u.y);
           }
         }
         if (!ok) {  // exact codes where the fast one may differ
@@ -891,9 +900,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           for (int j = 0; j < 16; ++j) {
             const float xv = __fmul_rn(__uint_as_float(hb[j] << 16), g_ci);
             const float rn = g_s[C::BN + j0 + j];
-            const float t = __fmul_rn(xv, rn);
+            const float t = clamp_nan(__fmul_rn(xv, rn), kq);
             const float d = __fsub_rn(t, __fsub_rn(__fadd_rn(t, kRoundMagic), kRoundMagic));
-            if (!(fabsf(d) < 0.5f - 0x1p-12f || fabsf(t) >= kq + 1.0f))
+            if (!(fabsf(d) < 0.5f - 0x1p-12f))
               code[j] = code_exact_next<C::QMAX_NEXT>(xv, g_s[j0 + j], rn);
           }
         }

@@ -148,11 +148,29 @@ __device__ __forceinline__ void scale8(const uint4 raw, const float (&ci)[8], fl
   }
 }
 
+// x' = x * cinv for one chunk of 8 channels as four value pairs (packed fp32x2
+// multiplies: the same IEEE products as scale8).
+__device__ __forceinline__ void scale8_pairs(const uint4 raw, const float* cinv_s, int c,
+                                             float2 (&v)[4]) {
+  const float4 a = reinterpret_cast<const float4*>(cinv_s)[2 * c];
+  const float4 b = reinterpret_cast<const float4*>(cinv_s)[2 * c + 1];
+  const float2 ci[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w), make_float2(b.x, b.y),
+                        make_float2(b.z, b.w)};
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) v[e] = __fmul2_rn(make_float2(bf16lo(w[e]), bf16hi(w[e])), ci[e]);
+}
+
+template <int QMAX, int GW>
+__device__ __forceinline__ uint2 codes_packed(const float2 (&v)[GW / 2], float s, float r,
+                                              bool narrow);
+
 // Persistent CTAs; each pass handles RPC token rows, one row per TPR threads.
 // cinv is copied to shared memory once per CTA.  Each thread loads its CPT
 // chunks of 8 channels (128-bit loads, all issued before any use, so x is read
 // from HBM once with CPT loads in flight per thread), then forms x * cinv twice:
-// once for the row maximum and once for the codes, which keeps register use low.
+// once for the row maximum and once for the codes, which keeps register use low;
+// both in packed fp32x2 arithmetic, the codes two at a time (codes_packed).
 // STORE_BITS: 8 writes one code per int8 byte (the int4 codes too, for the fused
 // linear's workspace), 4 packs two int4 codes per byte (low nibble = even k).
 // STATIC: the clip comes from the layer-step table alone (§4.3 read as a shared
@@ -207,11 +225,10 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
       for (int i = 0; i < CPT; ++i) {
         const int c = t + i * TPR;
         if (c < nchunk) {
-          float ci[8], v[8];
-          load_cinv8(cinv_s, c, ci);
-          scale8(raw[i], ci, v);
+          float2 v[4];
+          scale8_pairs(raw[i], cinv_s, c, v);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+          for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fmaxf(fabsf(v[e].x), fabsf(v[e].y)));
         }
       }
       amax = warp_max(amax);
@@ -247,23 +264,37 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
     for (int i = 0; i < CPT; ++i) {
       const int c = t + i * TPR;
       if (c >= nchunk) continue;
-      float ci[8], v[8];
-      load_cinv8(cinv_s, c, ci);
-      scale8(raw[i], ci, v);
-      uint32_t q[8];  // low byte of each: the code
+      float2 v[4];
+      scale8_pairs(raw[i], cinv_s, c, v);
+      uint2 cw;  // the 8 codes, one per byte
       if (fast) {
-        quantize8_recip<QMAX>(v, s, r, q);
-      } else {
+        // codes_packed's 16-bit clamp needs |x'| / s < 2^15: the row maximum bounds
+        // it (dynamic clipping), else this chunk's own maximum
+        float cmax = amax;
+        if constexpr (STATIC) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) q[e] = static_cast<uint32_t>(quantize<QMAX>(v[e], s));
+          for (int e = 0; e < 4; ++e) cmax = fmaxf(cmax, fmaxf(fabsf(v[e].x), fabsf(v[e].y)));
+        }
+        cw = codes_packed<QMAX, 8>(v, s, r, cmax <= 16384.0f * s);
+      } else {
+        uint32_t q[8];  // low byte of each: the code
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          q[2 * e] = static_cast<uint32_t>(quantize<QMAX>(v[e].x, s));
+          q[2 * e + 1] = static_cast<uint32_t>(quantize<QMAX>(v[e].y, s));
+        }
+        cw = make_uint2(pack_low_bytes(q[0], q[1], q[2], q[3]),
+                        pack_low_bytes(q[4], q[5], q[6], q[7]));
       }
       if constexpr (STORE_BITS == 8) {
-        const uint2 o = make_uint2(pack_low_bytes(q[0], q[1], q[2], q[3]),
-                                   pack_low_bytes(q[4], q[5], q[6], q[7]));
-        reinterpret_cast<uint2*>(static_cast<int8_t*>(qx) + (size_t)row * K)[c] = o;
+        reinterpret_cast<uint2*>(static_cast<int8_t*>(qx) + (size_t)row * K)[c] = cw;
       } else {
+        // nibbles: bytes 0 and 2 of n hold (c0 | c1 << 4) and (c2 | c3 << 4)
+        uint32_t n0 = cw.x & 0x0F0F0F0Fu, n1 = cw.y & 0x0F0F0F0Fu;
+        n0 |= n0 >> 4;
+        n1 |= n1 >> 4;
         reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(qx) + (size_t)row * (K / 2))[c] =
-            pack_low_nibbles(q);
+            __byte_perm(n0, n1, 0x6420);
       }
     }
   }

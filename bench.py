@@ -41,7 +41,8 @@ from activation_quantized_gemm_wq_b200 import synth as S  # noqa: E402
 METRIC = "fused W4A8/W4A4 linear TOPS (and GB/s at small M) vs roofline; vs oracle"
 DATA = "synthetic (seeded; stream-structured token rows, outlier channels)"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
-FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_BF16_TFLOPS = 1590.0            # burst: a kernel timed alone
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0  # a seconds-long loop under the 1000 W power cap
 FALLBACK_HBM_GBS = 6650.0
 INT8_PER_BF16 = 2.0  # nominal dense ratio (4.5 POPS int8 / 2.25 PFLOP/s bf16)
 L2_BYTES = 126 * 2 ** 20
@@ -124,7 +125,7 @@ def peaks():
         return d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), d["hbm_gbs"], \
             "measured"
     except (OSError, KeyError, ValueError):
-        return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, FALLBACK_HBM_GBS, "fallback"
+        return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS_SUSTAINED, FALLBACK_HBM_GBS, "fallback"
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -400,7 +401,11 @@ def measure_workload(args, wl, wq, torch, world, local, dev):
     e2e = run_e2e(args, layers, wq, torch, world)
 
     bf16_burst, bf16_sust, hbm, src = peaks()
-    peak = bf16_burst * INT8_PER_BF16
+    # The GEMM is timed inside the whole run (every step's launches, back to back for
+    # about a second at the default step count), i.e. under the power cap: its roof is
+    # the sustained figure; the burst one is reported beside it.
+    peak = bf16_sust * INT8_PER_BF16
+    peak_burst = bf16_burst * INT8_PER_BF16
     gemm_launches = args.steps * len(layers)
     achieved = ops_step * args.steps / (gemm_ms * 1e-3) / 1e12
     ms_step = t_max / args.steps
@@ -416,8 +421,11 @@ def measure_workload(args, wl, wq, torch, world, local, dev):
             "frac": round(achieved / peak, 4),
             "traffic": gemm_traffic(wl.name),
             "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
-            "peak_source": f"{src} bf16 burst {bf16_burst} TFLOP/s x{INT8_PER_BF16} (dense int8 "
-                           "/ bf16 nominal ratio); units are int8 tera-ops",
+            "peak_source": f"{src} bf16 sustained {bf16_sust} TFLOP/s x{INT8_PER_BF16} (dense "
+                           "int8 / bf16 nominal ratio; the GEMM is timed inside the whole "
+                           "power-capped run); units are int8 tera-ops",
+            "frac_of_burst": round(achieved / peak_burst, 4),
+            "peak_burst": round(peak_burst, 1),
             "frac_of_nominal_int8": round(achieved / NOMINAL_INT8_TOPS, 4),
             "gemm_avg_launch_ms": round(gemm_ms / gemm_launches, 5),
             "gemm_share_of_step": round(sum(per_layer_ms) / ms_step, 4),
