@@ -474,9 +474,8 @@ struct Ring {
   static constexpr int K = NT * C;
   static constexpr int R = kRingElemsPerThread / C;       // rows per round
   static constexpr int ROUND_BYTES = R * K * 2;
-  static constexpr int OFF_AMAX = kRingSlots * ROUND_BYTES;  // uint32 [2][R]
-  static constexpr int OFF_SCALE = OFF_AMAX + 2 * R * 4;    // float [R] s, then [R] 1/s
-  static constexpr int OFF_BAR = (OFF_SCALE + 2 * R * 4 + 7) / 8 * 8;
+  static constexpr int OFF_AMAX = kRingSlots * ROUND_BYTES;  // uint32 [3][R], rounds mod 3
+  static constexpr int OFF_BAR = (OFF_AMAX + 3 * R * 4 + 7) / 8 * 8;
   static constexpr int SMEM = OFF_BAR + kRingSlots * 8;
   static_assert(R >= 1 && C >= 4 && C % 4 == 0, "C = K / 512 channels per thread");
 };
@@ -597,7 +596,6 @@ __global__ void __launch_bounds__(NT, 512 / NT) act_quant_ring_kernel(
   constexpr int P = C / 2;  // value pairs per row and thread
   extern __shared__ __align__(128) uint8_t ring_smem[];
   uint32_t* amax_s = reinterpret_cast<uint32_t*>(ring_smem + G::OFF_AMAX);
-  float* scale_s = reinterpret_cast<float*>(ring_smem + G::OFF_SCALE);
   uint64_t* full = reinterpret_cast<uint64_t*>(ring_smem + G::OFF_BAR);
   const int t = threadIdx.x;
   const int lane = t & 31;
@@ -606,7 +604,7 @@ __global__ void __launch_bounds__(NT, 512 / NT) act_quant_ring_kernel(
     for (int i = 0; i < kRingSlots; ++i) mbar_init(&full[i], 1);
     fence_mbar_init();
   }
-  if (t < 2 * R) amax_s[t] = 0u;
+  if (t < 3 * R) amax_s[t] = 0u;
   float2 ci[P];
 #pragma unroll
   for (int j = 0; j < NG; ++j) {
@@ -686,19 +684,24 @@ __global__ void __launch_bounds__(NT, 512 / NT) act_quant_ring_kernel(
       constexpr int SH = 5 - log2_of<R>();
       const float wmax = warp_max_multi<R>(pmax, lane);
       if ((lane & ((1 << SH) - 1)) == 0 && wmax > 0.0f)
-        atomicMax(&amax_s[(local & 1) * R + (lane >> SH)], __float_as_uint(wmax));
+        atomicMax(&amax_s[(local % 3) * R + (lane >> SH)], __float_as_uint(wmax));
     }
-    if (t < R) amax_s[((local + 1) & 1) * R + t] = 0u;  // the next round's maxima
+    // the next round's maxima (the round before last, whose readers all passed the
+    // previous barrier, used this third of the buffer)
+    if (t < R) amax_s[((local + 1) % 3) * R + t] = 0u;
     // every thread has read its channels of the slot, and every row maximum is in
     if (__syncthreads_or(!landed)) { ok = false; break; }
     if (t == 0 && issued < kRingSlots + local + 1) {  // refill the slot just read
       issue(local + kRingSlots);
       issued = kRingSlots + local + 1;
     }
-    if (t < rows) {
-      const int row = row0 + t;
-      const float amax = __uint_as_float(amax_s[(local & 1) * R + t]);
-      float sc = 0.0f;
+    // Every warp derives the round's scales itself (lane i takes row i) and passes
+    // them along by shuffles: one CTA barrier per round.  Warp 0 alone writes s_tok
+    // and reports a bad stream id.
+    float sc_l = 0.0f, rs_l = 0.0f;
+    if (lane < rows) {
+      const int row = row0 + lane;
+      const float amax = __uint_as_float(amax_s[(local % 3) * R + lane]);
       const int sid = stream_id[row];
       if (sid < S) {
         float clip;
@@ -708,22 +711,21 @@ __global__ void __launch_bounds__(NT, 512 / NT) act_quant_ring_kernel(
         } else {
           clip = __fmul_rn(__ldg(alpha + step * S + sid), amax);
         }
-        sc = __fdiv_rn(clip, static_cast<float>(QMAX));
-      } else {
+        sc_l = __fdiv_rn(clip, static_cast<float>(QMAX));
+      } else if (t < 32) {
         raise_error(kErrBadStreamId);
       }
-      s_tok[row] = sc;
-      const float rc = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+      if (t < 32) s_tok[row] = sc_l;
+      const float rc = sc_l > 0.0f ? __frcp_rn(sc_l) : 0.0f;
       // negative reciprocal: this row takes the general path (a zero or tiny scale)
-      const bool fast = sc > 0.0f && isfinite(rc);
-      scale_s[t] = sc;
-      scale_s[R + t] = fast ? (amax <= 16384.0f * sc ? rc : -rc) : 0.0f;
+      const bool fast = sc_l > 0.0f && isfinite(rc);
+      rs_l = fast ? (amax <= 16384.0f * sc_l ? rc : -rc) : 0.0f;
     }
-    __syncthreads();
 #pragma unroll
     for (int i = 0; i < R; ++i) {
+      const float sc = __shfl_sync(0xFFFFFFFFu, sc_l, i);
+      const float rs = __shfl_sync(0xFFFFFFFFu, rs_l, i);
       if (i >= rows) break;
-      const float sc = scale_s[i], rs = scale_s[R + i];
       const float rc = fabsf(rs);
       const bool fast = rs != 0.0f;
       const bool narrow = rs > 0.0f;

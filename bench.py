@@ -530,6 +530,8 @@ def run_gpu(args, rank, world, local):
             out["roofline"]["achieved"] / out["int8_mm_probe"]["tops"], 4)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(wl, budget_s=12.0)
+        if "w4a4" in out:  # the oracle on the 4-bit workload too (a smaller sample)
+            out["w4a4"]["cpu_baseline"] = cpu_baseline(S.WORKLOADS[companion], budget_s=6.0)
     return out
 
 
