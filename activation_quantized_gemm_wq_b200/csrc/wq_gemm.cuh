@@ -199,8 +199,15 @@ struct Cfg {
                                                            : -1;
   }
 
+  // ATMEM (the 256-deep stages of narrow token tiles): the unpack warps write the
+  // int8 weight tile into TMEM (tcgen05.st) and the MMA reads its A operand from
+  // there.  Shared memory then carries 2 bytes per packed weight byte (the copy in,
+  // the unpack's read) instead of 6 (also the int8 tile's write and the MMA's read
+  // of it), which bounded these tiles at about 40 GB/s of weights per SM.
+  static constexpr bool ATMEM = KS == 2 && EPI == 0;
+  static constexpr int A_COLS = KS * 32;  // TMEM columns of one int8 weight tile
   static constexpr int WP_BYTES = BM * BK / 2;                               // packed W
-  static constexpr int WU_BYTES = BM * BK;                                   // int8 W
+  static constexpr int WU_BYTES = ATMEM ? 0 : BM * BK;                       // int8 W
   static constexpr int XS_BYTES = ACT_BITS == 8 ? BNX * BK : BNX * BK / 2;   // staged x
   static constexpr int XU_BYTES = ACT_BITS == 8 ? 0 : BNX * BK;             // int8 x (A4)
   // one 128-deep sub-block of an int8 operand tile: [rows][128 B], 128-byte swizzle
@@ -212,7 +219,7 @@ struct Cfg {
   // Pipeline: NS TMA stages (packed weights + activation tile), NU unpacked
   // buffers, and one "MMA done with K block g" barrier per stage (a ring of NS).
   // Each MMA-issuing thread does one wait and one commit per K block of its own.
-  static constexpr int NU_BASE = ACT_BITS == 8 && KS == 1 ? 3 : 2;
+  static constexpr int NU_BASE = (ACT_BITS == 8 && KS == 1) || ATMEM ? 3 : 2;
   static constexpr int NU = MMA_WARPS > NU_BASE ? MMA_WARPS : NU_BASE;
   static constexpr int EPI_ELEM = 2;  // bf16 y (the codes of EPI > 0 use half of it)
   // The tensor cores accumulate 16x (int8 activations) or 256x (both operands
@@ -260,12 +267,16 @@ struct Cfg {
 
   // two tile buffers x MMA_WARPS partial accumulators of BN columns
   static constexpr int ACC_COLS = 2 * MMA_WARPS * BN;
-  static_assert(ACC_COLS <= 512, "TMEM holds 512 columns");
-  static constexpr uint32_t TMEM_COLS = ACC_COLS <= 32    ? 32
-                                        : ACC_COLS <= 64  ? 64
-                                        : ACC_COLS <= 128 ? 128
-                                        : ACC_COLS <= 256 ? 256
-                                                          : 512;
+  // ATMEM: NU int8 weight tiles after the accumulators
+  static constexpr int A_COL0 = ACC_COLS;
+  static constexpr int USED_COLS = ACC_COLS + (ATMEM ? NU * A_COLS : 0);
+  static_assert(USED_COLS <= 512, "TMEM holds 512 columns");
+  static constexpr uint32_t TMEM_COLS = USED_COLS <= 32    ? 32
+                                        : USED_COLS <= 64  ? 64
+                                        : USED_COLS <= 128 ? 128
+                                        : USED_COLS <= 256 ? 256
+                                                           : 512;
+  static_assert(!ATMEM || UNPACK_WARPS % 4 == 0, "unpack warps cover the lane quadrants");
 };
 
 __device__ __forceinline__ void decode_tile(const TileArgs& a, int tile, int& n_tile,
@@ -507,13 +518,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
               C::ACT_BITS == 8 ? smem_u32(smem + C::OFF_XS + s * C::XS_BYTES)
                                : smem_u32(smem + C::OFF_XU + u * C::XU_BYTES);
           const uint32_t a_addr = smem_u32(smem + C::OFF_WU + u * C::WU_BYTES);
+          // ATMEM: the int8 weight tile u in TMEM, 8 columns per 32-deep MMA
+          const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(C::A_COL0 + u * C::A_COLS);
 #pragma unroll
           for (int kk = 0; kk < C::BK / 32; ++kk) {  // sub-block kk / 4, 32 deep each
-            const uint64_t ad = smem_desc_sw128(a_addr + (kk >> 2) * C::SUB_W + (kk & 3) * 32);
             const uint64_t bd = smem_desc_sw128(b_addr + (kk >> 2) * C::SUB_X + (kk & 3) * 32);
             const uint32_t acc = (kb - kb0 >= C::MMA_WARPS || kk != 0) ? 1u : 0u;
-            if constexpr (C::PAIR) mma_i8_ss_pair(d_tmem, ad, bd, idesc, acc);
-            else mma_i8_ss(d_tmem, ad, bd, idesc, acc);
+            if constexpr (C::ATMEM) {
+              mma_i8_ts(d_tmem, a_tmem + static_cast<uint32_t>(kk * 8), bd, idesc, acc);
+            } else {
+              const uint64_t ad =
+                  smem_desc_sw128(a_addr + (kk >> 2) * C::SUB_W + (kk & 3) * 32);
+              if constexpr (C::PAIR) mma_i8_ss_pair(d_tmem, ad, bd, idesc, acc);
+              else mma_i8_ss(d_tmem, ad, bd, idesc, acc);
+            }
           }
           if constexpr (C::PAIR) mma_commit_pair(&done[s], 3);  // both CTAs' stage s
           else mma_commit(&done[s]);
@@ -556,8 +574,45 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         // int8 activations arrive in k order, so the weights must too; int4
         // activations are unpacked exactly like the weights, so both may keep
         // the cheaper permuted order.
-        unpack_tile<C::BM, NT, C::ACT_BITS == 8, C::KS>(smem + C::OFF_WP + s * C::WP_BYTES,
-                                                        smem + C::OFF_WU + u * C::WU_BYTES, tid);
+        if constexpr (C::ATMEM) {
+          // Weight row r = 32q + lane of the tile, q = warp % 4 (the TMEM lane quadrant
+          // this warp reaches); with 8 unpack warps two share a quadrant, each taking
+          // half of the row's 16-byte packed chunks.  Chunk p (128-byte swizzle) holds
+          // k = 32p .. 32p + 31: columns 8p .. 8p + 7 of the tile in TMEM.
+          constexpr int PER_Q = C::UNPACK_WARPS / 4;
+          constexpr int CH = 4 * C::KS / PER_Q;
+          static_assert(CH % 2 == 0, "16-column TMEM stores");
+          tc_fence_after();  // the MMA that read this tile before has completed
+          const int q = warp & 3, part = C::unpack_index(warp) / 4;
+          const int r = q * 32 + lane;
+          const uint8_t* src = smem + C::OFF_WP + s * C::WP_BYTES + r * (C::BK / 2);
+          uint4 v[CH];
+#pragma unroll
+          for (int i = 0; i < CH; ++i) {
+            const int p = part * CH + i;
+            v[i] = *reinterpret_cast<const uint4*>(src + ((p ^ (r & 7)) << 4));
+          }
+          const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                              static_cast<uint32_t>(C::A_COL0 + u * C::A_COLS + part * CH * 8);
+#pragma unroll
+          for (int i = 0; i < CH; i += 2) {
+            uint32_t w[16];
+            uint4 lo, hi;
+            unpack32<C::ACT_BITS == 8>(v[i], lo, hi);
+            w[0] = lo.x; w[1] = lo.y; w[2] = lo.z; w[3] = lo.w;
+            w[4] = hi.x; w[5] = hi.y; w[6] = hi.z; w[7] = hi.w;
+            unpack32<C::ACT_BITS == 8>(v[i + 1], lo, hi);
+            w[8] = lo.x; w[9] = lo.y; w[10] = lo.z; w[11] = lo.w;
+            w[12] = hi.x; w[13] = hi.y; w[14] = hi.z; w[15] = hi.w;
+            tmem_st_32x32b_x16(ta + static_cast<uint32_t>(i * 8), w);
+          }
+          tmem_wait_st();
+          tc_fence_before();  // the stores, before the arrival the MMA waits for
+        } else {
+          unpack_tile<C::BM, NT, C::ACT_BITS == 8, C::KS>(smem + C::OFF_WP + s * C::WP_BYTES,
+                                                          smem + C::OFF_WU + u * C::WU_BYTES,
+                                                          tid);
+        }
         if constexpr (C::ACT_BITS == 4) {
           unpack_tile<C::BNX, NT, false, C::KS>(smem + C::OFF_XS + s * C::XS_BYTES,
                                                 smem + C::OFF_XU + u * C::XU_BYTES, tid);
