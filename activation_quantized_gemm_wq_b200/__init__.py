@@ -36,6 +36,9 @@ _SIGS = {
     "wq_pack_int4": (_I, [_P, _P, _I, _I, _P, _P, _P]),
     "wq_act_quant": (_I, [_P, _I, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "wq_gemm_w4ax": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "wq_gemm_scratch_bytes": (ctypes.c_size_t, [_I, _I, _I]),
+    "wq_gemm_w4ax_ws": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P,
+                             ctypes.c_size_t, _P]),
     "wq_linear_w4a8": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P,
                             ctypes.c_size_t, _P]),
     "wq_linear_w4a4": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P,
@@ -216,6 +219,24 @@ def wq_gemm_w4ax(qx, s_tok, act_bits, K, stream_id, beta, S, T, step, qw, s_w, b
           _ptr(stream_id, "stream_id", _BYTES, M), _ptr(beta, "beta", _F32, T * S * N), S, T,
           step, _ptr(qw, "qw", _BYTES, N * (K // 2)), _ptr(s_w, "s_w", _F32, N),
           _ptr(bias, "bias", _F32, N), _ptr(y, "y", _BF16, M * N), _stream(stream))
+
+
+def wq_gemm_scratch_bytes(M, K, N):
+    return int(lib().wq_gemm_scratch_bytes(M, K, N))
+
+
+def wq_gemm_w4ax_ws(qx, s_tok, act_bits, K, stream_id, beta, S, T, step, qw, s_w, bias, y,
+                    workspace=None, stream=None):
+    """wq_gemm_w4ax splitting K over every SM for few tokens, through `workspace`
+    (at least wq_gemm_scratch_bytes(M, K, N) bytes; None when that is 0)."""
+    M, N = y.shape
+    _call("wq_gemm_w4ax_ws", _ptr(qx, "qx", _BYTES, M * _codes_per_row(K, act_bits)),
+          _ptr(s_tok, "s_tok", _F32, M), act_bits, M, K, N,
+          _ptr(stream_id, "stream_id", _BYTES, M), _ptr(beta, "beta", _F32, T * S * N), S, T,
+          step, _ptr(qw, "qw", _BYTES, N * (K // 2)), _ptr(s_w, "s_w", _F32, N),
+          _ptr(bias, "bias", _F32, N), _ptr(y, "y", _BF16, M * N),
+          _ptr(workspace, "workspace"), 0 if workspace is None else _nbytes(workspace),
+          _stream(stream))
 
 
 def _linear(name, x, cinv, stream_id, alpha, beta, step, qw, s_w, bias, y, workspace, stream):

@@ -307,6 +307,36 @@ wq_status wq_gemm_w4ax(const void* qx, const float* s_tok, int act_bits, int M, 
                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t wq_gemm_scratch_bytes(int M, int K, int N) {
+  if (check_mk(M, K) != WQ_OK || check_n(N) != WQ_OK || M == 0) return 0;
+  return wq::gemm_split_scratch_bytes(M, N, K);
+}
+
+wq_status wq_gemm_w4ax_ws(const void* qx, const float* s_tok, int act_bits, int M, int K, int N,
+                          const uint8_t* stream_id, const float* beta, int S, int T, int step,
+                          const uint8_t* qw, const float* s_w, const float* bias, wq_bf16* y,
+                          void* workspace, size_t ws_bytes, wq_stream_t stream) {
+  WQ_TRY(gemm_checks(qx, s_tok, act_bits, M, K, N, stream_id, beta, S, T, step, qw, s_w, bias,
+                     y));
+  const wq::EpilogueArgs ep{s_tok, stream_id, s_w, bias, beta, S, step};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t split_bytes = M > 0 ? wq::gemm_split_scratch_bytes(M, N, K) : 0;
+  wq::SplitScratch sc{nullptr, nullptr};
+  if (split_bytes > 0) {
+    if (!workspace) return WQ_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return WQ_ERR_ALIGN;
+    if (ws_bytes < split_bytes) return WQ_ERR_ARG;
+    const int BN = wq::bn_for(M);
+    const size_t tiles = static_cast<size_t>((M + BN - 1) / BN) * ((N + 127) / 128);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    sc.partial = reinterpret_cast<int32_t*>(ws);
+    sc.counters = reinterpret_cast<int*>(ws + round_up(tiles * BN * 128 * sizeof(int32_t)));
+    WQ_TRY(from_cuda(cudaMemsetAsync(workspace, 0, split_bytes, st)));
+  }
+  return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, y,
+                                   split_bytes > 0 ? &sc : nullptr, st));
+}
+
 wq_status wq_linear_w4a8(const wq_bf16* x, int M, int K, int N, const float* cinv,
                          const uint8_t* stream_id, const float* alpha, const float* beta,
                          int S, int T, int step, const uint8_t* qw, const float* s_w,

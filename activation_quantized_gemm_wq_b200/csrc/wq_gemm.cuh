@@ -1293,6 +1293,11 @@ int gemm_splits(int M, int N, int K) {
   const int tiles = ((M + BN - 1) / BN) * ((N + 127) / 128);
   const int num_k = K / 128;
   if (tiles * 2 > kSplitTargetCtas) return 1;
+  // Splitting pays only when each tile's K loop is long: measured at 16-256 tokens,
+  // K = 2048 ran faster unsplit (the partial sums, their reduction and the lost CTA
+  // pairs of 256-token tiles outweigh the extra SMs), K = 4096 about even (split
+  // kept for the narrow tiles), K >= 8192 up to twice as fast split.
+  if (num_k < 32 || (num_k < 64 && BN > 64)) return 1;
   int s = kSplitTargetCtas / tiles;
   const int cap = num_k / 2 > 1 ? num_k / 2 : 1;  // at least two K blocks per split
   s = s < cap ? s : cap;

@@ -920,8 +920,12 @@ def sweep(args):
             for r in range(ncopy):
                 wq.wq_act_quant(xs[r], cinv, sid, alpha, step, bits, qxs[r], s_tok)
             calls = max(100 if M <= 256 else 10, ncopy)  # small M: at least 100 calls
-            g_fns = [lambda r=r: wq.wq_gemm_w4ax(qxs[r % ncopy], s_tok, bits, K, sid, beta, 3, T,
-                                                 step, qws[r % ncopy], s_w, bias, y)
+            # the GEMM-only call with its split-K scratch (few tokens split K over
+            # every SM, as inside the fused linear; the scratch is cleared per call)
+            n_scr = wq.wq_gemm_scratch_bytes(M, K, N)
+            gws = torch.empty(n_scr, dtype=torch.uint8, device="cuda") if n_scr else None
+            g_fns = [lambda r=r: wq.wq_gemm_w4ax_ws(qxs[r % ncopy], s_tok, bits, K, sid, beta, 3,
+                                                    T, step, qws[r % ncopy], s_w, bias, y, gws)
                      for r in range(calls)]
             l_fns = [lambda r=r: lin_fn(xs[r % ncopy], cinv, sid, alpha, beta, step,
                                         qws[r % ncopy], s_w, bias, y, ws) for r in range(calls)]
@@ -971,7 +975,7 @@ def sweep(args):
 def ffn(args):
     """The FFN pair of each block (up-projection, GELU, down-projection), W4A8, full
     token batch: the up-projection quantizing for the down-projection in its epilogue
-    (wq_linear_gelu_quant, then wq_gemm_w4ax on its codes), against the same steps
+    (wq_linear_gelu_quant, then wq_gemm_w4ax_ws on its codes), against the same steps
     unfused: wq_linear_w4a8 for the up-projection, GELU on its bf16 output as a
     separate kernel (torch's exact-erf GELU, a library kernel standing in for any
     elementwise pass), then the static-clipping linear reading the GELU output.  One
@@ -1001,8 +1005,8 @@ def ffn(args):
             wq.wq_linear_gelu_quant(up.x[r], up.cinv, up.sid, up.alpha, up.beta, 0, 8, up.qw,
                                     up.s_w, up.bias, down.cinv, thr, gain, 8, codes, s_next, None,
                                     up.ws)
-            wq.wq_gemm_w4ax(codes, s_next, 8, Kh, down.sid, down.beta, down.S, down.T, 0, down.qw,
-                            down.s_w, down.bias, down.y)
+            wq.wq_gemm_w4ax_ws(codes, s_next, 8, Kh, down.sid, down.beta, down.S, down.T, 0,
+                               down.qw, down.s_w, down.bias, down.y, ws_static)
 
         def unfused(r):
             wq.wq_linear_w4a8(up.x[r], up.cinv, up.sid, up.alpha, up.beta, 0, up.qw, up.s_w,

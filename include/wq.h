@@ -125,6 +125,23 @@ wq_status wq_gemm_w4ax(const void* qx, const float* s_tok, int act_bits, int M, 
                        const uint8_t* qw, const float* s_w, const float* bias, wq_bf16* y,
                        wq_stream_t stream);
 
+/* Bytes of scratch wq_gemm_w4ax_ws uses to split K across SMs for (M, K, N): the
+ * int32 partial tiles and their arrival counters, 0 when the shape does not split
+ * (enough output tiles to fill the GPU).  0 for invalid sizes too. */
+size_t wq_gemm_scratch_bytes(int M, int K, int N);
+
+/* wq_gemm_w4ax with a caller workspace (device memory, 256-byte aligned, at least
+ * wq_gemm_scratch_bytes(M, K, N) bytes; may be NULL when that is 0) through which
+ * few-token shapes split K over every SM, as the fused linear does.  The call
+ * clears the scratch on `stream` (one memset) before the GEMM; the int32 sums of
+ * the splits are exact, so y is bit-identical to wq_gemm_w4ax's.  Returns
+ * WQ_ERR_NULL / WQ_ERR_ALIGN / WQ_ERR_ARG for a missing, misaligned or short
+ * workspace; other arguments as in wq_gemm_w4ax. */
+wq_status wq_gemm_w4ax_ws(const void* qx, const float* s_tok, int act_bits, int M, int K, int N,
+                          const uint8_t* stream_id, const float* beta, int S, int T, int step,
+                          const uint8_t* qw, const float* s_w, const float* bias, wq_bf16* y,
+                          void* workspace, size_t ws_bytes, wq_stream_t stream);
+
 /* The fused W4A8 linear: wq_act_quant (8-bit) then wq_gemm_w4ax, with the codes
  * and token scales kept in the caller's workspace (device memory of at least
  * wq_workspace_bytes(M, K, N, 8) bytes, 256-byte aligned; its contents are

@@ -130,6 +130,19 @@ def gpu_gemm_w4ax(qx, s_tok, bits, K, sid, beta, step, qw, s_w, bias):
     return host(y.view(torch.int16), np.uint16)
 
 
+def gpu_gemm_w4ax_ws(qx, s_tok, bits, K, sid, beta, step, qw, s_w, bias):
+    """wq_gemm_w4ax_ws: the GEMM-only call splitting K through a workspace.  The
+    workspace is filled with garbage first: the call must clear what it uses."""
+    M, N = qx.shape[0], qw.shape[0]
+    T, S_, _ = beta.shape
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    n = wq.wq_gemm_scratch_bytes(M, K, N)
+    ws = torch.full((max(n, 256),), 0xA5, dtype=torch.uint8, device="cuda") if n else None
+    wq.wq_gemm_w4ax_ws(dev(qx), dev(s_tok), bits, K, dev(sid), dev(beta), S_, T, step, dev(qw),
+                       dev(s_w), None if bias is None else dev(bias), y, ws)
+    return host(y.view(torch.int16), np.uint16), n
+
+
 def gpu_act_quant_static(x, cinv, sid, thr, gain, step, bits):
     M, K = x.shape
     qx = torch.empty((M, K) if bits == 8 else (M, K // 2),

@@ -92,6 +92,25 @@ def test_other_entry_points_reject_on_host(lib):
     assert lib.wq_channel_scale(None, 4, FAKE, 4, 128, FAKE, FAKE, None) == 1
 
 
+def test_gemm_ws_scratch_rule_on_host(lib):
+    """wq_gemm_w4ax_ws: the scratch is needed exactly when K is split (few tokens,
+    few output tiles); a missing, misaligned or short one is refused before any
+    launch, and a shape that does not split needs none."""
+    lib.wq_gemm_scratch_bytes.restype = ctypes.c_size_t
+    n = lib.wq_gemm_scratch_bytes(16, 4096, 128)
+    assert n > 0
+    assert lib.wq_gemm_scratch_bytes(8512, 4096, 16384) == 0
+    assert lib.wq_gemm_scratch_bytes(16, 100, 128) == 0  # invalid K
+    args = [FAKE, FAKE, 8, 16, 4096, 128, FAKE, None, 3, 1, 0, FAKE, FAKE, None, FAKE]
+    ws = ctypes.c_size_t
+    assert lib.wq_gemm_w4ax_ws(*args, None, ws(0), None) == 1
+    assert lib.wq_gemm_w4ax_ws(*args, FAKE + 16, ws(n), None) == 3
+    assert lib.wq_gemm_w4ax_ws(*args, FAKE, ws(n - 1), None) == 4
+    # the usual checks first: a bad act_bits is refused whatever the workspace
+    bad = list(args); bad[2] = 5
+    assert lib.wq_gemm_w4ax_ws(*bad, FAKE, ws(n), None) == 4
+
+
 def test_static_clipping_entry_points_reject_on_host(lib):
     # wq_act_quant_static(x, M, K, cinv, sid, thr, gain, S, T, step, bits, qx, s_tok, st)
     assert lib.wq_act_quant_static(FAKE, 8, 256, None, FAKE, None, FAKE, 3, 1, 0, 8, FAKE, FAKE,

@@ -15,8 +15,9 @@ import activation_quantized_gemm_wq_b200 as wq
 from activation_quantized_gemm_wq_b200 import synth as S
 
 import oracle_pins as P
-from gpu_util import (dev, gpu_act_quant, gpu_gemm_s32, gpu_gemm_w4ax, gpu_linear,
-                      gpu_linear_debug, gpu_prep, host, unpack_codes, within_tolerance)
+from gpu_util import (dev, gpu_act_quant, gpu_gemm_s32, gpu_gemm_w4ax, gpu_gemm_w4ax_ws,
+                      gpu_linear, gpu_linear_debug, gpu_prep, host, unpack_codes,
+                      within_tolerance)
 
 pytestmark = pytest.mark.gpu
 
@@ -104,10 +105,12 @@ def test_act_quant_near_ties(oracle, bits, qmax):
 
 # ------------------------------------------------------------------ int32 core
 
-# the last four split K over several CTAs (few output tiles), as the fused linear does
+# the next four split K over several CTAs (few output tiles, long K), as the fused
+# linear does: 16-, 64-, 128- and 256-token tiles
 GEMM_SHAPES = [(1, 16, 128), (16, 144, 256), (17, 128, 512), (64, 256, 256), (100, 272, 384),
                (128, 128, 128), (129, 400, 256), (300, 384, 512), (513, 128, 1024),
-               (16, 128, 4096), (40, 512, 2048), (100, 1024, 1024), (256, 2048, 2048),
+               (16, 128, 4096), (40, 512, 8192), (100, 384, 8192), (256, 512, 8192),
+               (256, 2048, 2048),
                # K % 256 == 128 at narrow token tiles: 128-deep stages over 2-4 issuers
                (33, 256, 384), (48, 192, 1152)]
 
@@ -295,6 +298,34 @@ def test_gemm_w4ax_against_oracle(oracle, M, K, N, bits):
     ok, worst = within_tolerance(y[rows], y_ref)
     assert ok, worst
 
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("M,K,N", [(16, 4096, 512), (40, 8192, 256), (64, 4096, 384),
+                                   (1, 256, 16), (300, 8192, 384)])
+def test_gemm_w4ax_ws_split_matches(oracle, M, K, N, bits):
+    """wq_gemm_w4ax_ws: few tokens split K over every SM through the workspace (a
+    garbage-filled one: the call clears it); y bit-identical to wq_gemm_w4ax (int32
+    sums are exact in any order) and within tolerance of the oracle.  300 tokens at
+    K = 8192 split on single-CTA 256-token tiles; one token with K = 256 does not split
+    (no workspace needed)."""
+    rows_ = ((0, M - M // 4 - M // 8), (1, M // 8), (2, M // 4))
+    wl = S.custom(f"gemmws{M}x{K}x{N}", K, N, tuple(r for r in rows_ if r[1] > 0),
+                  act_bits=bits, T=3)
+    L = S.layer_inputs(wl, 0)
+    x = S.activations(wl, 0, step=1)
+    sid = S.stream_ids(wl)
+    c, cinv = oracle.channel_scale(L.x_cal, L.W)
+    qw, s_w = oracle.pack_int4(L.W, c)
+    qx, s_tok = oracle.act_quant(x, cinv, sid, L.alpha, 1, bits)
+    y_ws, nbytes = gpu_gemm_w4ax_ws(qx, s_tok, bits, K, sid, L.beta, 1, qw, s_w, L.bias)
+    assert (nbytes > 0) == (M != 1)  # the 1-token shape (K = 256) does not split
+    y = gpu_gemm_w4ax(qx, s_tok, bits, K, sid, L.beta, 1, qw, s_w, L.bias)
+    assert np.array_equal(y_ws, y)
+    acc = oracle.gemm_s32(qx, bits, qw, K)
+    y_ref = oracle.epilogue(acc, s_tok, s_w, L.bias, L.beta, sid, 1)
+    ok, worst = within_tolerance(y_ws, y_ref)
+    assert ok, worst
 
 
 @pytest.mark.parametrize("M", [16, 256])
