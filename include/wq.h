@@ -242,8 +242,9 @@ wq_status wq_debug_linear_s32(const wq_bf16* x, int M, int K, int N, const float
  *             widths; 0 when s_next[m] is 0.
  * Dynamic clipping needs the maximum over the whole row before any code, which
  * spans every output tile, so only static clipping can be fused here.
- * The down-projection then runs wq_gemm_w4ax(codes_next, s_next, 8, ...) (int8
- * operands for both widths; the int32 sums are the same).
+ * The down-projection then runs wq_gemm_w4ax(codes_next, s_next, 8, ...), or
+ * wq_gemm_w4ax_ws for few tokens (int8 operands for both widths; the int32 sums
+ * are the same).
  *   cinv_next [N] fp32 or NULL (= 1); thr_next [T]; gain_next [T][S];
  *   s_next [M] fp32 out; h [M][N] bf16 out or NULL (a debug copy; not needed).
  * Workspace and other arguments as wq_linear_w4a8.
