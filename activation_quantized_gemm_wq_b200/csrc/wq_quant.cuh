@@ -833,6 +833,13 @@ cudaError_t dispatch_act_quant(const uint16_t* x, int M, int K, const float* cin
 #define WQ_AQ(TPR, CPT) \
   return run_act_quant<ACT_BITS, STORE_BITS, TPR, CPT, STATIC>(x, M, K, cinv, sid, alpha, thr, S, \
                                                                step, qx, s_tok, zero, zero_n16, st)
+  // Few rows (the launch is one pass): a whole CTA per row, so each thread's
+  // share, and the pass's latency, stays small.
+  if (M <= 64) {
+    if (nchunk <= 256) WQ_AQ(256, 1);
+    if (nchunk <= 512) WQ_AQ(256, 2);
+    if (nchunk <= 1024) WQ_AQ(256, 4);
+  }
   // one warp per row up to K = 2048 (no block-level reduction), 8 chunks of 8
   // channels per thread beyond that
   if (nchunk <= 32) WQ_AQ(32, 1);
