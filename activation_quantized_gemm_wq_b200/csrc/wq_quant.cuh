@@ -194,27 +194,6 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
   // prologue (and its weight loads) while this one runs.
   griddep_wait();
   griddep_launch_dependents();
-
-  const int local_row = threadIdx.x / TPR;
-  const int t = threadIdx.x % TPR;
-  const int nchunk = K >> 3;
-  const int groups = (M + RPC - 1) / RPC;
-  // With one pass per CTA (few rows) the row is requested before cinv is staged,
-  // so the two loads' latencies overlap; with many passes the first row's loads
-  // would only compete with the staging (measured 5 % slower at 8512 x 16384).
-  const bool one_pass = groups <= static_cast<int>(gridDim.x);
-  uint4 raw[CPT];
-  auto load_row = [&](int grp) {
-    const int row = grp * RPC + local_row;
-#pragma unroll
-    for (int i = 0; i < CPT; ++i) {
-      const int c = t + i * TPR;
-      raw[i] = (row < M && c < nchunk)
-                   ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)row * K) + c)
-                   : make_uint4(0u, 0u, 0u, 0u);
-    }
-  };
-  if (one_pass && blockIdx.x < groups) load_row(blockIdx.x);
   // Clear the next GEMM's split-K accumulators and counters (16-byte words) here
   // rather than in a separate launch.
   for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < zero_n16; i += (size_t)gridDim.x * 256)
@@ -224,10 +203,22 @@ __global__ void __launch_bounds__(256) act_quant_kernel(
         cinv ? __ldg(reinterpret_cast<const float4*>(cinv + k)) : make_float4(1.f, 1.f, 1.f, 1.f);
   __syncthreads();
 
+  const int local_row = threadIdx.x / TPR;
+  const int t = threadIdx.x % TPR;
+  const int nchunk = K >> 3;
+  const int groups = (M + RPC - 1) / RPC;
+
   for (int grp = blockIdx.x; grp < groups; grp += gridDim.x) {  // CTA-uniform loop
     const int row = grp * RPC + local_row;
     const bool row_ok = row < M;
-    if (!one_pass) load_row(grp);
+    uint4 raw[CPT];
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+      const int c = t + i * TPR;
+      raw[i] = (row_ok && c < nchunk)
+                   ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)row * K) + c)
+                   : make_uint4(0u, 0u, 0u, 0u);
+    }
     float amax = 0.0f;
     if constexpr (!STATIC) {
 #pragma unroll
