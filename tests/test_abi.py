@@ -111,6 +111,19 @@ def test_gemm_ws_scratch_rule_on_host(lib):
     assert lib.wq_gemm_w4ax_ws(*bad, FAKE, ws(n), None) == 4
 
 
+@pytest.mark.parametrize("M,K,N,splits", [
+    (16, 2048, 512, False),    # short K loop: unsplit
+    (16, 4096, 512, True),     # narrow tiles from K = 4096 on
+    (128, 4096, 512, False),   # wider tiles split only from K = 8192 on
+    (256, 8192, 2048, True),
+    (4288, 8192, 2048, False),  # enough output tiles to fill the GPU
+    (16, 16384, 4096, True)])
+def test_split_rule_on_host(lib, M, K, N, splits):
+    """K is split (scratch needed) only for few output tiles with a long K loop."""
+    lib.wq_gemm_scratch_bytes.restype = ctypes.c_size_t
+    assert (lib.wq_gemm_scratch_bytes(M, K, N) > 0) == splits
+
+
 def test_static_clipping_entry_points_reject_on_host(lib):
     # wq_act_quant_static(x, M, K, cinv, sid, thr, gain, S, T, step, bits, qx, s_tok, st)
     assert lib.wq_act_quant_static(FAKE, 8, 256, None, FAKE, None, FAKE, 3, 1, 0, 8, FAKE, FAKE,
