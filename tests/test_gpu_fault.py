@@ -28,8 +28,9 @@ def _device():
     assert wq.wq_device_status() == ("WQ_OK", 0)
 
 
-# one CTA and one tile; a split of K over two CTAs; many CTAs with several tiles each
-@pytest.mark.parametrize("M,K,N", [(64, 256, 128), (300, 512, 384), (4288, 2048, 2048)])
+# one CTA and one tile; a split of K over many CTAs (few tiles, long K); many CTAs with
+# several tiles each
+@pytest.mark.parametrize("M,K,N", [(64, 256, 128), (300, 8192, 384), (4288, 2048, 2048)])
 def test_stalled_stage_times_out_and_the_context_recovers(oracle, M, K, N):
     rows = ((0, M - M // 4), (2, M // 4))
     wl = S.custom(f"stall{M}x{K}x{N}", K, N, rows, act_bits=8, T=1)

@@ -51,8 +51,8 @@ def _f32bits(a):
 
 @pytest.mark.parametrize("bits_up,bits_next", [(8, 8), (8, 4), (4, 8)])
 @pytest.mark.parametrize("M,K,N,wide", [(300, 512, 384, False), (33, 1024, 256, True),
-                                        (16, 2048, 1024, False), (4288, 2048, 8192, False)],
-                         ids=["300x512x384", "33x1024x256_wide", "16x2048x1024_split",
+                                        (16, 4096, 1024, False), (4288, 2048, 8192, False)],
+                         ids=["300x512x384", "33x1024x256_wide", "16x4096x1024_split",
                               "block2048_mlp_up"])
 def test_gelu_quant_against_oracle(oracle, M, K, N, wide, bits_up, bits_next):
     g = np.random.default_rng(M + K + N + 10 * bits_up + bits_next)
