@@ -136,6 +136,7 @@ __device__ __forceinline__ void split_range(int num_k, int splits, int sp, int& 
 // EPI > 0: the up-projection of an FFN whose epilogue emits the down-projection's
 // activation codes (qmax 127 for EPI 8, 7 for EPI 4) instead of y.
 // PAIR: two CTAs (a cluster) share one tile of 256 output channels x BN tokens
+// (BN = 224 with the weights in TMEM, 256 for the GELU-and-quantize epilogue)
 // through the pair MMA (tcgen05 cta_group::2): each CTA unpacks its own 128
 // weight rows and loads half of the token rows (BN/2), rank 0 issues the MMAs, and
 // each CTA's TMEM receives the accumulators of its own 128 channels for all BN
@@ -160,8 +161,8 @@ struct Cfg {
                 "the single-kernel linear quantizes into the int8 mainloop, one token tile");
   static_assert(EPI == 0 || ((EPI == 8 || EPI == 4) && QBITS == 0 && ACT_BITS == 8),
                 "the GELU-and-quantize epilogue follows the int8-activation mainloop");
-  static_assert(!PAIR || (QBITS == 0 && BN == 256 && ACT_BITS == 8),
-                "CTA pairs serve the 256-token tiles of int8 activation codes");
+  static_assert(!PAIR || (QBITS == 0 && (BN == 256 || BN == 224) && ACT_BITS == 8),
+                "CTA pairs serve the 224- and 256-token tiles of int8 activation codes");
   static constexpr int KS = KS_;
   static_assert(KS == 1 || (KS == 2 && !PAIR && QBITS == 0 && BN <= 64),
                 "256-deep stages serve the narrow token tiles of the two-kernel path");
@@ -199,12 +200,14 @@ struct Cfg {
                                                            : -1;
   }
 
-  // ATMEM (the 256-deep stages of narrow token tiles): the unpack warps write the
-  // int8 weight tile into TMEM (tcgen05.st) and the MMA reads its A operand from
-  // there.  Shared memory then carries 2 bytes per packed weight byte (the copy in,
-  // the unpack's read) instead of 6 (also the int8 tile's write and the MMA's read
-  // of it), which bounded these tiles at about 40 GB/s of weights per SM.
-  static constexpr bool ATMEM = KS == 2 && EPI == 0;
+  // ATMEM (the 256-deep stages of narrow token tiles, and the 224-token CTA pairs):
+  // the unpack warps write the int8 weight tile into TMEM (tcgen05.st) and the MMA
+  // reads its A operand from there.  Shared memory then carries 2 bytes per packed
+  // weight byte (the copy in, the unpack's read) instead of 6 (also the int8 tile's
+  // write and the MMA's read of it), which bounded the narrow tiles at about 40 GB/s
+  // of weights per SM and left the wide tiles' tensor pipe waiting on shared memory.
+  // A pair's TMEM then holds two 224-column accumulators and two weight tiles.
+  static constexpr bool ATMEM = (KS == 2 && EPI == 0) || (PAIR && BN == 224);
   static constexpr int A_COLS = KS * 32;  // TMEM columns of one int8 weight tile
   static constexpr int WP_BYTES = BM * BK / 2;                               // packed W
   static constexpr int WU_BYTES = ATMEM ? 0 : BM * BK;                       // int8 W
@@ -219,7 +222,8 @@ struct Cfg {
   // Pipeline: NS TMA stages (packed weights + activation tile), NU unpacked
   // buffers, and one "MMA done with K block g" barrier per stage (a ring of NS).
   // Each MMA-issuing thread does one wait and one commit per K block of its own.
-  static constexpr int NU_BASE = (ACT_BITS == 8 && KS == 1) || ATMEM ? 3 : 2;
+  // (224-token pairs: two 32-column weight tiles beside 2 x 224 accumulator columns)
+  static constexpr int NU_BASE = PAIR && ATMEM ? 2 : (ACT_BITS == 8 && KS == 1) || ATMEM ? 3 : 2;
   static constexpr int NU = MMA_WARPS > NU_BASE ? MMA_WARPS : NU_BASE;
   static constexpr int EPI_ELEM = 2;  // bf16 y (the codes of EPI > 0 use half of it)
   // The tensor cores accumulate 16x (int8 activations) or 256x (both operands
@@ -524,7 +528,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           for (int kk = 0; kk < C::BK / 32; ++kk) {  // sub-block kk / 4, 32 deep each
             const uint64_t bd = smem_desc_sw128(b_addr + (kk >> 2) * C::SUB_X + (kk & 3) * 32);
             const uint32_t acc = (kb - kb0 >= C::MMA_WARPS || kk != 0) ? 1u : 0u;
-            if constexpr (C::ATMEM) {
+            if constexpr (C::ATMEM && C::PAIR) {
+              mma_i8_ts_pair(d_tmem, a_tmem + static_cast<uint32_t>(kk * 8), bd, idesc, acc);
+            } else if constexpr (C::ATMEM) {
               mma_i8_ts(d_tmem, a_tmem + static_cast<uint32_t>(kk * 8), bd, idesc, acc);
             } else {
               const uint64_t ad =
@@ -590,7 +596,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
           for (int i = 0; i < CH; ++i) {
             const int p = part * CH + i;
-            v[i] = *reinterpret_cast<const uint4*>(src + ((p ^ (r & 7)) << 4));
+            // 64-byte rows: 64-byte swizzle; 128-byte rows: 128-byte swizzle
+            const int sw = C::KS == 1 ? (p ^ ((r >> 1) & 3)) : (p ^ (r & 7));
+            v[i] = *reinterpret_cast<const uint4*>(src + (sw << 4));
           }
           const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                               static_cast<uint32_t>(C::A_COL0 + u * C::A_COLS + part * CH * 8);
@@ -1226,15 +1234,23 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
   return launch_pdl(gemm_kernel<C>, grid, C::THREADS, C::SMEM_BYTES, st, 1, tm_w, tm_x, tm_out, a);
 }
 
-// 256-token tiles go to CTA pairs unless K is split (few tokens, few tiles).
+// More than 128 tokens go to CTA pairs unless K is split (few tiles, long K): tiles
+// of 224 tokens with the weights in TMEM (measured 4 % faster per step than 256-token
+// pairs with the weights in shared memory on the hidden-4096 block), or 256 for the
+// GELU-and-quantize epilogue, whose twelve warps keep the shared-memory design.
 template <int ACT_BITS, int EPI = 0>
 cudaError_t dispatch_bn(const void* qx, const uint8_t* qw, int M, int N, int K,
                         const EpilogueArgs& ep, void* out, const SplitScratch* sc,
                         cudaStream_t st, bool wp, const GemmExtras* ex) {
   if constexpr (ACT_BITS == 8) {
-    if (bn_for(M) == 256 && (sc == nullptr || gemm_splits(M, N, K) == 1))
-      return run_gemm<Cfg<256, 8, 0, EPI, true>>(qx, qw, M, N, K, ep, out, nullptr, st, wp,
+    if (bn_for(M) == 256 && (sc == nullptr || gemm_splits(M, N, K) == 1)) {
+      if constexpr (EPI == 0)
+        return run_gemm<Cfg<224, 8, 0, 0, true>>(qx, qw, M, N, K, ep, out, nullptr, st, wp,
                                                  nullptr, ex);
+      else
+        return run_gemm<Cfg<256, 8, 0, EPI, true>>(qx, qw, M, N, K, ep, out, nullptr, st, wp,
+                                                   nullptr, ex);
+    }
   }
   // narrow token tiles stream 256-deep stages when K allows
   const bool ks2 = K % 256 == 0;
