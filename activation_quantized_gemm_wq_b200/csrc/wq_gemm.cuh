@@ -1132,6 +1132,21 @@ int sm_count() {
 
 int bn_for(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
 
+// Token tile of a CTA pair on the plain epilogue.  224-token tiles (weights in TMEM)
+// run a little faster per token than 256-token tiles, but every pair works through
+// whole tiles, so the busiest pair does ceil(tiles / pairs) x BN token columns per
+// 256 output channels: where 224 leaves it more of them (4288 tokens on 2048 channels:
+// 160 tiles, three per pair, against 136 tiles, two per pair), 256 is taken.
+int pair_bn(int M, int N) {
+  const long long pairs = sm_count() / 2;
+  const long long ch = (N + 255) / 256;
+  const auto busiest = [&](long long bn) {
+    const long long tiles = ch * ((M + bn - 1) / bn);
+    return (tiles + pairs - 1) / pairs * bn;
+  };
+  return busiest(224) <= busiest(256) ? 224 : 256;
+}
+
 // Inputs of the single-kernel linear (Cfg QBITS > 0).
 struct SingleArgs {
   const uint16_t* x;   // bf16 [M][K]
@@ -1236,20 +1251,25 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
 
 // More than 128 tokens go to CTA pairs unless K is split (few tiles, long K): tiles
 // of 224 tokens with the weights in TMEM (measured 4 % faster per step than 256-token
-// pairs with the weights in shared memory on the hidden-4096 block), or 256 for the
-// GELU-and-quantize epilogue, whose twelve warps keep the shared-memory design.
+// pairs with the weights in shared memory on the hidden-4096 block) where pair_bn
+// finds them no worse balanced, else 256; always 256 for the GELU-and-quantize
+// epilogue, whose twelve warps keep the shared-memory design.
 template <int ACT_BITS, int EPI = 0>
 cudaError_t dispatch_bn(const void* qx, const uint8_t* qw, int M, int N, int K,
                         const EpilogueArgs& ep, void* out, const SplitScratch* sc,
                         cudaStream_t st, bool wp, const GemmExtras* ex) {
   if constexpr (ACT_BITS == 8) {
     if (bn_for(M) == 256 && (sc == nullptr || gemm_splits(M, N, K) == 1)) {
-      if constexpr (EPI == 0)
-        return run_gemm<Cfg<224, 8, 0, 0, true>>(qx, qw, M, N, K, ep, out, nullptr, st, wp,
+      if constexpr (EPI == 0) {
+        if (pair_bn(M, N) == 224)
+          return run_gemm<Cfg<224, 8, 0, 0, true>>(qx, qw, M, N, K, ep, out, nullptr, st, wp,
+                                                   nullptr, ex);
+        return run_gemm<Cfg<256, 8, 0, 0, true>>(qx, qw, M, N, K, ep, out, nullptr, st, wp,
                                                  nullptr, ex);
-      else
+      } else {
         return run_gemm<Cfg<256, 8, 0, EPI, true>>(qx, qw, M, N, K, ep, out, nullptr, st, wp,
                                                    nullptr, ex);
+      }
     }
   }
   // narrow token tiles stream 256-deep stages when K allows
