@@ -27,6 +27,16 @@ WQ_OK = 0
 STATUS = {0: "WQ_OK", 1: "WQ_ERR_NULL", 2: "WQ_ERR_SHAPE", 3: "WQ_ERR_ALIGN", 4: "WQ_ERR_ARG",
           5: "WQ_ERR_CUDA", 6: "WQ_ERR_TIMEOUT", 7: "WQ_ERR_DEVICE", 8: "WQ_ERR_SCRATCH"}
 
+
+
+class GemmPlan(ctypes.Structure):
+    """struct wq_gemm_plan of include/wq.h."""
+    _fields_ = [(n, ctypes.c_int) for n in ("tile_tokens", "tile_channels", "ctas_per_tile",
+                                             "k_splits", "k_stage", "tiles", "weights_in_tmem")]
+
+
+PLAN_CALLS = {"gemm": 0, "gemm_ws": 1, "linear": 2, "gelu_quant": 3}
+
 # name -> (restype, argtypes); mirrors include/wq.h
 _SIGS = {
     "wq_status_string": (ctypes.c_char_p, [_I]),
@@ -37,6 +47,7 @@ _SIGS = {
     "wq_act_quant": (_I, [_P, _I, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "wq_gemm_w4ax": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "wq_gemm_scratch_bytes": (ctypes.c_size_t, [_I, _I, _I]),
+    "wq_gemm_plan_query": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(GemmPlan)]),
     "wq_gemm_w4ax_ws": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P,
                              ctypes.c_size_t, _P]),
     "wq_linear_w4a8": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P,
@@ -223,6 +234,14 @@ def wq_gemm_w4ax(qx, s_tok, act_bits, K, stream_id, beta, S, T, step, qw, s_w, b
 
 def wq_gemm_scratch_bytes(M, K, N):
     return int(lib().wq_gemm_scratch_bytes(M, K, N))
+
+
+def wq_gemm_plan_query(M, K, N, act_bits=8, call="linear"):
+    """Which GEMM instance `call` ("gemm", "gemm_ws", "linear" or "gelu_quant") runs
+    for an (M, K, N) shape, as a dict of the wq_gemm_plan fields (no device work)."""
+    plan = GemmPlan()
+    _call("wq_gemm_plan_query", M, K, N, act_bits, PLAN_CALLS[call], ctypes.byref(plan))
+    return {n: getattr(plan, n) for n, _ in GemmPlan._fields_}
 
 
 def wq_gemm_w4ax_ws(qx, s_tok, act_bits, K, stream_id, beta, S, T, step, qw, s_w, bias, y,

@@ -78,11 +78,7 @@ Workspace carve(void* workspace, int M, int K, int N) {
   w.s_tok = reinterpret_cast<float*>(ws + off_stok);
   const size_t off_part = off_stok + round_up(sizeof(float) * static_cast<size_t>(M));
   if (wq::gemm_splits(M, N, K) > 1) {
-    const int BN = wq::bn_for(M);
-    const size_t tiles = static_cast<size_t>((M + BN - 1) / BN) * ((N + 127) / 128);
-    const size_t part_bytes = round_up(tiles * BN * 128 * sizeof(int32_t));
-    w.scratch.partial = reinterpret_cast<int32_t*>(ws + off_part);
-    w.scratch.counters = reinterpret_cast<int*>(ws + off_part + part_bytes);
+    w.scratch = wq::split_scratch_at(ws + off_part, M, N);
     w.zero = ws + off_part;
     w.zero_bytes = wq::gemm_split_scratch_bytes(M, N, K);
   }
@@ -312,6 +308,27 @@ size_t wq_gemm_scratch_bytes(int M, int K, int N) {
   return wq::gemm_split_scratch_bytes(M, N, K);
 }
 
+wq_status wq_gemm_plan_query(int M, int K, int N, int act_bits, int call, wq_gemm_plan* plan) {
+  if (!plan) return WQ_ERR_NULL;
+  *plan = wq_gemm_plan{};
+  if (call < WQ_PLAN_GEMM || call > WQ_PLAN_GELU_QUANT) return WQ_ERR_ARG;
+  const bool gemm_only = call == WQ_PLAN_GEMM || call == WQ_PLAN_GEMM_WS;
+  if (gemm_only && act_bits != 8 && act_bits != 4) return WQ_ERR_ARG;
+  WQ_TRY(check_mk(M, K));
+  WQ_TRY(check_n(N));
+  // the fused linears keep one code per int8 byte for both widths
+  const wq::GemmPlan g = wq::gemm_plan(M, N, K, gemm_only ? act_bits : 8, call != WQ_PLAN_GEMM,
+                                       call == WQ_PLAN_GELU_QUANT);
+  plan->tile_tokens = g.tile_tokens;
+  plan->tile_channels = g.tile_channels;
+  plan->ctas_per_tile = g.ctas_per_tile;
+  plan->k_splits = g.k_splits;
+  plan->k_stage = g.k_stage;
+  plan->tiles = g.tiles;
+  plan->weights_in_tmem = g.weights_in_tmem;
+  return WQ_OK;
+}
+
 wq_status wq_gemm_w4ax_ws(const void* qx, const float* s_tok, int act_bits, int M, int K, int N,
                           const uint8_t* stream_id, const float* beta, int S, int T, int step,
                           const uint8_t* qw, const float* s_w, const float* bias, wq_bf16* y,
@@ -326,11 +343,7 @@ wq_status wq_gemm_w4ax_ws(const void* qx, const float* s_tok, int act_bits, int 
     if (!workspace) return WQ_ERR_NULL;
     if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return WQ_ERR_ALIGN;
     if (ws_bytes < split_bytes) return WQ_ERR_ARG;
-    const int BN = wq::bn_for(M);
-    const size_t tiles = static_cast<size_t>((M + BN - 1) / BN) * ((N + 127) / 128);
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    sc.partial = reinterpret_cast<int32_t*>(ws);
-    sc.counters = reinterpret_cast<int*>(ws + round_up(tiles * BN * 128 * sizeof(int32_t)));
+    sc = wq::split_scratch_at(workspace, M, N);
     WQ_TRY(from_cuda(cudaMemsetAsync(workspace, 0, split_bytes, st)));
   }
   return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, y,
@@ -374,11 +387,7 @@ wq_status wq_debug_gemm_s32(const void* qx, int act_bits, const uint8_t* qw, int
     if (!workspace) return WQ_ERR_NULL;
     if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return WQ_ERR_ALIGN;
     if (ws_bytes < split_bytes) return WQ_ERR_ARG;
-    const int BN = wq::bn_for(M);
-    const size_t tiles = static_cast<size_t>((M + BN - 1) / BN) * ((N + 127) / 128);
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    sc.partial = reinterpret_cast<int32_t*>(ws);
-    sc.counters = reinterpret_cast<int*>(ws + round_up(tiles * BN * 128 * sizeof(int32_t)));
+    sc = wq::split_scratch_at(workspace, M, N);
     WQ_TRY(from_cuda(cudaMemsetAsync(workspace, 0, split_bytes, st)));
   }
   return from_cuda(wq::launch_gemm(qx, act_bits, qw, M, N, K, ep, nullptr,

@@ -1253,7 +1253,8 @@ cudaError_t run_gemm(const void* qx, const uint8_t* qw, int M, int N, int K,
 // of 224 tokens with the weights in TMEM (measured 4 % faster per step than 256-token
 // pairs with the weights in shared memory on the hidden-4096 block) where pair_bn
 // finds them no worse balanced, else 256; always 256 for the GELU-and-quantize
-// epilogue, whose twelve warps keep the shared-memory design.
+// epilogue, whose twelve warps keep the shared-memory design.  gemm_plan writes
+// these choices out for reporting; a change here changes it too.
 template <int ACT_BITS, int EPI = 0>
 cudaError_t dispatch_bn(const void* qx, const uint8_t* qw, int M, int N, int K,
                         const EpilogueArgs& ep, void* out, const SplitScratch* sc,
@@ -1340,14 +1341,53 @@ int gemm_splits(int M, int N, int K) {
   return s > 1 ? s : 1;
 }
 
-size_t gemm_split_scratch_bytes(int M, int N, int K) {
-  const int splits = gemm_splits(M, N, K);
-  if (splits == 1) return 0;
+// Output tiles of the single-CTA instances (128 channels each), and the split
+// scratch's two parts, each rounded up to 256 bytes.
+size_t split_tiles(int M, int N) {
   const int BN = bn_for(M);
-  const size_t tiles = static_cast<size_t>((M + BN - 1) / BN) * ((N + 127) / 128);
-  const size_t partial = tiles * BN * 128 * sizeof(int32_t);
-  const size_t counters = tiles * kMaxEpiWarps * sizeof(int);
-  return (partial + 255) / 256 * 256 + (counters + 255) / 256 * 256;
+  return static_cast<size_t>((M + BN - 1) / BN) * ((N + 127) / 128);
+}
+size_t split_partial_bytes(int M, int N) {
+  const size_t partial = split_tiles(M, N) * bn_for(M) * 128 * sizeof(int32_t);
+  return (partial + 255) / 256 * 256;
+}
+
+size_t gemm_split_scratch_bytes(int M, int N, int K) {
+  if (gemm_splits(M, N, K) == 1) return 0;
+  const size_t counters = split_tiles(M, N) * kMaxEpiWarps * sizeof(int);
+  return split_partial_bytes(M, N) + (counters + 255) / 256 * 256;
+}
+
+SplitScratch split_scratch_at(void* base, int M, int N) {
+  uint8_t* p = static_cast<uint8_t*>(base);
+  return SplitScratch{reinterpret_cast<int32_t*>(p),
+                      reinterpret_cast<int*>(p + split_partial_bytes(M, N))};
+}
+
+// The choices of dispatch_bn and run_gemm, written out.
+GemmPlan gemm_plan(int M, int N, int K, int act_bits, bool split_scratch, bool gelu_quant) {
+  GemmPlan p{};
+  if (M <= 0) return p;
+  const int BN = bn_for(M);
+  const int splits = split_scratch ? gemm_splits(M, N, K) : 1;
+  if (act_bits == 8 && BN == 256 && splits == 1) {  // CTA pairs
+    p.tile_tokens = gelu_quant ? 256 : pair_bn(M, N);
+    p.tile_channels = 256;
+    p.ctas_per_tile = 2;
+    p.k_splits = 1;
+    p.k_stage = 128;
+    p.weights_in_tmem = p.tile_tokens == 224 ? 1 : 0;
+  } else {
+    p.tile_tokens = BN;
+    p.tile_channels = 128;
+    p.ctas_per_tile = 1;
+    p.k_splits = splits;
+    p.k_stage = BN <= 64 && K % 256 == 0 ? 256 : 128;
+    p.weights_in_tmem = p.k_stage == 256 && !gelu_quant ? 1 : 0;
+  }
+  p.tiles = ((M + p.tile_tokens - 1) / p.tile_tokens) *
+            ((N + p.tile_channels - 1) / p.tile_channels);
+  return p;
 }
 
 cudaError_t launch_gemm(const void* qx, int act_bits, const uint8_t* qw, int M, int N, int K,

@@ -116,6 +116,27 @@ struct SplitScratch {
   int* counters;     // [tiles][kMaxEpiWarps], zero before the launch
 };
 
+// The split-K scratch of a shape whose K is split, laid out from base (256-byte
+// aligned): the partial tiles, then the counters, each part rounded up to 256 bytes;
+// gemm_split_scratch_bytes(M, N, K) bytes in all.
+SplitScratch split_scratch_at(void* base, int M, int N);
+
+// How the GEMM runs one shape: the rules launch_gemm and launch_gemm_gelu_quant
+// follow, for reporting (host arithmetic only; the SM count is the current
+// device's, 148 when none is visible).
+struct GemmPlan {
+  int tile_tokens;      // token tile (the MMA's N): 16, 32, 64, 128, 224 or 256
+  int tile_channels;    // output channels per tile: 128, or 256 on a CTA pair
+  int ctas_per_tile;    // 1, or 2 for a CTA pair (tcgen05 cta_group::2)
+  int k_splits;         // CTAs sharing one tile's K loop (1: K not split)
+  int k_stage;          // K depth of one pipeline stage: 128 or 256
+  int tiles;            // output tiles
+  int weights_in_tmem;  // 1 when the unpacked int8 weight tile is the MMA's A in TMEM
+};
+// split_scratch: the call passes a split-K scratch (the fused linears,
+// wq_gemm_w4ax_ws, the debug calls); gelu_quant: the GELU-and-quantize epilogue.
+GemmPlan gemm_plan(int M, int N, int K, int act_bits, bool split_scratch, bool gelu_quant);
+
 // Optional parts of a GEMM launch.
 struct GemmExtras {
   int32_t* acc_out = nullptr;  // int32 [M][N]: a copy of the accumulators (debug view)

@@ -142,6 +142,38 @@ wq_status wq_gemm_w4ax_ws(const void* qx, const float* s_tok, int act_bits, int 
                           const uint8_t* qw, const float* s_w, const float* bias, wq_bf16* y,
                           void* workspace, size_t ws_bytes, wq_stream_t stream);
 
+/* Which instance of the §4.4 GEMM a call runs for one shape (introspection: host
+ * arithmetic only, no device work; the SM count is the current device's, 148 when
+ * none is visible).  `call` names the entry point:
+ *   WQ_PLAN_GEMM        wq_gemm_w4ax (K is never split);
+ *   WQ_PLAN_GEMM_WS     wq_gemm_w4ax_ws and wq_debug_gemm_s32;
+ *   WQ_PLAN_LINEAR      wq_linear_w4a8 / _w4a4 / _w4ax_static / _w4a8_noalloc and
+ *                       wq_debug_linear_s32 (both widths keep one code per byte, so
+ *                       both run the int8-activation GEMM);
+ *   WQ_PLAN_GELU_QUANT  wq_linear_gelu_quant.
+ * act_bits (8 or 4) is the codes' format for WQ_PLAN_GEMM and WQ_PLAN_GEMM_WS and is
+ * ignored otherwise.  *plan is zeroed first, and stays zero for M == 0.  Returns
+ * WQ_ERR_NULL (plan NULL), WQ_ERR_ARG (call or act_bits), WQ_ERR_SHAPE (M, K, N as
+ * in wq_gemm_w4ax). */
+typedef struct wq_gemm_plan {
+  int tile_tokens;     /* token tile, the MMA's N: 16, 32, 64, 128, 224 or 256 */
+  int tile_channels;   /* output channels per tile: 128, or 256 on a CTA pair */
+  int ctas_per_tile;   /* 1, or 2 for a CTA pair (tcgen05 cta_group::2) */
+  int k_splits;        /* CTAs sharing one tile's K loop (1: K not split) */
+  int k_stage;         /* K depth of one pipeline stage: 128 or 256 */
+  int tiles;           /* output tiles of the launch */
+  int weights_in_tmem; /* 1: the unpacked int8 weight tile is the MMA's A operand in TMEM */
+} wq_gemm_plan;
+
+enum {
+  WQ_PLAN_GEMM = 0,
+  WQ_PLAN_GEMM_WS = 1,
+  WQ_PLAN_LINEAR = 2,
+  WQ_PLAN_GELU_QUANT = 3
+};
+
+wq_status wq_gemm_plan_query(int M, int K, int N, int act_bits, int call, wq_gemm_plan* plan);
+
 /* The fused W4A8 linear: wq_act_quant (8-bit) then wq_gemm_w4ax, with the codes
  * and token scales kept in the caller's workspace (device memory of at least
  * wq_workspace_bytes(M, K, N, 8) bytes, 256-byte aligned; its contents are

@@ -251,3 +251,85 @@ def test_noalloc_scratch_limit_is_exact(lib):
     assert wq.STATUS[lib.wq_linear_w4a8_noalloc(*args(4093))] == "WQ_ERR_SCRATCH"
     # 4092 passes the size check; without a GPU the next step (finding the device) fails
     assert wq.STATUS[lib.wq_linear_w4a8_noalloc(*args(4092))] != "WQ_ERR_SCRATCH"
+
+
+# ------------------------------------------------------------------ the GEMM's launch plan
+# wq_gemm_plan_query reports which GEMM instance a call runs for a shape (host
+# arithmetic only).  The hidden-4096 block takes 224-token CTA pairs for all four
+# linears; at 4288 tokens, 224-token tiles would give the busiest of the 74 pairs
+# more token columns on qkv, attn_out and mlp_down than 256-token tiles do.
+BLOCK4096 = [(8512, 4096, 12288), (8512, 4096, 4096), (8512, 4096, 16384), (8512, 16384, 4096)]
+BLOCK2048 = [(4288, 2048, 6144), (4288, 2048, 2048), (4288, 2048, 8192), (4288, 8192, 2048)]
+
+
+@pytest.mark.parametrize("M,K,N,tile", [(*s, 224) for s in BLOCK4096] +
+                         list(zip(*zip(*BLOCK2048), (256, 256, 224, 256))))
+def test_plan_of_the_configured_blocks(lib, M, K, N, tile):
+    p = wq.wq_gemm_plan_query(M, K, N)
+    assert (p["tile_tokens"], p["tile_channels"], p["ctas_per_tile"]) == (tile, 256, 2)
+    assert p["k_splits"] == 1 and p["k_stage"] == 128
+    assert p["weights_in_tmem"] == (tile == 224)
+    assert p["tiles"] == -(-M // tile) * (N // 256)
+    # the GELU-and-quantize epilogue keeps 256-token pairs with the weights in shared memory
+    g = wq.wq_gemm_plan_query(M, K, N, call="gelu_quant")
+    assert (g["tile_tokens"], g["ctas_per_tile"], g["weights_in_tmem"]) == (256, 2, 0)
+
+
+def _busiest(M, N, bn, pairs=74):
+    tiles = -(-N // 256) * -(-M // bn)
+    return -(-tiles // pairs) * bn
+
+
+@pytest.mark.parametrize("M", [129, 200, 256, 300, 513, 1000, 2048, 4288, 6000, 8512])
+@pytest.mark.parametrize("N", [256, 2048, 4096, 6144, 12288])
+def test_pair_width_balances_the_pairs(lib, M, N):
+    """Pair tiles take 224 tokens unless that leaves the busiest pair more token
+    columns than 256 does (whole tiles per pair; 148 SMs without a device)."""
+    p = wq.wq_gemm_plan_query(M, 4096, N, call="gemm")
+    assert p["ctas_per_tile"] == 2
+    want = 224 if _busiest(M, N, 224) <= _busiest(M, N, 256) else 256
+    assert p["tile_tokens"] == want
+
+
+@pytest.mark.parametrize("M", [1, 16, 33, 64, 100, 128, 256, 300])
+@pytest.mark.parametrize("K,N", [(2048, 512), (4096, 384), (8192, 2048), (16384, 4096),
+                                 (384, 256)])
+@pytest.mark.parametrize("act_bits", [8, 4])
+def test_plan_agrees_with_the_scratch_rule(lib, M, K, N, act_bits):
+    """K is split exactly when the call takes a scratch and wq_gemm_scratch_bytes is
+    not 0; split shapes and packed int4 codes run single CTAs; 256-deep stages only
+    for tiles of at most 64 tokens with K a multiple of 256."""
+    lib.wq_gemm_scratch_bytes.restype = ctypes.c_size_t
+    split = lib.wq_gemm_scratch_bytes(M, K, N) > 0
+    for call in ("gemm", "gemm_ws", "linear"):
+        bits = 8 if call == "linear" else act_bits
+        p = wq.wq_gemm_plan_query(M, K, N, act_bits, call)
+        assert (p["k_splits"] > 1) == (split and call != "gemm")
+        pair = p["ctas_per_tile"] == 2
+        assert pair == (bits == 8 and M > 128 and p["k_splits"] == 1)
+        assert p["tile_channels"] == (256 if pair else 128)
+        if not pair:
+            assert p["tile_tokens"] == next((b for b in (16, 32, 64, 128) if M <= b), 256)
+        assert p["k_stage"] == (256 if p["tile_tokens"] <= 64 and K % 256 == 0 else 128)
+        assert p["weights_in_tmem"] == (p["k_stage"] == 256 or p["tile_tokens"] == 224)
+        assert p["tiles"] == -(-M // p["tile_tokens"]) * -(-N // p["tile_channels"])
+
+
+def test_plan_rejects_on_host(lib):
+    plan = wq.GemmPlan()
+    q = lib.wq_gemm_plan_query
+    assert q(16, 4096, 512, 8, 0, None) == 1                      # no plan
+    assert q(16, 4096, 512, 8, 4, ctypes.byref(plan)) == 4        # unknown call
+    assert q(16, 4096, 512, 5, 0, ctypes.byref(plan)) == 4        # bad act_bits
+    assert q(16, 4096, 512, 5, 2, ctypes.byref(plan)) == 0        # ignored for the linears
+    assert q(16, 100, 512, 8, 2, ctypes.byref(plan)) == 2         # K not a multiple of 128
+    assert q(16, 4096, 8, 8, 2, ctypes.byref(plan)) == 2          # N below 16
+    plan.tiles = 7
+    assert q(0, 4096, 512, 8, 2, ctypes.byref(plan)) == 0 and plan.tiles == 0  # empty batch
+
+
+def test_plan_call_names_match_the_header():
+    src = open(os.path.join(ROOT, "include", "wq.h")).read()
+    enum = {m.group(1).lower(): int(m.group(2))
+            for m in re.finditer(r"\bWQ_PLAN_([A-Z_]+)\s*=\s*(\d+)", src)}
+    assert enum == wq.PLAN_CALLS

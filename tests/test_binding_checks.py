@@ -254,3 +254,17 @@ def test_library_status_is_raised(monkeypatch):
     monkeypatch.setattr(wq, "_current_device", lambda: 0)
     with pytest.raises(wq.WQError, match="WQ_ERR_SHAPE"):
         _linear(tensors())
+
+
+def test_plan_query_marshals_in_header_order(fake):
+    """wq_gemm_plan_query(M, K, N, act_bits, call, plan*): the call's name maps to
+    the header's enum, and an unknown name is refused before the library."""
+    plan = wq.wq_gemm_plan_query(300, 4096, 512, 4, "gemm_ws")
+    name, args = fake.calls[-1]
+    assert name == "wq_gemm_plan_query" and args[:5] == (300, 4096, 512, 4, 1)
+    assert set(plan) == {"tile_tokens", "tile_channels", "ctas_per_tile", "k_splits",
+                         "k_stage", "tiles", "weights_in_tmem"}
+    assert [wq.PLAN_CALLS[c] for c in ("gemm", "gemm_ws", "linear", "gelu_quant")] == [0, 1, 2, 3]
+    with pytest.raises(KeyError):
+        wq.wq_gemm_plan_query(300, 4096, 512, 8, "single")
+    assert len(fake.calls) == 1
