@@ -199,7 +199,7 @@ const char* wq_status_string(wq_status s) {
   return "unknown wq_status";
 }
 
-int wq_version(void) { return 100; }
+int wq_version(void) { return 101; }
 
 size_t wq_workspace_bytes(int M, int K, int N, int act_bits) {
   if ((act_bits != 8 && act_bits != 4) || check_mk(M, K) != WQ_OK || check_n(N) != WQ_OK)

@@ -79,7 +79,9 @@ typedef enum {
 /* Human-readable name of a status code (static string, never NULL). */
 const char* wq_status_string(wq_status s);
 
-/* ABI version of this library (major * 100 + minor). */
+/* ABI version of this library (major * 100 + minor; the minor number grows when
+ * entry points are added, the major one when an existing signature or contract
+ * changes).  101: adds wq_gemm_plan_query. */
 int wq_version(void);
 
 /* Bytes of device workspace wq_linear_w4a8 / wq_linear_w4a4 need for M token

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert wq.wq_version() == 100
+    assert wq.wq_version() == 101
     for code, name in wq.STATUS.items():
         assert lib.wq_status_string(code).decode().startswith(name)
 
