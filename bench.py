@@ -302,6 +302,17 @@ COMPANION = {"block4096_w4a8_t10": "block4096_w4a4_t10", "block2048_w4a8": "bloc
 NOMINAL_INT8_TOPS = 4500.0  # B200 dense int8, NVIDIA's figure without sparsity
 
 
+def gemm_instance(wq, M, K, N):
+    """The fused linear's GEMM instance for one shape, as the library's plan reports
+    it (host arithmetic only)."""
+    p = wq.wq_gemm_plan_query(M, K, N, call="linear")
+    kind = "a CTA pair" if p["ctas_per_tile"] == 2 else "one CTA"
+    tmem = ", int8 weights in TMEM" if p["weights_in_tmem"] else ""
+    split = f", K split {p['k_splits']} ways" if p["k_splits"] > 1 else ""
+    return (f"{p['tile_channels']} channels x {p['tile_tokens']} tokens on {kind}, "
+            f"{p['k_stage']}-deep stages{tmem}{split}")
+
+
 def _round256(n):
     return (n + 255) // 256 * 256
 
@@ -432,7 +443,8 @@ def measure_workload(args, wl, wq, torch, world, local, dev):
             "per_linear": [
                 {"linear": f"{L.name} {L.K}->{L.N}", "gemm_us": round(1e3 * t, 2),
                  "tops": round(L.ops() / (t * 1e-3) / 1e12, 1),
-                 "frac": round(L.ops() / (t * 1e-3) / 1e12 / peak, 4)}
+                 "frac": round(L.ops() / (t * 1e-3) / 1e12 / peak, 4),
+                 "tile": gemm_instance(wq, L.M, L.K, L.N)}
                 for L, t in zip(layers, per_layer_ms)],
             "measured": "event pair around a GEMM-only launch (the same kernel instance, on "
                         "the codes each fused call left in its workspace) after every fused "

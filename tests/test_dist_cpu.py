@@ -86,3 +86,18 @@ def test_gemm_traffic_ignores_host_side_edits(tmp_path, monkeypatch):
     assert bench.gemm_traffic("block2048_w4a8") == 77
     src.write_text(f"__global__ void k() {{ int x; }}\n{marker}\nint host_b();\n")  # device
     assert bench.gemm_traffic("block2048_w4a8") is None
+
+
+def test_bench_names_the_gemm_instance_of_each_linear():
+    """The bench line's per-linear entries name the GEMM instance from the library's
+    plan: 224-token pairs with the weights in TMEM on the hidden-4096 block, 256-token
+    pairs for its attention output projection at 4288 tokens, one CTA with 256-deep
+    stages at 16 tokens."""
+    import activation_quantized_gemm_wq_b200 as wq
+    assert bench.gemm_instance(wq, 8512, 4096, 16384) == (
+        "256 channels x 224 tokens on a CTA pair, 128-deep stages, int8 weights in TMEM")
+    assert bench.gemm_instance(wq, 4288, 2048, 2048) == (
+        "256 channels x 256 tokens on a CTA pair, 128-deep stages")
+    assert bench.gemm_instance(wq, 16, 16384, 4096) == (
+        "128 channels x 16 tokens on one CTA, 256-deep stages, int8 weights in TMEM, "
+        "K split 4 ways")
