@@ -711,18 +711,26 @@ def cpu_baseline(wl, budget_s=12.0, rows=None):
     from concurrent.futures import ThreadPoolExecutor
     cores = os.cpu_count() or 1
     blocks = [b for b in np.array_split(sel, cores) if len(b)]
+    per_linear = []
     t0 = time.perf_counter()
     with ThreadPoolExecutor(max_workers=len(blocks)) as pool:
-        for L, cinv, qw, s_w, x in prepared:
+        for lin, (L, cinv, qw, s_w, x) in zip(wl.linears, prepared):
+            t1 = time.perf_counter()
             list(pool.map(lambda b: orc.linear(x[b], cinv, sid_all[b], L.alpha, L.beta, 0,
                                                wl.act_bits, qw, s_w, L.bias), blocks))
+            dt_lin = time.perf_counter() - t1
+            # every row costs the same, so the full batch takes M / rows times as long
+            per_linear.append({"linear": f"{lin.name} {lin.K}->{lin.N}",
+                               "seconds_full_batch": round(dt_lin * wl.M / len(sel), 2),
+                               "tops": round(2 * len(sel) * lin.N * lin.K / dt_lin / 1e12, 6)})
     dt_mt = time.perf_counter() - t0
     return {"value": ops / dt_mt / 1e12, "unit": "TOPS", "cores": len(blocks), "kind": "oracle",
             "sample": f"oracle_linear on {len(sel)} of {wl.M} token rows of each of the "
                       f"{len(wl.linears)} linears ({ops / 1e9:.1f} G ops), rows split over "
                       f"{len(blocks)} host threads, {dt_mt:.1f} s",
             "seconds": round(dt_mt, 2),
-            "single_thread": {"value": ops / dt / 1e12, "cores": 1, "seconds": round(dt, 2)}}
+            "single_thread": {"value": ops / dt / 1e12, "cores": 1, "seconds": round(dt, 2)},
+            "per_linear": per_linear}
 
 
 def run_reference(args, rank, world):

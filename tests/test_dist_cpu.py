@@ -101,3 +101,15 @@ def test_bench_names_the_gemm_instance_of_each_linear():
     assert bench.gemm_instance(wq, 16, 16384, 4096) == (
         "128 channels x 16 tokens on one CTA, 256-deep stages, int8 weights in TMEM, "
         "K split 4 ways")
+
+
+def test_cpu_baseline_reports_each_linear():
+    """The oracle's timing on the host: the aggregate over the sample, the same sample
+    on one thread, and each linear's time extrapolated to the full token batch."""
+    from activation_quantized_gemm_wq_b200 import synth as S
+    r = bench.cpu_baseline(S.TINY, rows=4)
+    assert r["kind"] == "oracle" and r["unit"] == "TOPS" and r["value"] > 0
+    assert r["cores"] >= 1 and r["single_thread"]["cores"] == 1
+    assert [p["linear"] for p in r["per_linear"]] == [
+        f"{lin.name} {lin.K}->{lin.N}" for lin in S.TINY.linears]
+    assert all(p["seconds_full_batch"] >= 0 and p["tops"] > 0 for p in r["per_linear"])
