@@ -83,6 +83,43 @@ MUTANTS = [
      [("return v * 0.5 * erfc(-v / sqrt(2.0));", "return v * 0.5 * erf(v / sqrt(2.0));")]),
     ("GELU skipped before the bf16 rounding",
      [("h[i] = oracle_double_to_bf16(oracle_gelu(a));", "h[i] = oracle_double_to_bf16(a);")]),
+    ("no clamp at -qmax", [("if (r < -qmax) r = -qmax;", "")]),
+    ("zero scale divides by zero", [("if (s == 0.0f) return 0;", "")]),
+    ("activation scale divided by 2^(b-1) instead of qmax",
+     [("float clip = alpha[(size_t)step * S + sid] * amax;\n    float s = clip / qmax;",
+       "float clip = alpha[(size_t)step * S + sid] * amax;\n    float s = clip / (qmax + 1.0f);")]),
+    ("clip ratio of stream 0 for every row",
+     [("float clip = alpha[(size_t)step * S + sid] * amax;",
+       "float clip = alpha[(size_t)step * S] * amax;")]),
+    ("x' rounded to bf16 before quantization",
+     [("xp[k] = oracle_bf16_to_float(x[(size_t)m * K + k]) * ck;",
+       "xp[k] = oracle_bf16_to_float(oracle_double_to_bf16("
+       "oracle_bf16_to_float(x[(size_t)m * K + k]) * ck));")]),
+    ("static scale without the division by qmax",
+     [("float clip = g > 0.0f ? thr[step] / g : 0.0f;\n    float s = clip / qmax;",
+       "float clip = g > 0.0f ? thr[step] / g : 0.0f;\n    float s = clip;")]),
+    ("weight scale from the signed maximum",
+     [("      float a = fabsf(wp[k]);", "      float a = wp[k];")]),
+    ("GEMM drops the last k",
+     [("for (int k = 0; k < K; ++k) {\n        int w = unpack_nibble",
+       "for (int k = 0; k < K - 1; ++k) {\n        int w = unpack_nibble")]),
+    ("compensation of stream 0 for every row",
+     [("if (beta) v += (double)beta[((size_t)step * S + sid) * N + n];",
+       "if (beta) v += (double)beta[((size_t)step * S) * N + n];")]),
+    ("4-bit activation codes always from the low nibble",
+     [("  return unpack_nibble(b, k & 1);", "  return unpack_nibble(b, 0);")]),
+    ("bf16 rounding truncates", [("double r = nearbyint(ldexp(a, 8 - e));",
+                                 "double r = trunc(ldexp(a, 8 - e));")]),
+    ("channel scale without the square root",
+     [("if (a > 0.0f && b > 0.0f) ck = sqrtf(a / b);", "if (a > 0.0f && b > 0.0f) ck = a / b;")]),
+    ("cinv equal to c", [("cinv[k] = 1.0f / ck;", "cinv[k] = ck;")]),
+    ("scale as alpha * (amax / qmax)",
+     [("float clip = alpha[(size_t)step * S + sid] * amax;\n    float s = clip / qmax;",
+       "float clip = alpha[(size_t)step * S + sid] * amax;\n"
+       "    float s = alpha[(size_t)step * S + sid] * (amax / qmax);")]),
+    ("static: a non-positive gain keeps the threshold",
+     [("float clip = g > 0.0f ? thr[step] / g : 0.0f;",
+       "float clip = g > 0.0f ? thr[step] / g : thr[step];")]),
 ]
 
 
