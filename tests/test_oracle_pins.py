@@ -2,10 +2,13 @@
 the invariants of the method; plus planted mistakes that the pins must catch.
 
 Each planted mistake is a textual edit of a temporary copy of oracle/oracle.c,
-built on the CPU; the real oracle source is never modified.
+built on the CPU; the real oracle source is never modified.  Mistakes in the
+Python composition of the FFN step (up-projection, GELU, the next linear's codes)
+are planted by overriding that one method on a separate oracle instance.
 """
 import os
 import tempfile
+import types
 
 import pytest
 
@@ -145,3 +148,36 @@ def test_planted_mistake_is_caught(golden, mutant_dir, desc, edits):
     mutant = Oracle(oracle_pkg.load(so))
     fails = P.all_failures(mutant, golden)
     assert fails, f"planted mistake '{desc}' passed every pin"
+
+
+# Mistakes in composing the FFN step: each replaces Oracle.linear_gelu_quant_static
+# on one instance with a wrong composition of the oracle's own (correct) parts.
+def _codes_of_y(o, x, cinv, sid, alpha, beta, step, bits, qw, s_w, bias, cinv_n, thr_n,
+                gain_n, bits_n):
+    y = o.linear(x, cinv, sid, alpha, beta, step, bits, qw, s_w, bias)[0]
+    codes, s = o.act_quant_static(y, cinv_n, sid, thr_n, gain_n, step, bits_n)
+    return codes, s, o.gelu_bf16(y), y
+
+
+def _next_channel_scale_dropped(o, x, cinv, sid, alpha, beta, step, bits, qw, s_w, bias,
+                                cinv_n, thr_n, gain_n, bits_n):
+    y = o.linear(x, cinv, sid, alpha, beta, step, bits, qw, s_w, bias)[0]
+    h = o.gelu_bf16(y)
+    codes, s = o.act_quant_static(h, None, sid, thr_n, gain_n, step, bits_n)
+    return codes, s, h, y
+
+
+def _next_codes_4_bit(o, x, cinv, sid, alpha, beta, step, bits, qw, s_w, bias, cinv_n,
+                      thr_n, gain_n, bits_n):
+    y = o.linear(x, cinv, sid, alpha, beta, step, bits, qw, s_w, bias)[0]
+    h = o.gelu_bf16(y)
+    codes, s = o.act_quant_static(h, cinv_n, sid, thr_n, gain_n, step, 4)
+    return codes, s, h, y
+
+
+@pytest.mark.parametrize("wrong", [_codes_of_y, _next_channel_scale_dropped, _next_codes_4_bit],
+                         ids=lambda f: f.__name__.strip("_"))
+def test_planted_composition_mistake_is_caught(golden, wrong):
+    mutant = Oracle()
+    mutant.linear_gelu_quant_static = types.MethodType(wrong, mutant)
+    assert P.all_failures(mutant, golden), f"{wrong.__name__} passed every pin"
