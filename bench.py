@@ -118,13 +118,20 @@ def gemm_traffic(workload):
         return None
 
 
-def peaks():
+def peaks(path=None):
+    """(bf16 burst TFLOP/s, bf16 sustained TFLOP/s, HBM GB/s, source): the measured
+    figures when the peaks file holds them as positive numbers, else the fallback."""
+    def number(v):
+        if isinstance(v, bool) or not isinstance(v, (int, float)) or not v > 0 or v == float("inf"):
+            raise ValueError(f"not a positive number: {v!r}")
+        return float(v)
     try:
-        with open(PEAKS_FILE) as f:
+        with open(path or PEAKS_FILE) as f:
             d = json.load(f)
-        return d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), d["hbm_gbs"], \
-            "measured"
-    except (OSError, KeyError, ValueError):
+        burst = number(d["bf16_tflops"])
+        sustained = number(d.get("bf16_tflops_sustained", burst))
+        return burst, sustained, number(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError, TypeError, AttributeError):
         return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS_SUSTAINED, FALLBACK_HBM_GBS, "fallback"
 
 

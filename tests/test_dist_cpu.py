@@ -113,3 +113,19 @@ def test_cpu_baseline_reports_each_linear():
     assert [p["linear"] for p in r["per_linear"]] == [
         f"{lin.name} {lin.K}->{lin.N}" for lin in S.TINY.linears]
     assert all(p["seconds_full_batch"] >= 0 and p["tops"] > 0 for p in r["per_linear"])
+
+
+def test_peaks_file_is_read_only_when_it_holds_numbers(tmp_path):
+    f = tmp_path / "peaks.json"
+    f.write_text('{"hbm_gbs": 6550.5, "bf16_tflops": 1630, "bf16_tflops_sustained": 1410}')
+    assert bench.peaks(str(f)) == (1630.0, 1410.0, 6550.5, "measured")
+    f.write_text('{"hbm_gbs": 6550.5, "bf16_tflops": 1630}')   # no sustained figure
+    assert bench.peaks(str(f)) == (1630.0, 1630.0, 6550.5, "measured")
+    fallback = (bench.FALLBACK_BF16_TFLOPS, bench.FALLBACK_BF16_TFLOPS_SUSTAINED,
+                bench.FALLBACK_HBM_GBS, "fallback")
+    for bad in ('{"hbm_gbs": {"value": 6550}, "bf16_tflops": 1630}', '[1, 2, 3]', 'not json',
+                '{"hbm_gbs": 0, "bf16_tflops": 1630}', '{"bf16_tflops": 1630}',
+                '{"hbm_gbs": "6550", "bf16_tflops": 1630}'):
+        f.write_text(bad)
+        assert bench.peaks(str(f)) == fallback, bad
+    assert bench.peaks(str(tmp_path / "absent.json")) == fallback
