@@ -333,3 +333,21 @@ def test_plan_call_names_match_the_header():
     enum = {m.group(1).lower(): int(m.group(2))
             for m in re.finditer(r"\bWQ_PLAN_([A-Z_]+)\s*=\s*(\d+)", src)}
     assert enum == wq.PLAN_CALLS
+
+
+@pytest.mark.parametrize("lang,std", [("c", "-std=c99"), ("c++", "-std=c++17")])
+def test_header_is_plain_c(lang, std):
+    """include/wq.h is a C header (plain pointers, sizes and enums; no CUDA or torch
+    types): it compiles as strict C99 and as C++, with every warning an error."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    src = ('#include "wq.h"\n'
+           "int main(void) { wq_gemm_plan p; wq_stream_t s = 0; (void)s; p.tiles = 0;\n"
+           "  return p.tiles + (int)WQ_PLAN_LINEAR + (int)WQ_ERR_SCRATCH; }\n")
+    r = subprocess.run([cc, std, "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only",
+                        "-I", os.path.join(ROOT, "include"), "-x", lang, "-"],
+                       input=src, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
