@@ -29,6 +29,24 @@ KNOWN_UNTESTED = {
 }
 
 
+# One small shape per untested instance: (call, M, K, N, code bits of the GEMM call, or
+# the next linear's code width for gelu_quant); K % 256 == 128 selects the 128-deep
+# stages at <= 64 tokens, and 200 tokens with K = 16384 on 256 channels split K.
+SHAPE_FOR_UNTESTED = {
+    (4, 0, 32, 1, 128): ("gemm", 32, 384, 256, 4),
+    (8, 0, 32, 1, 128): ("gemm", 32, 384, 256, 8),
+}
+for _e in (8, 4):
+    SHAPE_FOR_UNTESTED.update({
+        (8, _e, 16, 1, 128): ("gelu_quant", 16, 384, 256, _e),
+        (8, _e, 32, 1, 128): ("gelu_quant", 32, 384, 256, _e),
+        (8, _e, 32, 1, 256): ("gelu_quant", 32, 512, 256, _e),
+        (8, _e, 64, 1, 128): ("gelu_quant", 64, 384, 256, _e),
+        (8, _e, 128, 1, 128): ("gelu_quant", 100, 512, 256, _e),
+        (8, _e, 256, 1, 128): ("gelu_quant", 200, 16384, 256, _e),
+    })
+
+
 def instance(M, K, N, bits, call, epi=0):
     """The instance `call` runs for (M, K, N), or None for an empty batch.  The fused
     calls keep one code per byte, so their mainloop takes int8 codes at either width."""
@@ -131,3 +149,13 @@ def test_both_pair_widths_and_the_split_path_are_covered():
     cov = covered()
     assert {(8, 0, 224, 2, 128), (8, 0, 256, 2, 128), (8, 0, 256, 1, 128),
             (8, 8, 256, 2, 128), (8, 4, 256, 2, 128)} <= cov
+
+
+def test_each_untested_instance_has_a_shape_that_reaches_it():
+    """The parity shapes to add next: each reaches its instance."""
+    assert set(SHAPE_FOR_UNTESTED) == KNOWN_UNTESTED
+    for inst, (call, M, K, N, bits) in SHAPE_FOR_UNTESTED.items():
+        if call == "gelu_quant":
+            assert instance(M, K, N, 8, call, bits) == inst
+        else:
+            assert instance(M, K, N, bits, call) == inst
